@@ -1,0 +1,410 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+The pages print no tensor values, so the oracle is pinned by closed forms,
+invariants, brute force on tiny inputs, an independent number-format library
+(ml_dtypes), an independent quantile routine (scipy), the pages' printed
+storage and parameter counts, and exact finite differences.
+"""
+import math
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import oracle as O
+from bit_nf4_quantized_20_b200 import inputs
+
+F32, F64 = np.float32, np.float64
+
+
+# --------------------------------------------------------------------------
+# eq. 2 codebook ("QLoRA: Efficient Fine-Tuning", Step 1)
+# --------------------------------------------------------------------------
+
+def test_codebook_shape_order_symmetry_ends():
+    q = O.nf4_codebook()
+    assert q.dtype == F32 and q.shape == (16,)
+    assert np.all(np.diff(q.astype(F64)) > 0)                # strictly increasing
+    assert q[0] == F32(-1.0) and q[15] == F32(1.0)            # normalised to [-1, 1]
+    assert np.array_equal(q.view(np.uint32), (-q[::-1]).view(np.uint32))  # exact symmetry
+    assert not np.any(q == 0)                                  # eq. 2 has no zero level
+
+
+def test_codebook_equal_probability_mass():
+    """Phi(q_i) - Phi(q_{i-1}) = 1/16: the levels sit at the centres of 16
+    equal-probability intervals (eq. 2, 'equal-probability intervals')."""
+    p = O.nf4_levels_eq2()
+    cdf = np.array([O.normal_cdf(v) for v in p])
+    assert np.allclose(cdf, (np.arange(1, 17) - 0.5) / 16, atol=1e-13, rtol=0)
+    assert np.allclose(np.diff(cdf), 1 / 16, atol=1e-13, rtol=0)
+
+
+def test_codebook_matches_scipy_ndtri():
+    p = O.nf4_levels_eq2()
+    ref = scipy.special.ndtri((np.arange(1, 17) - 0.5) / 16)
+    assert np.allclose(p, ref, atol=1e-13, rtol=0)
+    q = O.nf4_codebook()
+    assert np.allclose(q.astype(F64), np.concatenate([-ref[8:][::-1], ref[8:]]) / ref[15], atol=1e-7)
+
+
+def test_codebook_golden_fixture():
+    """Regression fixture written by tests/golden/make_golden.py (oracle only)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nf4_codebook_eq2.txt")
+    vals = []
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            vals.append(int(line.split()[0], 16))
+    assert np.array_equal(np.array(vals, dtype=np.uint32), O.nf4_codebook().view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# nearest-level snapping ("snapped to the nearest NF4 quantile level")
+# --------------------------------------------------------------------------
+
+def _brute_nearest(v: float, q: np.ndarray) -> int:
+    """argmin_j |v - q_j| in exact rational arithmetic, ties to the upper level."""
+    best, bestd = 0, None
+    fv = Fraction(float(v))
+    for j in range(16):
+        d = abs(fv - Fraction(float(q[j])))
+        if bestd is None or d <= bestd:   # '<=' walks upward, so ties resolve to the larger j
+            best, bestd = j, d
+    return best
+
+
+def test_thresholds_are_exact_midpoint_ceilings():
+    q = [Fraction(float(v)) for v in O.nf4_codebook()]
+    t = O.snap_thresholds(O.nf4_codebook())
+    for j in range(15):
+        tj = Fraction(float(t[j]))
+        below = Fraction(float(np.nextafter(t[j], F32(-np.inf))))
+        assert abs(tj - q[j + 1]) <= abs(tj - q[j])          # t_j snaps up
+        assert abs(below - q[j]) < abs(below - q[j + 1])     # the fp32 below it snaps down
+    assert t[7] == 0.0
+
+
+def test_snap_equals_brute_force_nearest():
+    q = O.nf4_codebook()
+    t = O.snap_thresholds(q)
+    rng = np.random.default_rng(7)
+    cand = list(rng.uniform(-1, 1, 3000).astype(F32))
+    for tj in t:                                   # every boundary and its fp32 neighbours
+        for k in range(-3, 4):
+            v = tj
+            step = F32(np.inf) if k > 0 else F32(-np.inf)
+            for _ in range(abs(k)):
+                v = np.nextafter(v, step)
+            cand.append(F32(v))
+    cand += [F32(0.0), F32(-0.0), F32(1.0), F32(-1.0), F32(1e-45), F32(-1e-45)]
+    cand += list(q) + [F32((float(q[j]) + float(q[j + 1])) / 2) for j in range(15)]
+    cand = np.array(cand, dtype=F32)
+    got = O.snap(cand, q)
+    want = np.array([_brute_nearest(v, q) for v in cand])
+    assert np.array_equal(got, want)
+    # signed zero: -0.0 reaches the zero threshold, like +0.0
+    assert O.snap(np.array([-0.0], F32), q)[0] == 8
+
+
+def test_normalise_is_ieee_fp32_division():
+    """RN32(w / c1) equals RN32(RN64(w / c1)): double rounding through binary64
+    is innocuous for division (53 >= 2*24 + 2), so Python's float division is an
+    independent check of the fp32 quotient."""
+    rng = np.random.default_rng(3)
+    w = inputs.bf16_bits(torch.from_numpy(rng.normal(0, 0.02, (4, 64)).astype(F32)).to(torch.bfloat16))
+    c1 = O.block_absmax(w)
+    got = O.normalise(w, c1)
+    wf = O.bf16_bits_to_f32(w).reshape(-1, 64)
+    for b in range(4):
+        assert c1[b] == max(abs(float(v)) for v in wf[b])          # eq. 1 absmax
+        for i in range(64):
+            assert got[b, i] == F32(float(wf[b, i]) / float(c1[b]))
+
+
+# --------------------------------------------------------------------------
+# number formats against an independent implementation (ml_dtypes)
+# --------------------------------------------------------------------------
+
+def _dense_f32_sweep(lo, hi, n, seed):
+    rng = np.random.default_rng(seed)
+    return rng.uniform(lo, hi, n).astype(F32)
+
+
+def test_bf16_rne_matches_ml_dtypes():
+    x = np.concatenate([
+        _dense_f32_sweep(-4, 4, 200000, 1),
+        _dense_f32_sweep(-1e-36, 1e-36, 20000, 2),
+        _dense_f32_sweep(-3e38, 3e38, 20000, 3),
+    ])
+    # exact ties: a bf16 value plus half a bf16 ulp
+    base = np.arange(0x3F80, 0x4080, dtype=np.uint32) << 16
+    ties = (base | 0x8000).view(F32)
+    x = np.concatenate([x, ties, -ties]).astype(F32)
+    got = O.f32_to_bf16_bits(x)
+    want = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(got, want)
+    tw = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, tw)
+
+
+def test_e4m3_decode_matches_ml_dtypes():
+    b = np.arange(256, dtype=np.uint8)
+    finite = ~(((b & 0x7F) == 0x7F))
+    got = O.e4m3_to_f32(b)
+    want = b.view(ml_dtypes.float8_e4m3fn).astype(F32)
+    assert np.array_equal(got[finite], want[finite])
+    assert np.all(np.isnan(got[~finite]))
+
+
+def test_e4m3_encode_matches_ml_dtypes_below_saturation():
+    allv = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(F64)
+    allv = np.unique(allv[np.isfinite(allv) & (allv >= 0)])
+    mids = (allv[:-1] + allv[1:]) / 2                                 # exact ties
+    near = np.concatenate([np.nextafter(mids.astype(F32), F32(0)), np.nextafter(mids.astype(F32), F32(1e9))])
+    x = np.concatenate([allv.astype(F32), mids.astype(F32), near,
+                        _dense_f32_sweep(0, 463.9, 300000, 4),
+                        _dense_f32_sweep(0, 0.02, 100000, 5)]).astype(F32)
+    x = x[x < 464.0]
+    got = O.f32_to_e4m3(x)
+    want = x.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.f32_to_e4m3(-x), want | 0x80)
+
+
+def test_e4m3_saturates_at_448():
+    x = np.array([464.0, 500.0, 1e6, 3e38], dtype=F32)
+    assert np.all(O.f32_to_e4m3(x) == 0x7E)
+    assert O.e4m3_to_f32(np.array([0x7E], np.uint8))[0] == 448.0
+
+
+# --------------------------------------------------------------------------
+# double quantization ("QLoRA & 4-bit Fine-Tuning", Innovation 2)
+# --------------------------------------------------------------------------
+
+def test_double_quantization_rule_and_error_bound():
+    rng = np.random.default_rng(11)
+    c1 = np.abs(rng.normal(0, 0.02, 1000)).astype(F32) + F32(0.01)
+    f, c2 = O.double_quantize(c1)
+    assert c2.shape == (4,)                                  # ceil(1000 / 256), last group short
+    for g in range(4):
+        part = c1[g * 256:(g + 1) * 256]
+        assert c2[g] == F32(float(part.max()) / 448.0)       # fp32 RN of max/448 (innocuous double rounding)
+        dec = O.e4m3_to_f32(f[g * 256:(g + 1) * 256]).astype(F64) * float(c2[g])
+        # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 in the normal range
+        assert np.all(np.abs(dec - part) <= 2.0 ** -4 * part + 1e-30)
+        assert f[g * 256 + int(np.argmax(part))] == 0x7E     # the group max maps to 448
+
+
+def test_double_quantization_zero_group():
+    f, c2 = O.double_quantize(np.zeros(300, F32))
+    assert np.all(f == 0) and np.all(c2 == 0)
+
+
+# --------------------------------------------------------------------------
+# quantize / dequantize as a whole
+# --------------------------------------------------------------------------
+
+def _w(rows, cols, seed, std=0.02):
+    return inputs.bf16_bits(inputs.normal_bf16((rows, cols), std, seed))
+
+
+def test_quantize_special_blocks():
+    w = np.zeros((1, 256), np.uint16)                # block 0: all zero (+0.0)
+    w[0, 64:128] = 0x8000                            # block 1: all -0.0
+    w[0, 128 + 5] = 0x3F80                           # block 2: one-hot +1.0
+    w[0, 192 + 9] = 0xBF80                           # block 3: one-hot -1.0
+    codes, scales, c2 = O.quantize_nf4(w)
+    c = O.unpack_codes(codes)
+    assert np.all(c[:128] == 8)                      # w_hat = 0 snaps to the level just above 0
+    assert c[128 + 5] == 15 and c[192 + 9] == 0
+    assert np.all(np.delete(c[128:], [5, 64 + 9]) == 8)
+    assert np.array_equal(scales, [0, 0, 0x7E, 0x7E])
+    assert c2[0] == F32(1.0 / 448.0)
+    wd = O.dequantize_nf4(codes, scales, c2, 1, 256)
+    assert np.all(wd[0, :128] == 0) and wd[0, 128 + 5] == 0x3F80 and wd[0, 192 + 9] == 0xBF80
+
+
+def test_dequant_error_bound():
+    """|w - w'| <= c1 * (largest half-gap of the codebook + E4M3 and BF16 rounding)."""
+    w = _w(64, 512, 5)
+    codes, scales, c2 = O.quantize_nf4(w)
+    wd = O.dequantize_nf4(codes, scales, c2, 64, 512)
+    q = O.nf4_codebook().astype(F64)
+    half_gap = np.max(np.diff(q)) / 2
+    err = np.abs(O.bf16_bits_to_f32(wd).astype(F64) - O.bf16_bits_to_f32(w).astype(F64)).reshape(-1, 64)
+    c1 = O.block_absmax(w).astype(F64)[:, None]
+    assert np.all(err <= c1 * (half_gap + 2.0 ** -4 * 1.07 + 2.0 ** -8 * 1.07))
+
+
+def test_quantize_codes_are_nearest_levels_brute_force():
+    w = _w(2, 128, 9)
+    codes, _, _ = O.quantize_nf4(w)
+    c = O.unpack_codes(codes).reshape(-1, 64)
+    wf = O.bf16_bits_to_f32(w).reshape(-1, 64)
+    q = O.nf4_codebook()
+    for b in range(wf.shape[0]):
+        m = max(abs(float(v)) for v in wf[b])
+        for i in range(64):
+            assert c[b, i] == _brute_nearest(F32(float(wf[b, i]) / m), q)
+
+
+def test_packing_low_nibble_is_even_element():
+    assert np.array_equal(O.pack_codes(np.array([1, 2, 15, 0], np.uint8)), [0x21, 0x0F])
+    assert np.array_equal(O.unpack_codes(np.array([0x21, 0x0F], np.uint8)), [1, 2, 15, 0])
+
+
+def test_quantize_dequantize_idempotent():
+    """Q(D(Q(W))) = Q(W) bit-exactly (codes, scale bytes, c2)."""
+    w = _w(512, 512, 42)
+    codes, scales, c2 = O.quantize_nf4(w)
+    wd = O.dequantize_nf4(codes, scales, c2, 512, 512)
+    codes2, scales2, c22 = O.quantize_nf4(wd)
+    assert np.array_equal(codes, codes2)
+    assert np.array_equal(scales, scales2)
+    assert np.array_equal(c2.view(np.uint32), c22.view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# storage and parameter counts printed on the pages
+# --------------------------------------------------------------------------
+
+LLAMA8B = [(n, k) for (_, n, k) in inputs.LLAMA8B_PROJ]
+
+
+def test_storage_overhead_0127_bits():
+    """'What is QLoRA?': 0.5 -> 0.127 bits of scale overhead, 4.127 bits/param."""
+    assert 32 / 64 == 0.5
+    assert O.bits_per_param() == 4.126953125
+    assert round(O.bits_per_param() - 4, 3) == 0.127
+    assert round(0.5 - (O.bits_per_param() - 4), 2) == 0.37          # "saving about 0.37 bits"
+
+
+def test_storage_llama8b_4_14_gb():
+    """8.03e9 x 4.127 / 8 = 4.14 GB for the Llama 3.1 8B worked example."""
+    assert round(8.03e9 * O.bits_per_param() / 8 / 1e9, 2) == 4.14
+    assert round(8.03e9 * 2 / 1e9, 2) == 16.06                       # BF16 figure on the same page
+
+
+def test_storage_32_layer_stack_exact():
+    total_w, total_b = 0, 0
+    for (n, k) in LLAMA8B:
+        total_w += n * k
+        total_b += sum(O.storage_bytes(n, k))
+    total_w *= 32
+    total_b *= 32
+    assert total_w == 6_979_321_856
+    assert total_b == 3_489_660_928 + 109_051_904 + 1_703_936 == 3_600_416_768
+    assert total_b * 8 / total_w == O.bits_per_param()
+
+
+def test_adapter_parameter_counts():
+    """1,310,720 rank-16 adapter parameters per 8B block ('What is QLoRA?')."""
+    per_block = O.lora_params(LLAMA8B, 16)
+    assert per_block == 1_310_720
+    assert round(per_block * 32 / 1e6, 1) == 41.9
+    assert round(per_block * 32 * 16 / 1e9, 2) == 0.67                # fp32 + grads + Adam
+    assert 4096 * 8 + 8 * 4096 == 65_536                              # rank-8 example, 4096 x 4096
+
+
+def test_eq4_ratio():
+    """eq. 4: r (m + n) / (m n) ~ r / min(m, n).  For 4096 x 4096 at r = 16 the
+    exact value is 0.78 %, twice the page's '< 0.4 %' (recorded as a page error)."""
+    assert O.lora_fraction(4096, 4096, 16) == 0.0078125
+    assert abs(O.lora_fraction(8192, 4096, 8) - 8 / 4096) / (8 / 4096) < 0.51
+
+
+# --------------------------------------------------------------------------
+# eq. 3 forward and eq. 5 backward
+# --------------------------------------------------------------------------
+
+def _bits(shape, std, seed):
+    return inputs.bf16_bits(inputs.normal_bf16(shape, std, seed))
+
+
+def test_forward_brute_force_eq3():
+    """h = W0 x + s B (A x) per token, as explicit scalar loops in the page's
+    notation (W0 in R^{m x n}, A in R^{r x n}, B in R^{m x r}); odd sizes so a
+    transposed operand cannot pass."""
+    T, m, n, r, s = 3, 5, 7, 2, 1.75
+    X, W, A, B = _bits((T, n), 1, 1), _bits((m, n), 0.1, 2), _bits((r, n), 0.3, 3), _bits((m, r), 0.2, 4)
+    Y = O.linear_fwd(X, W, A, B, s)
+    Xf, Wf, Af, Bf = (O.bf16_bits_to_f32(v).astype(F64) for v in (X, W, A, B))
+    for t in range(T):
+        ax = [sum(Af[i, j] * Xf[t, j] for j in range(n)) for i in range(r)]
+        for o in range(m):
+            h = sum(Wf[o, j] * Xf[t, j] for j in range(n)) + s * sum(Bf[o, i] * ax[i] for i in range(r))
+            assert abs(Y[t, o] - h) <= 1e-12 * (1 + abs(h))
+
+
+def test_forward_merged_weight_identity():
+    """W' = W + s B A (the merged form): X (W + s B A)^T equals eq. 3."""
+    T, m, n, r, s = 4, 6, 64, 3, 2.0
+    X, W, A, B = _bits((T, n), 1, 5), _bits((m, n), 0.02, 6), _bits((r, n), 0.1, 7), _bits((m, r), 0.05, 8)
+    Wm = O.bf16_bits_to_f32(W).astype(F64) + s * O.bf16_bits_to_f32(B).astype(F64) @ O.bf16_bits_to_f32(A).astype(F64)
+    ref = O.bf16_bits_to_f32(X).astype(F64) @ Wm.T
+    assert np.allclose(O.linear_fwd(X, W, A, B, s), ref, rtol=1e-12, atol=1e-12)
+    # s = 0 (or B = 0) leaves the frozen layer alone
+    zero = np.zeros_like(B)
+    assert np.allclose(O.linear_fwd(X, W, A, zero, s), O.linear_fwd(X, W, A, B, 0.0), rtol=0, atol=1e-14)
+
+
+def test_backward_eq5_per_token_outer_products():
+    """eq. 5: dL/dA = B^T g x^T and dL/dB = g (A x)^T per token (times s), summed."""
+    T, m, n, r, s = 3, 5, 7, 2, 0.5
+    X, W, A, B, dY = (_bits((T, n), 1, 11), _bits((m, n), 0.1, 12), _bits((r, n), 0.3, 13),
+                      _bits((m, r), 0.2, 14), _bits((T, m), 1, 15))
+    dX, dA, dB = O.linear_bwd(dY, X, W, A, B, s)
+    Xf, Wf, Af, Bf, G = (O.bf16_bits_to_f32(v).astype(F64) for v in (X, W, A, B, dY))
+    dA_ref = np.zeros((r, n))
+    dB_ref = np.zeros((m, r))
+    dX_ref = np.zeros((T, n))
+    for t in range(T):
+        g, x = G[t], Xf[t]
+        btg = [sum(Bf[o, i] * g[o] for o in range(m)) for i in range(r)]
+        ax = [sum(Af[i, j] * x[j] for j in range(n)) for i in range(r)]
+        for i in range(r):
+            for j in range(n):
+                dA_ref[i, j] += s * btg[i] * x[j]
+        for o in range(m):
+            for i in range(r):
+                dB_ref[o, i] += s * g[o] * ax[i]
+        for j in range(n):
+            dX_ref[t, j] = sum(g[o] * Wf[o, j] for o in range(m)) + s * sum(btg[i] * Af[i, j] for i in range(r))
+    assert np.allclose(dA, dA_ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dB, dB_ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dX, dX_ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("which", ["X", "A", "B"])
+def test_backward_is_the_derivative_of_the_forward(which):
+    """L = <dY, Y> is linear in each of X, A and B separately, so a central
+    difference is exact up to rounding: dL/dV . D = (L(V + eD) - L(V - eD)) / 2e."""
+    T, m, n, r, s = 6, 9, 64, 4, 2.0
+    X, W, A, B, dY = (_bits((T, n), 1, 21), _bits((m, n), 0.02, 22), _bits((r, n), 0.1, 23),
+                      _bits((m, r), 0.05, 24), _bits((T, m), 1, 25))
+    dX, dA, dB = O.linear_bwd(dY, X, W, A, B, s)
+    Xf, Wf, Af, Bf, G = (O.bf16_bits_to_f32(v).astype(F64) for v in (X, W, A, B, dY))
+
+    def L(Xv, Av, Bv):
+        Y = Xv @ Wf.T + s * (Xv @ Av.T) @ Bv.T
+        return float(np.sum(G * Y))
+
+    rng = np.random.default_rng(99)
+    e = 1e-3
+    if which == "X":
+        D = rng.normal(size=Xf.shape)
+        fd = (L(Xf + e * D, Af, Bf) - L(Xf - e * D, Af, Bf)) / (2 * e)
+        an = float(np.sum(dX * D))
+    elif which == "A":
+        D = rng.normal(size=Af.shape)
+        fd = (L(Xf, Af + e * D, Bf) - L(Xf, Af - e * D, Bf)) / (2 * e)
+        an = float(np.sum(dA * D))
+    else:
+        D = rng.normal(size=Bf.shape)
+        fd = (L(Xf, Af, Bf + e * D) - L(Xf, Af, Bf - e * D)) / (2 * e)
+        an = float(np.sum(dB * D))
+    assert abs(fd - an) <= 1e-8 * (1 + abs(an))
