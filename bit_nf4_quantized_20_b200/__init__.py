@@ -1,0 +1,188 @@
+"""QLoRA NF4 linear layer for B200 (sm_100a): Python entry points.
+
+PyTorch supplies device memory and the current CUDA stream; every computation
+runs in libqlora.so (include/qlora.h) through the ctypes binding in ``_lib``.
+There is no CPU or PyTorch fallback: if the library is missing, or a tensor is
+not on a CUDA device, the call raises.
+
+    qw = quantize_nf4(w)                     # w: [N, K] bf16 on cuda
+    y = linear_fwd(x, qw, A, B, s)           # x: [T, K], A: [r, K], B: [N, r]
+    dx, dA, dB = linear_bwd(dy, x, qw, A, B, s)
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import OP_BWD, OP_FWD, OP_QUANTIZE, NF4Weight, QLoraError, check, lib
+
+__all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "linear_fwd",
+           "linear_bwd", "workspace", "workspace_bytes", "get_error", "QLoraError", "lib"]
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> C.c_void_p:
+    return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def nf4_codebook() -> list[float]:
+    """The library's eq. 2 codebook (16 ascending fp32 levels in [-1, 1])."""
+    buf = (C.c_float * 16)()
+    check("qlora_nf4_codebook_eq2", lib().qlora_nf4_codebook_eq2(buf))
+    return [float(v) for v in buf]
+
+
+def storage_bytes(rows: int, cols: int, blocksize: int = 64, dq_block: int = 256):
+    """(codes, scales, c2) bytes of a quantized rows x cols weight."""
+    a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    check("qlora_nf4_storage_bytes",
+          lib().qlora_nf4_storage_bytes(rows, cols, blocksize, dq_block, C.byref(a), C.byref(b), C.byref(c)))
+    return a.value, b.value, c.value
+
+
+@dataclass
+class QuantizedNF4:
+    codes: torch.Tensor      # uint8 [rows*cols/2]
+    scales: torch.Tensor     # uint8 [rows*cols/64], FP8-E4M3FN bytes
+    c2: torch.Tensor         # float32 [ceil(rows*cols/16384)]
+    rows: int
+    cols: int
+    codebook: list
+    blocksize: int = 64
+    dq_block: int = 256
+
+    def struct(self) -> NF4Weight:
+        s = NF4Weight()
+        s.codes, s.scales, s.c2 = _ptr(self.codes), _ptr(self.scales), _ptr(self.c2)
+        s.rows, s.cols, s.blocksize, s.dq_block = self.rows, self.cols, self.blocksize, self.dq_block
+        for i, v in enumerate(self.codebook):
+            s.codebook[i] = v
+        return s
+
+    @property
+    def device(self):
+        return self.codes.device
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.scales.numel() + 4 * self.c2.numel()
+
+
+def workspace_bytes(op: int, T: int, N: int, K: int, r: int) -> int:
+    return int(lib().qlora_workspace_bytes(op, T, N, K, r))
+
+
+_WS: dict = {}
+
+
+def workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    """A zeroed, 256-byte aligned workspace of at least nbytes on `device` (cached, grows)."""
+    key = torch.device(device)
+    ws = _WS.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=key)
+        _WS[key] = ws
+    return ws
+
+
+def get_error(device=None) -> None:
+    """Synchronize and raise if a kernel recorded a device-side failure."""
+    dev = torch.device(device if device is not None else torch.cuda.current_device())
+    ws = _WS.get(dev)
+    if ws is None:
+        return
+    check("qlora_get_error", lib().qlora_get_error(C.c_void_p(ws.data_ptr()), _stream(dev)))
+
+
+def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: int = 256) -> QuantizedNF4:
+    """NF4 + double quantization of a BF16 weight w[rows, cols] on the GPU."""
+    _need_cuda("w", w)
+    if w.dim() != 2:
+        raise ValueError("w must be 2-D [rows, cols]")
+    rows, cols = w.shape
+    cb = list(nf4_codebook() if codebook is None else [float(v) for v in codebook])
+    if len(cb) != 16:
+        raise ValueError("codebook must have 16 entries")
+    nc, ns, n2 = storage_bytes(rows, cols, blocksize, dq_block)
+    dev = w.device
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+    scales = torch.empty(ns, dtype=torch.uint8, device=dev)
+    c2 = torch.empty(n2 // 4, dtype=torch.float32, device=dev)
+    out = NF4Weight()
+    out.codes, out.scales, out.c2 = codes.data_ptr(), scales.data_ptr(), c2.data_ptr()
+    cbuf = (C.c_float * 16)(*cb)
+    wsb = workspace_bytes(OP_QUANTIZE, 0, 0, 0, 1)
+    ws = workspace(dev, wsb)
+    check("qlora_quantize_nf4", lib().qlora_quantize_nf4(
+        C.c_void_p(w.data_ptr()), rows, cols, blocksize, dq_block, cbuf, C.byref(out),
+        C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
+    return QuantizedNF4(codes, scales, c2, rows, cols, cb, blocksize, dq_block)
+
+
+def dequantize(qw: QuantizedNF4) -> torch.Tensor:
+    out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.device)
+    s = qw.struct()
+    check("qlora_dequantize", lib().qlora_dequantize(C.byref(s), C.c_void_p(out.data_ptr()), _stream(qw.device)))
+    return out
+
+
+def _check_linear(x, qw, A, B):
+    for n, t in (("x", x), ("A", A), ("B", B)):
+        _need_cuda(n, t)
+    if x.dim() != 2 or x.shape[1] != qw.cols:
+        raise ValueError(f"x must be [T, {qw.cols}]")
+    r = A.shape[0]
+    if tuple(A.shape) != (r, qw.cols) or tuple(B.shape) != (qw.rows, r):
+        raise ValueError(f"A must be [r, {qw.cols}] and B [{qw.rows}, r]")
+    return x.shape[0], r
+
+
+def linear_fwd(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = x W'^T + s (x A^T) B^T (BF16), W' dequantized inside the kernel."""
+    T, r = _check_linear(x, qw, A, B)
+    dev = x.device
+    y = out if out is not None else torch.empty(T, qw.rows, dtype=torch.bfloat16, device=dev)
+    ws = workspace(dev, workspace_bytes(OP_FWD, T, qw.rows, qw.cols, r))
+    st = qw.struct()
+    check("qlora_linear_fwd", lib().qlora_linear_fwd(
+        C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()), C.c_void_p(B.data_ptr()), r,
+        float(s), C.c_void_p(y.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
+    return y
+
+
+def linear_bwd(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
+               outs=None):
+    """(dX, dA, dB) of the layer for upstream gradient dy[T, N]."""
+    T, r = _check_linear(x, qw, A, B)
+    _need_cuda("dy", dy)
+    if tuple(dy.shape) != (T, qw.rows):
+        raise ValueError(f"dy must be [{T}, {qw.rows}]")
+    dev = x.device
+    if outs is None:
+        dx = torch.empty(T, qw.cols, dtype=torch.bfloat16, device=dev)
+        dA = torch.empty(r, qw.cols, dtype=torch.bfloat16, device=dev)
+        dB = torch.empty(qw.rows, r, dtype=torch.bfloat16, device=dev)
+    else:
+        dx, dA, dB = outs
+    ws = workspace(dev, workspace_bytes(OP_BWD, T, qw.rows, qw.cols, r))
+    st = qw.struct()
+    check("qlora_linear_bwd", lib().qlora_linear_bwd(
+        C.c_void_p(dy.data_ptr()), C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()),
+        C.c_void_p(B.data_ptr()), r, float(s), C.c_void_p(dx.data_ptr()), C.c_void_p(dA.data_ptr()),
+        C.c_void_p(dB.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
+    return dx, dA, dB

@@ -1,0 +1,508 @@
+// api.cu -- the C ABI of the library (include/qlora.h): argument validation,
+// workspace layout, TMA descriptors and the launch sequence of each call.
+
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/qlora.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace qlora;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// trace hook
+// ---------------------------------------------------------------------------
+struct Trace {
+  qlora_trace_rec *recs = nullptr;
+  int32_t cap = 0;
+  int32_t *count = nullptr;
+};
+Trace g_trace;
+
+enum KernelId : int32_t {
+  K_QUANTIZE = 0,
+  K_DEQUANTIZE = 1,
+  K_LORA_U = 2,
+  K_LORA_DU = 3,
+  K_LORA_DB = 4,
+  K_LORA_DA = 5,
+  K_GEMM_FWD = 6,
+  K_GEMM_BWD = 7,
+  K_COUNT = 8,
+};
+
+const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",   "lora_du",
+                                     "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx"};
+
+struct TraceScope {
+  cudaStream_t st;
+  qlora_trace_rec *rec = nullptr;
+  TraceScope(int32_t kernel, double flops, double bytes, cudaStream_t s) : st(s) {
+    if (!g_trace.recs || !g_trace.count) return;
+    const int32_t i = (*g_trace.count)++;
+    if (i < g_trace.cap) {
+      rec = &g_trace.recs[i];
+      rec->kernel = kernel;
+      rec->flops = flops;
+      rec->bytes = bytes;
+      if (rec->start) cudaEventRecord(static_cast<cudaEvent_t>(rec->start), st);
+    }
+  }
+  ~TraceScope() {
+    if (rec && rec->stop) cudaEventRecord(static_cast<cudaEvent_t>(rec->stop), st);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// device properties
+// ---------------------------------------------------------------------------
+int num_sms_current() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Splits of the rank-r GEMMs are sized for a fixed CTA target so that the
+// workspace size does not depend on the device.
+constexpr int kSplitSms = 148;
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D BF16 row-major matrix [rows, cols] (row stride ld elements), box [box_rows, box_cols].
+bool make_map_bf16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows,
+                   int box_cols, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qlora_status check_codebook(const float *cb) {
+  for (int i = 0; i < 16; ++i)
+    if (!isfinite(cb[i])) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < 15; ++i)
+    if (!(cb[i] < cb[i + 1])) return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+// t_j = the smallest fp32 value >= (q_j + q_{j+1}) / 2 (midpoint formed in double):
+// a normalised weight reaching t_j is at least as close to q_{j+1} as to q_j.
+void snap_thresholds(const float *cb, float *thr) {
+  for (int j = 0; j < 15; ++j) {
+    const double mid = (static_cast<double>(cb[j]) + static_cast<double>(cb[j + 1])) * 0.5;
+    float t = static_cast<float>(mid);
+    if (static_cast<double>(t) < mid) t = nextafterf(t, INFINITY);
+    thr[j] = t;
+  }
+}
+
+qlora_status check_weight(const qlora_nf4_weight *qw) {
+  if (!qw || !qw->codes || !qw->scales || !qw->c2) return QLORA_ERR_INVALID_ARG;
+  if (qw->rows <= 0 || qw->cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (qw->blocksize != 64 || qw->dq_block != 256 || (qw->cols % 64) != 0) return QLORA_ERR_UNSUPPORTED;
+  if (!aligned16(qw->codes)) return QLORA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(qw->c2) & 3u) != 0) return QLORA_ERR_MISALIGNED;
+  return check_codebook(qw->codebook);
+}
+
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// ---------------------------------------------------------------------------
+// workspace layout
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  size_t counters = 0, su_hi = 0, su_lo = 0, du_hi = 0, du_lo = 0, partials = 0, total = 0;
+};
+
+WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
+  WsLayout L;
+  size_t off = kWsHeaderBytes;
+  L.counters = off;
+  off += kWsCounterBytes;
+  if (op == QLORA_OP_QUANTIZE) {
+    L.total = off;
+    return L;
+  }
+  const int64_t r64 = round_up(r, 64);
+  const size_t plane = static_cast<size_t>(round_up(T * r64 * 2, 256));
+  L.su_hi = off; off += plane;
+  L.su_lo = off; off += plane;
+  size_t part = skinny_partials_bytes(T, K, r, kSplitSms);
+  if (op == QLORA_OP_BWD) {
+    L.du_hi = off; off += plane;
+    L.du_lo = off; off += plane;
+    const size_t p2 = skinny_partials_bytes(T, N, r, kSplitSms);
+    const size_t p3 = skinny_partials_bytes(N, T, r, kSplitSms);
+    const size_t p4 = skinny_partials_bytes(K, T, r, kSplitSms);
+    if (p2 > part) part = p2;
+    if (p3 > part) part = p3;
+    if (p4 > part) part = p4;
+  }
+  L.partials = off;
+  off += static_cast<size_t>(round_up(static_cast<int64_t>(part), 256));
+  L.total = off;
+  return L;
+}
+
+SkinnyParams skinny_base(int64_t M, int64_t C, int R, uint8_t *ws, const WsLayout &L) {
+  SkinnyParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.C = C;
+  p.R = R;
+  p.splits = skinny_splits(M, C, kSplitSms);
+  int64_t per = (C + p.splits - 1) / p.splits;
+  p.c_per_split = round_up(per, 64);
+  p.partials = reinterpret_cast<float *>(ws + L.partials);
+  p.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+  p.status = reinterpret_cast<uint32_t *>(ws);
+  return p;
+}
+
+qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, const void *lact, int64_t r64,
+                      const void *lora, int r, void *out, int64_t T, uint32_t *status, cudaStream_t st) {
+  const int64_t N = qw->rows, K = qw->cols;
+  const int64_t Mside = mode == 0 ? N : K;     // weight-side extent
+  const int64_t Cext = mode == 0 ? K : N;      // contraction extent
+  CUtensorMap m_act, m_lact, m_out;
+  if (!make_map_bf16(&m_act, act, T, Cext, Cext, 256, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&m_lact, lact, T, r64, r64, 256, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&m_out, out, T, Mside, Mside, 32, 128, false)) return QLORA_ERR_CUDA;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.codes = qw->codes;
+  p.scales = qw->scales;
+  p.c2 = qw->c2;
+  for (int i = 0; i < 16; ++i) p.codebook[i] = qw->codebook[i];
+  p.N = N;
+  p.K = K;
+  p.T = T;
+  p.mode = mode;
+  p.lora = static_cast<const uint16_t *>(lora);
+  p.r = r;
+  p.m_tiles = static_cast<int>((Mside + 127) / 128);
+  p.n_tiles = static_cast<int>((T + 255) / 256);
+  p.k_main = static_cast<int>((Cext + 63) / 64);
+  p.k_lora = static_cast<int>(r64 / 64);
+  p.status = status;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(nf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes()) !=
+        cudaSuccess)
+      return QLORA_ERR_CUDA;
+    attr_set = true;
+  }
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int grid = static_cast<int>(tiles < num_sms_current() ? tiles : num_sms_current());
+  const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
+  const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
+  TraceScope ts(mode == 0 ? K_GEMM_FWD : K_GEMM_BWD, flops, bytes, st);
+  nf4_gemm_kernel<<<grid, 320, gemm_smem_bytes(), st>>>(m_act, m_lact, m_out, p);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status run_skinny(int32_t kid, const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st) {
+  const double flops = 2.0 * p.M * p.C * p.R * (p.Q1 ? 2 : 1);
+  const double bytes = 2.0 * p.M * p.C;
+  TraceScope ts(kid, flops, bytes, st);
+  return launch_skinny(p, p_col, q_cj, out_mode, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *qlora_status_string(qlora_status st) {
+  switch (st) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case QLORA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_NONFINITE: return "non-finite weight";
+    case QLORA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char *qlora_version(void) { return "1.0.0 sm_100a"; }
+
+qlora_status qlora_nf4_codebook_eq2(float out[16]) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  // Phi(x) = erfc(-x / sqrt 2) / 2; its inverse by bisection to full double precision.
+  auto phi = [](double x) { return 0.5 * erfc(-x / sqrt(2.0)); };
+  auto inv_phi = [&](double p) {
+    double lo = -12.0, hi = 12.0;
+    for (int i = 0; i < 200; ++i) {
+      const double mid = 0.5 * (lo + hi);
+      if (phi(mid) < p) lo = mid; else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+  };
+  double q[16];
+  for (int i = 1; i <= 16; ++i) q[i - 1] = inv_phi((i - 0.5) / 16.0);
+  // normalise by the largest level; the negative half mirrors the positive one
+  for (int i = 8; i < 16; ++i) {
+    const float v = static_cast<float>(q[i] / q[15]);
+    out[i] = v;
+    out[15 - i] = -v;
+  }
+  return QLORA_OK;
+}
+
+qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, int32_t blocksize, int32_t dq_block,
+                                     size_t *codes_bytes, size_t *scales_bytes, size_t *c2_bytes) {
+  if (!codes_bytes || !scales_bytes || !c2_bytes) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (blocksize != 64 || dq_block != 256 || cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
+  const int64_t n = rows * cols;
+  const int64_t blocks = n / 64;
+  *codes_bytes = static_cast<size_t>(n / 2);
+  *scales_bytes = static_cast<size_t>(blocks);
+  *c2_bytes = static_cast<size_t>((blocks + 255) / 256) * 4;
+  return QLORA_OK;
+}
+
+size_t qlora_workspace_bytes(int32_t op, int64_t T, int64_t N, int64_t K, int32_t r) {
+  if (op == QLORA_OP_QUANTIZE) return ws_layout(op, 0, 0, 0, 1).total;
+  if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || T < 0 || N <= 0 || K <= 0 || r < 1 || r > 128) return 0;
+  return ws_layout(op, T, N, K, r).total;
+}
+
+qlora_status qlora_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!ws || ws_bytes < kWsHeaderBytes) return QLORA_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? QLORA_OK
+                                                                                              : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_get_error(void *ws, void *stream) {
+  if (!ws) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+  if (word & DEV_TIMEOUT) return QLORA_ERR_TIMEOUT;
+  if (word & DEV_NONFINITE) return QLORA_ERR_NONFINITE;
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
+                                int32_t dq_block, const float codebook[16], qlora_nf4_weight *out, void *ws,
+                                size_t ws_bytes, void *stream) {
+  if (!w_bf16 || !codebook || !out || !out->codes || !out->scales || !out->c2) return QLORA_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (blocksize != 64 || dq_block != 256 || cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (!aligned16(w_bf16) || !aligned16(out->codes) || (reinterpret_cast<uintptr_t>(out->c2) & 3u))
+    return QLORA_ERR_MISALIGNED;
+  qlora_status cs = check_codebook(codebook);
+  if (cs != QLORA_OK) return cs;
+  if (!ws || ws_bytes < qlora_workspace_bytes(QLORA_OP_QUANTIZE, 0, 0, 0, 1)) return QLORA_ERR_WORKSPACE;
+  out->rows = rows;
+  out->cols = cols;
+  out->blocksize = blocksize;
+  out->dq_block = dq_block;
+  SnapTable tab;
+  for (int i = 0; i < 16; ++i) {
+    tab.codebook[i] = codebook[i];
+    out->codebook[i] = codebook[i];
+  }
+  snap_thresholds(codebook, tab.thr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t nblocks = rows * cols / 64;
+  const double n = static_cast<double>(rows) * cols;
+  TraceScope ts(K_QUANTIZE, 0.0, n * 2.0 + n * (0.5 + 1.0 / 64) + 4.0 * ((nblocks + 255) / 256), st);
+  cudaError_t e = launch_quantize(static_cast<const uint16_t *>(w_bf16), nblocks, out->codes, out->scales, out->c2,
+                                  tab, static_cast<uint32_t *>(ws), st, num_sms_current());
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight *qw, void *w_bf16_out, void *stream) {
+  qlora_status s = check_weight(qw);
+  if (s != QLORA_OK) return s;
+  if (!w_bf16_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16_out)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const double n = static_cast<double>(qw->rows) * qw->cols;
+  TraceScope ts(K_DEQUANTIZE, 0.0, n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + n * 2.0, st);
+  cudaError_t e = launch_dequantize(qw->codes, qw->scales, qw->c2, qw->rows * qw->cols, qw->codebook,
+                                    static_cast<uint16_t *>(w_bf16_out), st, num_sms_current());
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+static qlora_status check_linear(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                                 const void *B, int32_t r, float s) {
+  qlora_status st = check_weight(qw);
+  if (st != QLORA_OK) return st;
+  if (!x || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (T < 0 || r < 1 || r > 128 || !isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (qw->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (T > 0x7fffffff || qw->rows > 0x7fffffff || qw->cols > 0x7fffffff) return QLORA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A, const void *B,
+                              int32_t r, float s, void *y, void *ws, size_t ws_bytes, void *stream) {
+  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
+  if (cs != QLORA_OK) return cs;
+  if (!y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(y)) return QLORA_ERR_MISALIGNED;
+  const int64_t N = qw->rows, K = qw->cols;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_FWD, T, N, K, r))
+    return QLORA_ERR_WORKSPACE;
+  if (T == 0) return QLORA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  const WsLayout L = ws_layout(QLORA_OP_FWD, T, N, K, r);
+  const int64_t r64 = round_up(r, 64);
+  uint16_t *su_hi = reinterpret_cast<uint16_t *>(w8 + L.su_hi);
+  // U' = s X A^T (hi plane only: the forward reads it as the rank-r MMA operand)
+  SkinnyParams pu = skinny_base(T, K, r, w8, L);
+  pu.P = static_cast<const uint16_t *>(x);
+  pu.ldp = K;
+  pu.Q0 = static_cast<const uint16_t *>(A);
+  pu.ldq = K;
+  pu.alpha = s;
+  pu.out0 = su_hi;
+  pu.out1 = nullptr;
+  pu.ldo = r64;
+  qlora_status rs = run_skinny(K_LORA_U, pu, false, false, OUT_HILO, st);
+  if (rs != QLORA_OK) return rs;
+  return run_gemm(0, qw, x, su_hi, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), st);
+}
+
+qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                              const void *B, int32_t r, float s, void *dx, void *dA, void *dB, void *ws,
+                              size_t ws_bytes, void *stream) {
+  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
+  if (cs != QLORA_OK) return cs;
+  if (!dy || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(dx) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
+  const int64_t N = qw->rows, K = qw->cols;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    // no tokens: the adapter gradients are empty sums
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  const WsLayout L = ws_layout(QLORA_OP_BWD, T, N, K, r);
+  const int64_t r64 = round_up(r, 64);
+  uint16_t *su_hi = reinterpret_cast<uint16_t *>(w8 + L.su_hi);
+  uint16_t *su_lo = reinterpret_cast<uint16_t *>(w8 + L.su_lo);
+  uint16_t *du_hi = reinterpret_cast<uint16_t *>(w8 + L.du_hi);
+  uint16_t *du_lo = reinterpret_cast<uint16_t *>(w8 + L.du_lo);
+  // sU = s X A^T, as hi + lo planes
+  SkinnyParams pu = skinny_base(T, K, r, w8, L);
+  pu.P = static_cast<const uint16_t *>(x);
+  pu.ldp = K;
+  pu.Q0 = static_cast<const uint16_t *>(A);
+  pu.ldq = K;
+  pu.alpha = s;
+  pu.out0 = su_hi;
+  pu.out1 = su_lo;
+  pu.ldo = r64;
+  qlora_status rs = run_skinny(K_LORA_U, pu, false, false, OUT_HILO, st);
+  if (rs != QLORA_OK) return rs;
+  // dU = s dY B, as hi + lo planes
+  SkinnyParams pd = skinny_base(T, N, r, w8, L);
+  pd.P = static_cast<const uint16_t *>(dy);
+  pd.ldp = N;
+  pd.Q0 = static_cast<const uint16_t *>(B);
+  pd.ldq = r;
+  pd.alpha = s;
+  pd.out0 = du_hi;
+  pd.out1 = du_lo;
+  pd.ldo = r64;
+  rs = run_skinny(K_LORA_DU, pd, false, true, OUT_HILO, st);
+  if (rs != QLORA_OK) return rs;
+  // dX = dY W' + dU A
+  rs = run_gemm(1, qw, dy, du_hi, r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
+  if (rs != QLORA_OK) return rs;
+  // dB = dY^T (sU)
+  SkinnyParams pb = skinny_base(N, T, r, w8, L);
+  pb.P = static_cast<const uint16_t *>(dy);
+  pb.ldp = N;
+  pb.Q0 = su_hi;
+  pb.Q1 = su_lo;
+  pb.ldq = r64;
+  pb.alpha = 1.0f;
+  pb.out0 = static_cast<uint16_t *>(dB);
+  rs = run_skinny(K_LORA_DB, pb, true, true, OUT_ROW, st);
+  if (rs != QLORA_OK) return rs;
+  // dA = dU^T X
+  SkinnyParams pa = skinny_base(K, T, r, w8, L);
+  pa.P = static_cast<const uint16_t *>(x);
+  pa.ldp = K;
+  pa.Q0 = du_hi;
+  pa.Q1 = du_lo;
+  pa.ldq = r64;
+  pa.alpha = 1.0f;
+  pa.out0 = static_cast<uint16_t *>(dA);
+  return run_skinny(K_LORA_DA, pa, true, true, OUT_T, st);
+}
+
+qlora_status qlora_trace_attach(qlora_trace_rec *recs, int32_t capacity, int32_t *count) {
+  if (recs && (!count || capacity < 0)) return QLORA_ERR_INVALID_ARG;
+  g_trace.recs = recs;
+  g_trace.cap = recs ? capacity : 0;
+  g_trace.count = recs ? count : nullptr;
+  return QLORA_OK;
+}
+
+const char *qlora_kernel_name(int32_t kernel) {
+  if (kernel < 0 || kernel >= K_COUNT) return "unknown";
+  return kKernelNames[kernel];
+}
+
+}  // extern "C"

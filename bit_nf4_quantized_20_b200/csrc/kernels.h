@@ -1,0 +1,82 @@
+// kernels.h -- parameter blocks and launch helpers shared between the C-ABI
+// layer (api.cu) and the kernels.  Internal to the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qlora {
+
+// Codebook and its snapping thresholds, passed by value to the quantizer.
+struct SnapTable {
+  float codebook[16];
+  float thr[15];   // t_j = smallest fp32 >= (q_j + q_{j+1}) / 2
+};
+
+// ---------------------------------------------------------------------------
+// quantize / dequantize (quant.cu)
+// ---------------------------------------------------------------------------
+cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
+                            const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms);
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t n_weights,
+                              const float (&codebook)[16], uint16_t *out, cudaStream_t st, int num_sms);
+
+// ---------------------------------------------------------------------------
+// fused NF4 GEMM (gemm_nf4.cu)
+// ---------------------------------------------------------------------------
+struct GemmParams {
+  const uint8_t *codes;
+  const uint8_t *scales;
+  const float *c2;
+  float codebook[16];
+  int64_t N, K;            // quantized weight is N x K
+  int64_t T;               // tokens
+  int mode;                // 0: forward (M side = N rows), 1: backward dX (M side = K columns)
+  const uint16_t *lora;    // forward: B[N, r]; backward: A[r, K]
+  int r;
+  int m_tiles, n_tiles;    // weight-side tiles of 128, token tiles of 256
+  int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part
+  uint32_t *status;
+};
+int gemm_smem_bytes();
+__global__ void nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                                const __grid_constant__ CUtensorMap tmap_lact,
+                                const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
+
+// ---------------------------------------------------------------------------
+// rank-r LoRA GEMMs on the legacy tensor path (skinny.cu)
+//   C[M, R] = alpha * sum_c P(m, c) * Q(c, j),  Q = Q0 (+ Q1)
+// ---------------------------------------------------------------------------
+enum SkinnyOut : int {
+  OUT_HILO = 0,      // two BF16 planes [M, ldo]: hi = bf16(v), lo = bf16(v - hi); cols R..ldo zero
+  OUT_ROW = 1,       // BF16 [M, R] row-major
+  OUT_T = 2,         // BF16 [R, M] (transposed) row-major
+};
+
+struct SkinnyParams {
+  const uint16_t *P;   // BF16
+  int64_t ldp;
+  const uint16_t *Q0;  // BF16
+  const uint16_t *Q1;  // optional second plane (nullptr if none)
+  int64_t ldq;
+  int64_t M, C;        // rows, contraction length
+  int R;               // output columns (<= 128)
+  int splits;          // contraction splits
+  int64_t c_per_split; // multiple of 64
+  float alpha;
+  uint16_t *out0;      // OUT_HILO: hi plane; else output
+  uint16_t *out1;      // OUT_HILO: lo plane
+  int64_t ldo;         // OUT_HILO: plane row stride (>= R); unused otherwise
+  float *partials;     // [splits][M][RP] when splits > 1
+  uint32_t *counters;  // one per 64-row tile when splits > 1 (zero on entry, zero on exit)
+  uint32_t *status;
+};
+
+// p_col: P stored as [c][m] (else [m][c]); q_cj: Q stored as [c][j] (else [j][c]).
+cudaError_t launch_skinny(const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st);
+// Split count and partial-buffer bytes the launcher will use for (M, C).
+int skinny_splits(int64_t M, int64_t C, int num_sms);
+size_t skinny_partials_bytes(int64_t M, int64_t C, int R, int num_sms);
+
+}  // namespace qlora

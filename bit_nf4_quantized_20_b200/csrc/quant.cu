@@ -1,0 +1,168 @@
+// quant.cu -- NF4 quantization with double quantization, and dequantization.
+//
+// Quantize ("QLoRA: Efficient Fine-Tuning", Step 1 eq. 1 and eq. 2, Step 2;
+// "QLoRA & 4-bit Fine-Tuning", Innovation 2):
+//   c1_b   = max |w| over block b of 64 consecutive weights (eq. 1, alpha = 1)
+//   w_hat  = RN32(w / c1_b)                       (0 for an all-zero block)
+//   code   = #{ j : w_hat >= t_j }                (nearest level, ties up)
+//   c2_g   = RN32(max_{b in g} c1_b / 448)        (g = 256 consecutive blocks)
+//   f_b    = E4M3_RNE_satfinite(RN32(c1_b / c2_g))  (0 when c2_g == 0)
+// Dequantize:  W' = BF16_RNE(RN32(codebook[code] * RN32(fp8(f_b) * c2_g)))
+//
+// One CTA quantizes one double-quantization group (256 blocks = 16,384
+// weights): 8 lanes share a block, each loading 8 BF16 weights with one
+// 128-bit load; the block absmax is an integer max of |bits| reduced with
+// three xor-shuffles; the group max is a CTA reduction.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int QT = 256;
+
+// Number of thresholds t_j <= x, by a branch-free binary search: the first
+// two levels select between register-held thresholds, the last two read the
+// table in shared memory.
+__device__ __forceinline__ uint32_t snap_code(float x, float t3, float t7, float t11, const float *s_thr) {
+  uint32_t c = (x >= t7) ? 8u : 0u;
+  const float th = c ? t11 : t3;
+  c += (x >= th) ? 4u : 0u;
+  c += (x >= s_thr[c + 1]) ? 2u : 0u;
+  c += (x >= s_thr[c]) ? 1u : 0u;
+  return c;
+}
+
+__global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ w, int64_t n_blocks,
+                                                      uint32_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                      float *__restrict__ c2, const SnapTable tab,
+                                                      uint32_t *status) {
+  __shared__ float s_thr[16];
+  __shared__ float s_wmax[QT / 32];
+  if (threadIdx.x < 15) s_thr[threadIdx.x] = tab.thr[threadIdx.x];
+
+  const int64_t g = blockIdx.x;
+  const int64_t b0 = g * 256;
+  const int nb = static_cast<int>(min(static_cast<int64_t>(256), n_blocks - b0));
+  const int tid = threadIdx.x;
+  const int sub = tid & 7;    // which 8 weights of the block
+  const int bw = tid >> 3;    // block within a slab of 32 blocks
+
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bl = i * 32 + bw;
+    if (bl < nb) {
+      v[i] = __ldg(w + (b0 + bl) * 8 + sub);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  // block absmax as an integer max over |bits| (BF16 order = magnitude order)
+  float c1[8];
+  uint32_t bad = 0;
+  float tmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t a = v[i].x & 0x7FFF7FFFu, b = v[i].y & 0x7FFF7FFFu, c = v[i].z & 0x7FFF7FFFu,
+                   d = v[i].w & 0x7FFF7FFFu;
+    uint32_t m = max(max(max(a & 0xFFFFu, a >> 16), max(b & 0xFFFFu, b >> 16)),
+                     max(max(c & 0xFFFFu, c >> 16), max(d & 0xFFFFu, d >> 16)));
+    bad |= (m >= 0x7F80u) ? 1u : 0u;
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    c1[i] = __uint_as_float(m << 16);
+    tmax = fmaxf(tmax, c1[i]);
+  }
+#pragma unroll
+  for (int o = 8; o < 32; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+  if ((tid & 31) == 0) s_wmax[tid >> 5] = tmax;
+  __syncthreads();
+  float gmax = s_wmax[0];
+#pragma unroll
+  for (int i = 1; i < QT / 32; ++i) gmax = fmaxf(gmax, s_wmax[i]);
+
+  const float c2v = __fdiv_rn(gmax, 448.0f);
+  if (tid == 0) c2[g] = c2v;
+
+  const float t3 = s_thr[3], t7 = s_thr[7], t11 = s_thr[11];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bl = i * 32 + bw;
+    if (bl < nb) {
+      if (sub == 0) scales[b0 + bl] = static_cast<uint8_t>(c2v > 0.f ? float_to_e4m3(__fdiv_rn(c1[i], c2v)) : 0u);
+      const uint32_t hw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t word = 0;
+      const bool nz = c1[i] > 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t bits = (e & 1) ? (hw[e >> 1] & 0xFFFF0000u) : (hw[e >> 1] << 16);
+        const float x = nz ? __fdiv_rn(__uint_as_float(bits), c1[i]) : 0.f;
+        word |= snap_code(x, t3, t7, t11, s_thr) << (4 * e);
+      }
+      codes[(b0 + bl) * 8 + sub] = word;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) set_status(status, DEV_NONFINITE);
+}
+
+__global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ codes,
+                                                      const uint8_t *__restrict__ scales,
+                                                      const float *__restrict__ c2, int64_t n_units,
+                                                      const SnapTable tab, uint4 *__restrict__ out) {
+  __shared__ float s_cb[16];
+  if (threadIdx.x < 16) s_cb[threadIdx.x] = tab.codebook[threadIdx.x];
+  __syncthreads();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_units; i += stride) {
+    const uint2 c = __ldg(codes + i);       // 16 codes
+    const int64_t blk = i >> 2;             // 4 units of 16 weights per block
+    const float s = __fmul_rn(e4m3_to_float(__ldg(scales + blk)), __ldg(c2 + (blk >> 8)));
+    const uint32_t words[2] = {c.x, c.y};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t o[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float lo = s_cb[(words[h] >> (8 * p)) & 15u];
+        const float hi = s_cb[(words[h] >> (8 * p + 4)) & 15u];
+        o[p] = pack_bf16x2(__fmul_rn(lo, s), __fmul_rn(hi, s));
+      }
+      out[2 * i + h] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
+                            const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms) {
+  (void)num_sms;
+  const int64_t groups = (n_blocks + 255) / 256;
+  if (groups <= 0) return cudaSuccess;
+  quantize_kernel<<<static_cast<unsigned>(groups), QT, 0, st>>>(reinterpret_cast<const uint4 *>(w), n_blocks,
+                                                                 reinterpret_cast<uint32_t *>(codes), scales, c2,
+                                                                 tab, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t n_weights,
+                              const float (&codebook)[16], uint16_t *out, cudaStream_t st, int num_sms) {
+  const int64_t n_units = n_weights / 16;
+  if (n_units <= 0) return cudaSuccess;
+  SnapTable tab;
+  for (int i = 0; i < 16; ++i) tab.codebook[i] = codebook[i];
+  for (int i = 0; i < 15; ++i) tab.thr[i] = 0.f;
+  int64_t blocks = (n_units + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(reinterpret_cast<const uint2 *>(codes), scales,
+                                                                 c2, n_units, tab, reinterpret_cast<uint4 *>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

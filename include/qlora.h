@@ -1,0 +1,208 @@
+/*
+ * qlora.h -- C ABI of the B200 (sm_100a) QLoRA NF4 linear-layer library.
+ *
+ * The layer: a frozen weight W0[N, K] (out x in) stored as 4-bit NormalFloat
+ * codes with one absmax scale per 64 weights, the scales themselves stored as
+ * FP8-E4M3 with one FP32 second-level scale per 256 scales, plus a BF16 LoRA
+ * adapter A[r, K], B[N, r] with scaling s = lora_alpha / r.
+ *
+ * Sources (web pages on QLoRA, cited by title and section/equation):
+ *   "QLoRA: Efficient Fine-Tuning" (fermi.ai wiki): Step 1 eq. 1 (block absmax
+ *     normalisation, alpha = 1), eq. 2 (NF4 levels q_i = Phi^-1((i-1/2)/16)),
+ *     "snapped to the nearest NF4 quantile level"; Step 2 (double
+ *     quantization, 8-bit floats, block 256); Step 3 eq. 3 (h = W0 x + B A x,
+ *     W0 dequantized to BF16 at runtime; PEFT snippet: scaled by alpha / r);
+ *     Step 4 eq. 5 (adapter gradients).
+ *   "What is QLoRA?" (aquanode.io), "The three pieces": block of 64, scale
+ *     overhead 0.127 bits/param, BF16 conversion on the fly for each matmul.
+ *   "QLoRA & 4-bit Fine-Tuning" (prepfeed), Innovation 2: W ~ c1 * W_NF4, c1
+ *     quantized from FP32 to FP8 with a second scale c2; follow-up 1:
+ *     dequantization on the fly in every forward and backward pass.
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
+ *     never allocates, frees or keeps device memory between calls, apart from
+ *     small __constant__ tables that each call overwrites.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).  Work
+ *     is enqueued on it and the call returns after validating the arguments;
+ *     results are ready when the stream reaches that point.
+ *   - Row-major layouts.  BF16 tensors are arrays of uint16 bit patterns.
+ *   - A call that returns anything but QLORA_OK has enqueued nothing.
+ *   - Device-side failures (a bounded wait that ran out, a non-finite weight)
+ *     are recorded in the workspace's status word and read by qlora_get_error.
+ *   - Not thread-safe with respect to the trace hook; otherwise re-entrant.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad codebook */
+  QLORA_ERR_UNSUPPORTED = 2,   /* blocksize != 64, dq_block != 256, shape outside v1 limits */
+  QLORA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+  QLORA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_CUDA = 5,          /* a CUDA runtime/driver call or launch failed */
+  QLORA_ERR_NONFINITE = 6,     /* quantize saw an Inf/NaN weight (outputs undefined) */
+  QLORA_ERR_TIMEOUT = 7        /* a kernel's bounded wait ran out; it stopped early */
+} qlora_status;
+
+typedef enum {
+  QLORA_OP_QUANTIZE = 0,
+  QLORA_OP_FWD = 1,
+  QLORA_OP_BWD = 2
+} qlora_op;
+
+/*
+ * A quantized weight (all buffers on the device, caller-owned).
+ *   codes   uint8[rows*cols/2]: flat row-major order, two codes per byte, the
+ *           even element in the low nibble; code j selects codebook[j].
+ *   scales  uint8[rows*cols/64]: one OCP FP8-E4M3FN byte per block of 64
+ *           consecutive weights of a row (needs cols % 64 == 0).
+ *   c2      float[ceil(rows*cols/(64*256))]: one FP32 second-level scale per
+ *           256 consecutive blocks in flat order (the last group may be short).
+ *   codebook  the 16 ascending FP32 levels the codes index (by value).
+ * Dequantized weight: s_b = RN32(fp8(scales[b]) * c2[b/256]);
+ *                     W'  = BF16_RNE(RN32(codebook[code] * s_b)).
+ */
+typedef struct {
+  uint8_t *codes;
+  uint8_t *scales;
+  float *c2;
+  int64_t rows;        /* N: output features */
+  int64_t cols;        /* K: input features, a multiple of blocksize */
+  int32_t blocksize;   /* 64 */
+  int32_t dq_block;    /* 256 */
+  float codebook[16];
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static string; never NULL). */
+QLORA_API const char *qlora_status_string(qlora_status st);
+
+/* Library version string, e.g. "1.0.0 sm_100a". */
+QLORA_API const char *qlora_version(void);
+
+/*
+ * The 16 NF4 levels of eq. 2 ("QLoRA: Efficient Fine-Tuning", Step 1):
+ * q_i = Phi^-1((i - 1/2)/16), i = 1..16, divided by q_16 so that they span
+ * [-1, 1] like eq. 1's normalised weights, rounded to FP32, ascending.
+ * Host-only; writes out[0..15].  The library accepts any strictly ascending,
+ * finite 16-entry table; this is the default one.
+ */
+QLORA_API qlora_status qlora_nf4_codebook_eq2(float out[16]);
+
+/*
+ * Bytes of each buffer of a quantized rows x cols weight ("What is QLoRA?",
+ * "The three pieces": 4 bits + 8/64 + 32/(64*256) = 4.127 bits per weight).
+ * Host-only.  Errors: INVALID_ARG (null output, rows/cols <= 0),
+ * UNSUPPORTED (blocksize != 64, dq_block != 256, cols % 64 != 0).
+ */
+QLORA_API qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, int32_t blocksize, int32_t dq_block,
+                                     size_t *codes_bytes, size_t *scales_bytes, size_t *c2_bytes);
+
+/*
+ * Workspace bytes that `op` needs for T tokens, an N x K weight and rank r.
+ * Host-only; 0 on invalid arguments.  The workspace is caller-owned device
+ * memory, 256-byte aligned, that must be zeroed once (qlora_workspace_init)
+ * before its first use; every call leaves its counters zero again.  Calls that
+ * share a workspace must be ordered on one stream.
+ */
+QLORA_API size_t qlora_workspace_bytes(int32_t op, int64_t T, int64_t N, int64_t K, int32_t r);
+
+/* Zero a workspace (one cudaMemsetAsync on `stream`). */
+QLORA_API qlora_status qlora_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronize `stream`, read and clear the workspace status word.
+ * Returns QLORA_OK, QLORA_ERR_NONFINITE, QLORA_ERR_TIMEOUT or QLORA_ERR_CUDA.
+ */
+QLORA_API qlora_status qlora_get_error(void *ws, void *stream);
+
+/*
+ * Quantize a BF16 weight w[rows, cols] to NF4 with double quantization.
+ *   eq. 1 (alpha = 1): c1_b = max |w| over block b (64 consecutive weights);
+ *   w_hat = RN32(w / c1_b) (IEEE fp32 division; 0 for an all-zero block);
+ *   code = number of thresholds t_j <= w_hat, t_j = the smallest fp32 that is
+ *     >= (codebook[j] + codebook[j+1]) / 2 -- i.e. the nearest level, ties up;
+ *   double quantization (Step 2; prepfeed Innovation 2): per 256 blocks
+ *     c2 = RN32(max c1 / 448), scale byte = E4M3_RNE_satfinite(RN32(c1 / c2))
+ *     (0 when c2 == 0).
+ * `out` supplies the three device buffers (sizes from qlora_nf4_storage_bytes);
+ * the call fills out->rows/cols/blocksize/dq_block/codebook.
+ * ws: at least qlora_workspace_bytes(QLORA_OP_QUANTIZE, ...) bytes (status word).
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED (w, codes not 16-byte aligned),
+ * WORKSPACE, CUDA.  A non-finite weight is reported later by qlora_get_error.
+ */
+QLORA_API qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
+                                int32_t dq_block, const float codebook[16], qlora_nf4_weight *out,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Dequantize to BF16: w_out[rows, cols] = W' as defined above ("What is
+ * QLoRA?": NF4 converted to BF16 on the fly; prepfeed: W ~ c1 * W_NF4).
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+QLORA_API qlora_status qlora_dequantize(const qlora_nf4_weight *qw, void *w_bf16_out, void *stream);
+
+/*
+ * Forward, eq. 3 with the PEFT scaling (Step 3):
+ *   y[T, N] = x[T, K] W'^T + s (x A^T) B^T, BF16 out, FP32 accumulation,
+ *   W' dequantized inside the matmul and never written to memory.
+ * x[T, K], A[r, K], B[N, r], y[T, N]: BF16, row-major, 16-byte aligned.
+ * Requires N % 8 == 0, 1 <= r <= 128; T == 0 is a no-op.
+ * ws: at least qlora_workspace_bytes(QLORA_OP_FWD, T, N, K, r) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                              const void *B, int32_t r, float s, void *y, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/*
+ * Backward (Step 4 eq. 5, and the gradient through the frozen weight):
+ *   dU = s dY B;  dX = dY W' + dU A;  dB = s dY^T (x A^T);  dA = dU^T x.
+ * dy[T, N], x[T, K], A[r, K], B[N, r]; outputs dx[T, K], dA[r, K], dB[N, r]
+ * (BF16, overwritten, not accumulated).  Same requirements as the forward.
+ * ws: at least qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
+                              const void *A, const void *B, int32_t r, float s, void *dx, void *dA,
+                              void *dB, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Launch trace (profiling hook).  While attached, every kernel the library
+ * launches records recs[i].start before and recs[i].stop after it on the
+ * call's stream (cudaEvent_t handles the caller created), and fills kernel id,
+ * units and the algorithmic work of that launch.  *count counts the launches;
+ * launches beyond `capacity` are counted but not recorded.  Pass recs = NULL
+ * to detach.  Process-wide; not thread-safe.
+ */
+typedef struct {
+  int32_t kernel;      /* qlora_kernel_name(kernel) names it */
+  int32_t pad_;
+  void *start;         /* cudaEvent_t, caller-created */
+  void *stop;          /* cudaEvent_t, caller-created */
+  double flops;        /* algorithmic FLOPs of this launch (0 if bandwidth-bound) */
+  double bytes;        /* algorithmic DRAM bytes of this launch */
+} qlora_trace_rec;
+
+QLORA_API qlora_status qlora_trace_attach(qlora_trace_rec *recs, int32_t capacity, int32_t *count);
+QLORA_API const char *qlora_kernel_name(int32_t kernel);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

@@ -1,0 +1,171 @@
+"""The C-ABI library builds, loads and exports every symbol include/qlora.h
+declares; host-only entry points and argument validation behave as documented.
+No test here launches a kernel (it runs without a GPU)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_nf4_quantized_20_b200 import build
+    build.build()
+    from bit_nf4_quantized_20_b200 import _lib
+    return _lib.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API[^;(]*?\b(qlora_\w+)\s*\(", text, flags=re.S)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for need in ["qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+                 "qlora_nf4_storage_bytes", "qlora_workspace_bytes", "qlora_get_error", "qlora_status_string"]:
+        assert need in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    from bit_nf4_quantized_20_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (qlora_\w+)", out))
+    for s in declared_symbols():
+        assert s in exported, s
+        assert hasattr(L, s)
+    # nothing else leaks out under the qlora_ prefix
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings_and_version(L):
+    for code in range(8):
+        assert L.qlora_status_string(code)
+    assert b"sm_100a" in L.qlora_version()
+
+
+def test_library_codebook_equals_oracle_codebook(L):
+    """The library's own eq. 2 levels (bisection on erfc) match the oracle's
+    (statistics.NormalDist) bit for bit."""
+    buf = (C.c_float * 16)()
+    assert L.qlora_nf4_codebook_eq2(buf) == 0
+    got = np.array(list(buf), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), O.nf4_codebook().view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols", [(512, 512), (4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336),
+                                       (3, 320), (22016, 8192)])
+def test_storage_bytes_match_oracle(L, rows, cols):
+    a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    assert L.qlora_nf4_storage_bytes(rows, cols, 64, 256, C.byref(a), C.byref(b), C.byref(c)) == 0
+    assert (a.value, b.value, c.value) == O.storage_bytes(rows, cols)
+
+
+def test_storage_bytes_rejects(L):
+    a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    assert L.qlora_nf4_storage_bytes(4, 100, 64, 256, C.byref(a), C.byref(b), C.byref(c)) == 2
+    assert L.qlora_nf4_storage_bytes(4, 128, 32, 256, C.byref(a), C.byref(b), C.byref(c)) == 2
+    assert L.qlora_nf4_storage_bytes(4, 128, 64, 128, C.byref(a), C.byref(b), C.byref(c)) == 2
+    assert L.qlora_nf4_storage_bytes(0, 128, 64, 256, C.byref(a), C.byref(b), C.byref(c)) == 1
+    assert L.qlora_nf4_storage_bytes(4, 128, 64, 256, None, C.byref(b), C.byref(c)) == 1
+
+
+def test_workspace_bytes(L):
+    q = L.qlora_workspace_bytes(0, 0, 0, 0, 1)
+    f = L.qlora_workspace_bytes(1, 4096, 4096, 4096, 16)
+    b = L.qlora_workspace_bytes(2, 4096, 4096, 4096, 16)
+    assert 256 <= q < f < b
+    assert L.qlora_workspace_bytes(1, 4096, 4096, 4096, 0) == 0
+    assert L.qlora_workspace_bytes(1, 4096, 4096, 4096, 129) == 0
+    assert L.qlora_workspace_bytes(7, 16, 16, 64, 8) == 0
+    # grows with the token count
+    assert L.qlora_workspace_bytes(2, 8192, 4096, 4096, 16) > b
+
+
+def _weight(rows=128, cols=128, codes=0x1000, scales=0x2000, c2=0x3000, bs=64, dq=256):
+    from bit_nf4_quantized_20_b200._lib import NF4Weight
+    w = NF4Weight()
+    w.codes, w.scales, w.c2 = codes, scales, c2
+    w.rows, w.cols, w.blocksize, w.dq_block = rows, cols, bs, dq
+    for i, v in enumerate(O.nf4_codebook()):
+        w.codebook[i] = float(v)
+    return w
+
+
+FAKE = 0x10000   # never dereferenced: every call below fails validation first
+
+
+def test_quantize_validation(L):
+    from bit_nf4_quantized_20_b200._lib import NF4Weight
+    cb = (C.c_float * 16)(*[float(v) for v in O.nf4_codebook()])
+    out = _weight()
+    ws, wsb = C.c_void_p(FAKE), 1 << 20
+    q = L.qlora_quantize_nf4
+    assert q(None, 128, 128, 64, 256, cb, C.byref(out), ws, wsb, None) == 1            # null input
+    assert q(C.c_void_p(FAKE), 128, 100, 64, 256, cb, C.byref(out), ws, wsb, None) == 2  # cols % 64
+    assert q(C.c_void_p(FAKE), 128, 128, 32, 256, cb, C.byref(out), ws, wsb, None) == 2  # blocksize
+    assert q(C.c_void_p(FAKE + 2), 128, 128, 64, 256, cb, C.byref(out), ws, wsb, None) == 3  # misaligned
+    bad = (C.c_float * 16)(*([0.0] * 16))
+    assert q(C.c_void_p(FAKE), 128, 128, 64, 256, bad, C.byref(out), ws, wsb, None) == 1   # not ascending
+    nan = (C.c_float * 16)(*[float("nan")] + [float(v) for v in O.nf4_codebook()[1:]])
+    assert q(C.c_void_p(FAKE), 128, 128, 64, 256, nan, C.byref(out), ws, wsb, None) == 1
+    assert q(C.c_void_p(FAKE), 128, 128, 64, 256, cb, C.byref(out), None, wsb, None) == 4  # no workspace
+    assert q(C.c_void_p(FAKE), 128, 128, 64, 256, cb, C.byref(out), ws, 16, None) == 4     # too small
+    empty = NF4Weight()
+    assert q(C.c_void_p(FAKE), 128, 128, 64, 256, cb, C.byref(empty), ws, wsb, None) == 1  # no out buffers
+
+
+def test_linear_validation(L):
+    w = _weight()
+    ws = C.c_void_p(FAKE)
+    big = 1 << 30
+    fwd = L.qlora_linear_fwd
+    P = C.c_void_p(FAKE)
+    assert fwd(None, 16, C.byref(w), P, P, 8, 2.0, P, ws, big, None) == 1
+    assert fwd(P, 16, C.byref(w), P, P, 0, 2.0, P, ws, big, None) == 1       # r = 0
+    assert fwd(P, 16, C.byref(w), P, P, 129, 2.0, P, ws, big, None) == 1     # r > 128
+    assert fwd(P, 16, C.byref(w), P, P, 8, float("inf"), P, ws, big, None) == 1
+    assert fwd(P, -1, C.byref(w), P, P, 8, 2.0, P, ws, big, None) == 1
+    assert fwd(C.c_void_p(FAKE + 8), 16, C.byref(w), P, P, 8, 2.0, P, ws, big, None) == 3
+    assert fwd(P, 16, C.byref(w), P, P, 8, 2.0, P, C.c_void_p(FAKE + 16), big, None) == 4  # ws not 256-aligned
+    assert fwd(P, 16, C.byref(w), P, P, 8, 2.0, P, ws, 1024, None) == 4
+    odd = _weight(rows=100)
+    assert fwd(P, 16, C.byref(odd), P, P, 8, 2.0, P, ws, big, None) == 2     # N % 8
+    bs = _weight(bs=128)
+    assert fwd(P, 16, C.byref(bs), P, P, 8, 2.0, P, ws, big, None) == 2
+    mis = _weight(codes=FAKE + 4)
+    assert fwd(P, 16, C.byref(mis), P, P, 8, 2.0, P, ws, big, None) == 3
+    bwd = L.qlora_linear_bwd
+    assert bwd(P, P, 16, C.byref(w), P, P, 8, 2.0, P, None, P, ws, big, None) == 1
+    assert bwd(P, P, 16, C.byref(w), P, P, 8, 2.0, P, P, C.c_void_p(FAKE + 2), ws, big, None) == 3
+    assert bwd(P, P, 16, C.byref(w), P, P, 8, 2.0, P, P, P, ws, 64, None) == 4
+    deq = L.qlora_dequantize
+    assert deq(C.byref(w), None, None) == 1
+    assert deq(C.byref(w), C.c_void_p(FAKE + 1), None) == 3
+
+
+def test_trace_attach_validation(L):
+    from bit_nf4_quantized_20_b200._lib import TraceRec
+    recs = (TraceRec * 4)()
+    assert L.qlora_trace_attach(recs, 4, None) == 1
+    cnt = C.c_int32(0)
+    assert L.qlora_trace_attach(recs, 4, C.byref(cnt)) == 0
+    assert L.qlora_trace_attach(None, 0, None) == 0
+    assert L.qlora_kernel_name(6) == b"nf4_gemm_fwd"
+    assert L.qlora_kernel_name(99) == b"unknown"
+
+
+def test_product_fails_loudly_without_cuda():
+    """No CPU fallback: the Python entry points refuse CPU tensors."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    with pytest.raises(ValueError):
+        q.quantize_nf4(torch.zeros(64, 64, dtype=torch.bfloat16))

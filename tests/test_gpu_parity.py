@@ -1,0 +1,218 @@
+"""GPU path vs the CPU oracle, through the C ABI (ctypes binding).
+
+Bit-exact for quantize (codes, FP8 scale bytes, c2) and dequantize; within
+|gpu - oracle| <= 5e-3 + 1e-2 |oracle| per element for the forward and
+backward (oracle in float64 from the same BF16 inputs and the BF16
+dequantized weight).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from bit_nf4_quantized_20_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_ABS, TOL_REL = 5e-3, 1e-2
+
+
+def Q():
+    import bit_nf4_quantized_20_b200 as q
+    return q
+
+
+def bits(t):
+    return inputs.bf16_bits(t)
+
+
+def from_bits(b):
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16)
+
+
+def assert_close(name, gpu_bf16, ref64):
+    g = O.bf16_bits_to_f32(bits(gpu_bf16)).astype(np.float64).reshape(ref64.shape)
+    err = np.abs(g - ref64)
+    tol = TOL_ABS + TOL_REL * np.abs(ref64)
+    bad = err > tol
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - tol), err.shape)
+        raise AssertionError(f"{name}: {bad.sum()} of {bad.size} outside tolerance; worst at {i}: "
+                             f"gpu={g[i]!r} oracle={ref64[i]!r}")
+
+
+def quantize_and_check(w_dev):
+    q = Q()
+    qw = q.quantize_nf4(w_dev)
+    torch.cuda.synchronize()
+    codes, scales, c2 = O.quantize_nf4(bits(w_dev))
+    g_codes = qw.codes.cpu().numpy()
+    g_scales = qw.scales.cpu().numpy()
+    g_c2 = qw.c2.cpu().numpy()
+    assert np.array_equal(g_c2.view(np.uint32), c2.view(np.uint32)), "c2 differs"
+    assert np.array_equal(g_scales, scales), f"scale bytes differ at {np.flatnonzero(g_scales != scales)[:8]}"
+    if not np.array_equal(g_codes, codes):
+        d = np.flatnonzero(g_codes != codes)
+        raise AssertionError(f"codes differ at {d.size} bytes, first {d[:8]}")
+    return qw, (codes, scales, c2)
+
+
+# --------------------------------------------------------------------------
+# quantize / dequantize
+# --------------------------------------------------------------------------
+
+def test_quantize_dequantize_config0_bitexact():
+    w = inputs.normal_bf16((512, 512), 0.02, inputs.seed_of(0, 0, 0, "W"), "cuda")
+    qw, (codes, scales, c2) = quantize_and_check(w)
+    wd = Q().dequantize(qw)
+    torch.cuda.synchronize()
+    ref = O.dequantize_nf4(codes, scales, c2, 512, 512)
+    assert np.array_equal(bits(wd), ref)
+
+
+def _special_weight(rows, cols, seed):
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0, 0.02, (rows, cols)).astype(np.float32)
+    flat = w.reshape(-1, 64)
+    nb = flat.shape[0]
+    flat[0] = 0.0                                       # all +0
+    if nb > 1: flat[1] = -0.0                           # all -0
+    if nb > 2: flat[2] = 0.0; flat[2, 17] = 3.0          # one-hot
+    if nb > 3: flat[3] = rng.normal(0, 1e-38, 64)        # subnormal BF16 values
+    if nb > 4: flat[4] = rng.normal(0, 1e37, 64)         # huge values
+    if nb > 5: flat[5] = rng.normal(0, 1e-6, 64)         # scale in E4M3's subnormal range vs group max
+    if nb > 6: flat[6] = np.linspace(-1, 1, 64)          # exact ties and levels
+    if nb > 7: flat[7, :] = 1.0; flat[7, 5] = -1.0       # ties between +-c1
+    return torch.from_numpy(w).to(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("rows,cols", [(3, 320), (5, 448), (64, 64 * 257), (1, 64), (17, 1024)])
+def test_quantize_dequantize_ragged_and_special_bitexact(rows, cols):
+    w = _special_weight(rows, cols, rows * 1000 + cols)
+    qw, (codes, scales, c2) = quantize_and_check(w)
+    wd = Q().dequantize(qw)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(wd), O.dequantize_nf4(codes, scales, c2, rows, cols))
+
+
+def test_code_function_sweep_over_bf16_pairs():
+    """Every BF16 weight w with |w| <= c1 against c1 = every BF16 mantissa at a
+    spread of exponents (subnormal through near-max): the block holds c1 once
+    (so it is the absmax) and 63 test weights."""
+    c1_bits = []
+    for e in [0, 1, 2, 7, 30, 100, 126, 127, 128, 129, 160, 200, 250, 253, 254]:   # biased exponents
+        for m in range(128):
+            b = (e << 7) | m
+            if b != 0:
+                c1_bits.append(b)
+    blocks = []
+    all_w = np.arange(0, 0x7F80, dtype=np.uint16)                  # non-negative finite BF16 patterns
+    for cb in c1_bits:
+        mag = all_w[all_w <= cb]
+        ws = np.concatenate([mag, mag | 0x8000])
+        pad = (-ws.size) % 63
+        ws = np.concatenate([ws, np.zeros(pad, np.uint16)]).reshape(-1, 63)
+        blk = np.empty((ws.shape[0], 64), np.uint16)
+        blk[:, 0] = cb
+        blk[:, 1:] = ws
+        blocks.append(blk)
+    allb = np.concatenate(blocks)
+    pad = (-allb.shape[0]) % 256
+    allb = np.concatenate([allb, np.zeros((pad, 64), np.uint16)])
+    w = from_bits(allb.reshape(-1, 64 * 256)).cuda()
+    qw = Q().quantize_nf4(w)
+    torch.cuda.synchronize()
+    codes, _, _ = O.quantize_nf4(allb.reshape(-1, 64 * 256))
+    assert np.array_equal(qw.codes.cpu().numpy(), codes)
+
+
+def test_nonfinite_weight_is_reported():
+    q = Q()
+    w = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
+    w[2, 7] = float("inf")
+    q.quantize_nf4(w)
+    with pytest.raises(q.QLoraError) as e:
+        q.get_error()
+    assert e.value.status == 6
+    q.get_error()   # cleared
+
+
+# --------------------------------------------------------------------------
+# forward / backward
+# --------------------------------------------------------------------------
+
+def run_layer(T, N, K, r, s, config=90, a_std=None, b_std=0.01, check_quant=True):
+    W, X, A, B, dY = inputs.layer_inputs(config, 0, 0, T, N, K, r, device="cuda", a_std=a_std, b_std=b_std)
+    q = Q()
+    if check_quant:
+        qw, (codes, scales, c2) = quantize_and_check(W)
+    else:
+        qw = q.quantize_nf4(W)
+        codes, scales, c2 = O.quantize_nf4(bits(W))
+    y = q.linear_fwd(X, qw, A, B, s)
+    dx, dA, dB = q.linear_bwd(dY, X, qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    return (X, A, B, dY), wd, (y, dx, dA, dB)
+
+
+def check_layer(T, N, K, r, s, **kw):
+    (X, A, B, dY), wd, (y, dx, dA, dB) = run_layer(T, N, K, r, s, **kw)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    assert_close("Y", y, O.linear_fwd(xb, wd, ab, bb, s))
+    rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    assert_close("dX", dx, rdx)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
+
+
+def test_layer_config0():
+    """512x512, 16 tokens, rank 8, s = 2; A ~ N(0, 1/512), B ~ N(0, 0.01^2)."""
+    check_layer(16, 512, 512, 8, 2.0, config=0)
+
+
+def test_layer_multi_tile_ragged():
+    """Several weight tiles, two token tiles (one ragged), ragged rank."""
+    check_layer(300, 384, 320, 24, 0.5)
+
+
+@pytest.mark.parametrize("T,N,K,r,s", [
+    (1, 64, 64, 1, 1.0),          # single token, rank 1
+    (7, 136, 192, 16, 2.0),       # N not a multiple of the 128-row tile
+    (33, 256, 128, 128, 0.25),    # maximum rank: two rank stages
+    (257, 128, 256, 65, 1.0),     # ragged rank just over one stage, 2 token tiles
+    (64, 1024, 4096, 64, 1.0),    # decode-like token count on an 8B k/v shape
+])
+def test_layer_edge_shapes(T, N, K, r, s):
+    check_layer(T, N, K, r, s)
+
+
+def test_layer_zero_tokens():
+    q = Q()
+    W = inputs.normal_bf16((128, 128), 0.02, 1, "cuda")
+    qw = q.quantize_nf4(W)
+    X = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
+    A = inputs.normal_bf16((8, 128), 0.1, 2, "cuda")
+    B = inputs.normal_bf16((128, 8), 0.1, 3, "cuda")
+    y = q.linear_fwd(X, qw, A, B, 2.0)
+    dx, dA, dB = q.linear_bwd(torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"), X, qw, A, B, 2.0)
+    torch.cuda.synchronize()
+    assert y.shape == (0, 128) and dx.shape == (0, 128)
+    assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
+
+
+def test_layer_8b_q_projection_full_size_sampled():
+    """T = 4096 tokens on the 4096 x 4096 q projection, rank 16, s = 2: the
+    launch configuration of the bench.  Quantize is checked in full; Y and dX on
+    sampled tokens (every output feature); dA and dB in full."""
+    T, N, K, r, s = 4096, 4096, 4096, 16, 2.0
+    (X, A, B, dY), wd, (y, dx, dA, dB) = run_layer(T, N, K, r, s, config=1)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    rows = np.array([0, 1, 255, 256, 1000, 2047, 2048, 3333, 4094, 4095])
+    assert_close("Y[rows]", y[torch.from_numpy(rows).cuda()], O.linear_fwd(xb[rows], wd, ab, bb, s))
+    Xf, Wf, Af, Bf, G = (O.bf16_bits_to_f32(v).astype(np.float64) for v in (xb, wd, ab, bb, dyb))
+    dU = s * (G @ Bf)
+    assert_close("dX[rows]", dx[torch.from_numpy(rows).cuda()], G[rows] @ Wf + dU[rows] @ Af)
+    assert_close("dA", dA, dU.T @ Xf)
+    assert_close("dB", dB, s * (G.T @ (Xf @ Af.T)))
