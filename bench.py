@@ -1,0 +1,500 @@
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one forward + backward of the seven projections of a
+Llama-3.1-8B-shaped block (q, k, v, o: 4096<-4096 / 1024<-4096; gate, up:
+14336<-4096; down: 4096<-14336), T = 4096 tokens, LoRA rank 16, s = 2, NF4
+weights with double quantization: per projection one qlora_linear_fwd and one
+qlora_linear_bwd.  Metric: fwd+bwd TFLOP/s with 4 T N K + 6 T r (N + K) FLOPs
+per projection.  Inputs are synthetic (seeded normal draws of the workload's
+distributions) and resident in HBM; the step's working set (~0.8 GB) is far
+larger than the 126 MB L2, so no flush is needed between steps.
+
+The JSON line also carries: `e2e` (same metric with the step's X and dY copied
+from pinned host memory and dA, dB read back, inside the timed region),
+`roofline` of the dominant kernel (CUDA-event durations of every launch in the
+timed region, through the library's trace hook), `cpu_baseline` (the CPU
+oracle timed on a bounded token sample), `clocks` sampled with nvidia-smi
+during the timed region, and `secondary` figures for the decode-sized forward
+(T = 1, 4, 16, rank 64) and for quantize/dequantize.
+
+With --gpus N (launched under torchrun) every rank runs an independent replica
+of the step (the layer has no cross-GPU exchange); the time is the maximum over
+ranks and the value the work of all ranks divided by it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+T_TOKENS, RANK, SCALE = 4096, 16, 2.0
+METRIC = "QLoRA NF4 linear fwd+bwd TFLOP/s (8B shapes); decode GB/s; % of roofline"
+
+
+def proj_shapes():
+    from bit_nf4_quantized_20_b200.inputs import LLAMA8B_PROJ
+    return LLAMA8B_PROJ
+
+
+def step_flops(T=T_TOKENS, r=RANK):
+    return sum(4.0 * T * n * k + 6.0 * T * r * (n + k) for (_, n, k) in proj_shapes())
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [r[0] for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[3][1:]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def build_layers(device, T, r, config=1):
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    layers = []
+    for i, (name, N, K) in enumerate(proj_shapes()):
+        W, X, A, B, dY = inputs.layer_inputs(config, 0, i, T, N, K, r, device=device)
+        qw = q.quantize_nf4(W)
+        del W
+        layers.append(dict(name=name, N=N, K=K, qw=qw, X=X, A=A, B=B, dY=dY,
+                           Y=torch.empty(T, N, dtype=torch.bfloat16, device=device),
+                           dX=torch.empty(T, K, dtype=torch.bfloat16, device=device),
+                           dA=torch.empty(r, K, dtype=torch.bfloat16, device=device),
+                           dB=torch.empty(N, r, dtype=torch.bfloat16, device=device)))
+    torch.cuda.synchronize()
+    return layers
+
+
+def run_step(layers, s):
+    import bit_nf4_quantized_20_b200 as q
+    for L in layers:
+        q.linear_fwd(L["X"], L["qw"], L["A"], L["B"], s, out=L["Y"])
+        q.linear_bwd(L["dY"], L["X"], L["qw"], L["A"], L["B"], s, outs=(L["dX"], L["dA"], L["dB"]))
+
+
+class Tracer:
+    """Per-launch CUDA events through qlora_trace_attach."""
+
+    def __init__(self, capacity):
+        import ctypes as C
+        import torch
+        from bit_nf4_quantized_20_b200 import _lib
+        self.C, self.torch, self._lib = C, torch, _lib
+        self.recs = (_lib.TraceRec * capacity)()
+        self.count = C.c_int32(0)
+        self.events = []
+        for i in range(capacity):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()      # torch creates the CUDA event on first record
+            b.record()
+            self.events.append((a, b))
+            self.recs[i].start = C.c_void_p(a.cuda_event)
+            self.recs[i].stop = C.c_void_p(b.cuda_event)
+        self.capacity = capacity
+
+    def __enter__(self):
+        self._lib.check("qlora_trace_attach", self._lib.lib().qlora_trace_attach(
+            self.recs, self.capacity, self.C.byref(self.count)))
+        return self
+
+    def __exit__(self, *a):
+        self._lib.lib().qlora_trace_attach(None, 0, None)
+
+    def per_kernel(self):
+        lib = self._lib.lib()
+        n = min(self.count.value, self.capacity)
+        out = {}
+        for i in range(n):
+            rec = self.recs[i]
+            a, b = self.events[i]
+            ms = a.elapsed_time(b)
+            name = lib.qlora_kernel_name(rec.kernel).decode()
+            d = out.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
+            d["launches"] += 1
+            d["ms"] += ms
+            d["flops"] += rec.flops
+            d["bytes"] += rec.bytes
+        return out
+
+
+def bench_ours(args, rank, world, local_rank):
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    T, r, s = T_TOKENS, RANK, SCALE
+    layers = build_layers(dev, T, r)
+    for _ in range(args.warmup):
+        run_step(layers, s)
+    q.get_error(dev)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region ----
+    launches_per_step = 7 * 7
+    tracer = Tracer(args.steps * launches_per_step + 64)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with tracer:
+            start.record()
+            for _ in range(args.steps):
+                run_step(layers, s)
+            stop.record()
+        torch.cuda.synchronize()
+    q.get_error(dev)
+    ms = start.elapsed_time(stop) / args.steps
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    flops = step_flops(T, r)
+    value = world * flops / (ms * 1e-3) / 1e12
+    kern = tracer.per_kernel()
+    gpu_launches = int(tracer.count.value)
+
+    # ---- end-to-end: host inputs in, adapter gradients out ----
+    e2e = bench_e2e(args, layers, dev, s, world, dist)
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = measured_peaks()
+        dom_name = max(kern, key=lambda k: kern[k]["ms"]) if kern else None
+        roof = None
+        if dom_name:
+            d = kern[dom_name]
+            avg_ms = d["ms"] / d["launches"]
+            if d["flops"] > 0:
+                ach = (d["flops"] / d["launches"]) / (avg_ms * 1e-3) / 1e12
+                peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+                roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                        "frac": round(ach / peak, 4), "traffic": profile_traffic(dom_name),
+                        "kernel": dom_name, "peak_source": f"{peak_src} bf16_tflops_sustained",
+                        "launches": d["launches"], "avg_launch_ms": round(avg_ms, 4)}
+            else:
+                ach = (d["bytes"] / d["launches"]) / (avg_ms * 1e-3) / 1e9
+                peak = float(peaks["hbm_gbs"])
+                roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                        "frac": round(ach / peak, 4), "traffic": profile_traffic(dom_name), "kernel": dom_name,
+                        "peak_source": f"{peak_src} hbm_gbs"}
+        kernels = {k: {"launches": v["launches"], "ms_per_step": round(v["ms"] / args.steps, 4),
+                       "share": round(v["ms"] / sum(x["ms"] for x in kern.values()), 4),
+                       "tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1) if v["flops"] else None}
+                   for k, v in sorted(kern.items(), key=lambda kv: -kv[1]["ms"])}
+        secondary = None if args.no_secondary else bench_secondary(dev, peaks)
+        cpu = None if args.no_cpu else cpu_baseline(args)
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal draws: W~N(0,0.02^2), X,dY~N(0,1), A~N(0,1/K), B~N(0,0.01^2))",
+            "config": {"workload": "llama3.1-8b block, 7 NF4+DQ projections, fwd+bwd", "global_batch": world * T,
+                       "seq_len": T, "tokens_per_gpu": T, "lora_rank": r, "lora_scale": s,
+                       "flops_per_step_per_gpu": flops, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (0.8 GB working set per step), no flush"},
+            "e2e": e2e, "gpu_launches": gpu_launches, "roofline": roof, "kernels": kernels,
+            "cpu_baseline": cpu, "clocks": clk.summary(), "secondary": secondary,
+        }
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def bench_e2e(args, layers, dev, s, world, dist):
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    host = []
+    for L in layers:
+        host.append((L["X"].cpu().pin_memory(), L["dY"].cpu().pin_memory(),
+                     torch.empty_like(L["dA"], device="cpu").pin_memory(),
+                     torch.empty_like(L["dB"], device="cpu").pin_memory()))
+    h2d = sum(h[0].numel() * 2 + h[1].numel() * 2 for h in host)
+    d2h = sum(h[2].numel() * 2 + h[3].numel() * 2 for h in host)
+
+    def e2e_step():
+        for L, (hx, hdy, hda, hdb) in zip(layers, host):
+            L["X"].copy_(hx, non_blocking=True)
+            L["dY"].copy_(hdy, non_blocking=True)
+            q.linear_fwd(L["X"], L["qw"], L["A"], L["B"], s, out=L["Y"])
+            q.linear_bwd(L["dY"], L["X"], L["qw"], L["A"], L["B"], s, outs=(L["dX"], L["dA"], L["dB"]))
+            hda.copy_(L["dA"], non_blocking=True)
+            hdb.copy_(L["dB"], non_blocking=True)
+
+    steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    v = world * step_flops() / (ms * 1e-3) / 1e12
+    return {"value": round(v, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms, 3), "steps": steps}
+
+
+def profile_traffic(kernel_name):
+    """DRAM bytes per launch from a committed ncu summary of this exact kernel
+    source (profiles/traffic.json), else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        ent = d.get(kernel_name)
+        if not ent:
+            return None
+        import hashlib
+        src = os.path.join(ROOT, "bit_nf4_quantized_20_b200", "csrc", ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return ent["bytes_per_launch"] if h == ent["source_sha"] else None
+    except Exception:
+        return None
+
+
+def bench_secondary(dev, peaks):
+    """Decode-sized forward sweep (T = 1, 4, 16; rank 64; s = 1) over the seven
+    8B shapes, and quantize/dequantize of the 14336 x 4096 gate weight."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    out = {}
+    r = 64
+    shapes = proj_shapes()
+    qws, adapters = [], []
+    for i, (_, N, K) in enumerate(shapes):
+        W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(2, 0, i, "W"), dev)
+        qws.append(q.quantize_nf4(W))
+        del W
+        adapters.append((inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(2, 0, i, "A"), dev),
+                         inputs.normal_bf16((N, r), 0.01, inputs.seed_of(2, 0, i, "B"), dev)))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for T in (1, 4, 16):
+        xs = [inputs.normal_bf16((T, K), 1.0, inputs.seed_of(2, 0, i, "X") + T, dev)
+              for i, (_, N, K) in enumerate(shapes)]
+        ys = [torch.empty(T, N, dtype=torch.bfloat16, device=dev) for (_, N, K) in shapes]
+        nbytes = sum(N * K * (0.5 + 1 / 64) + 4 * ((N * K // 64 + 255) // 256) + 2 * r * (N + K) + 2 * T * (N + K)
+                     for (_, N, K) in shapes)
+        times = []
+        for rep in range(8):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for i in range(len(shapes)):
+                q.linear_fwd(xs[i], qws[i], adapters[i][0], adapters[i][1], 1.0, out=ys[i])
+            b.record()
+            torch.cuda.synchronize()
+            if rep >= 3:
+                times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        out[f"decode_T{T}"] = {"us_per_sweep": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                               "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                               "bytes_per_sweep": int(nbytes)}
+    # quantize / dequantize of one gate-shaped weight (58.7 M weights)
+    N, K = 14336, 4096
+    W = inputs.normal_bf16((N, K), 0.02, 7, dev)
+    qw = q.quantize_nf4(W)
+    wd = torch.empty_like(W)
+    per = 2.0 + 0.5 + 1 / 64
+    for name, fn in (("quantize", lambda: q.quantize_nf4(W)), ("dequantize", lambda: q.dequantize(qw))):
+        times = []
+        for rep in range(6):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        gbs = N * K * per / (ms * 1e-3) / 1e9
+        out[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                     "weights": N * K}
+    q.get_error(dev)
+    return out
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+# --------------------------------------------------------------------------
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(T_sample, r=RANK, s=SCALE, prepared=None):
+    """One pass of the CPU oracle over the 8B block at T_sample tokens:
+    dequantize each projection's NF4 weight, then fp64 forward and backward."""
+    from oracle import oracle as O
+    from bit_nf4_quantized_20_b200 import inputs
+    if prepared is None:
+        prepared = []
+        for i, (_, N, K) in enumerate(proj_shapes()):
+            W, X, A, B, dY = inputs.layer_inputs(1, 0, i, T_sample, N, K, r, device="cpu")
+            codes, scales, c2 = O.quantize_nf4(inputs.bf16_bits(W))
+            prepared.append((N, K, codes, scales, c2, inputs.bf16_bits(X), inputs.bf16_bits(A),
+                             inputs.bf16_bits(B), inputs.bf16_bits(dY)))
+        return prepared
+    t0 = time.perf_counter()
+    for (N, K, codes, scales, c2, xb, ab, bb, dyb) in prepared:
+        wd = O.dequantize_nf4(codes, scales, c2, N, K)
+        O.linear_fwd(xb, wd, ab, bb, s)
+        O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(args, T_sample=256):
+    prepared = oracle_sample_step(T_sample)
+    sec = oracle_sample_step(T_sample, prepared=prepared)
+    v = step_flops(T_sample) / sec / 1e12
+    return {"value": round(v, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"one fwd+bwd pass of all 7 projections at T={T_sample} tokens (of 4096), "
+                      f"including the per-step NF4 dequantization; {sec:.1f} s"}
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    T_sample = 128
+    prepared = oracle_sample_step(T_sample)
+    for _ in range(args.warmup):
+        pass   # the oracle has no warm-up state; warm-up steps are not repeated
+    secs = []
+    for _ in range(args.steps):
+        secs.append(oracle_sample_step(T_sample, prepared=prepared))
+    sec = sum(secs) / len(secs)
+    v = step_flops(T_sample) / sec / 1e12
+    cores = oracle_threads()
+    sample = f"each step: fwd+bwd of all 7 projections at T={T_sample} tokens (of 4096) with NF4 dequantization"
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "llama3.1-8b block, 7 NF4+DQ projections, fwd+bwd",
+                                            "seq_len": T_TOKENS, "lora_rank": RANK, "lora_scale": SCALE,
+                                            "token_sample": T_sample},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the decode and quantize figures")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+    else:
+        res = bench_ours(args, rank, world, local_rank)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

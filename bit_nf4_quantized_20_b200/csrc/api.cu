@@ -34,11 +34,13 @@ enum KernelId : int32_t {
   K_LORA_DA = 5,
   K_GEMM_FWD = 6,
   K_GEMM_BWD = 7,
-  K_COUNT = 8,
+  K_GEMV_FWD = 8,
+  K_COUNT = 9,
 };
 
 const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",   "lora_du",
-                                     "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx"};
+                                     "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx",
+                                     "nf4_gemv_fwd"};
 
 struct TraceScope {
   cudaStream_t st;
@@ -243,6 +245,37 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// Token counts up to this use the decode-sized forward (register-fragment
+// dequantization, split-K over a thread block cluster).
+constexpr int64_t kGemvMaxTokens = 16;
+
+qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
+                      const void *B, int r, void *y, cudaStream_t st) {
+  GemvParams p;
+  memset(&p, 0, sizeof(p));
+  p.codes = qw->codes;
+  p.scales = qw->scales;
+  p.c2 = qw->c2;
+  for (int i = 0; i < 16; ++i) p.codebook[i] = qw->codebook[i];
+  p.N = qw->rows;
+  p.K = qw->cols;
+  p.T = static_cast<int>(T);
+  p.x = static_cast<const uint16_t *>(x);
+  p.u = u;
+  p.ldu = ldu;
+  p.B = static_cast<const uint16_t *>(B);
+  p.r = r;
+  p.y = static_cast<uint16_t *>(y);
+  const GemvPlan pl = gemv_plan(p.N, p.K, num_sms_current());
+  const double n = static_cast<double>(p.N) * p.K;
+  const double bytes = n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * T * (p.N + p.K) +
+                       2.0 * static_cast<double>(p.N) * r;
+  TraceScope ts(K_GEMV_FWD, 0.0, bytes, st);
+  // programmatic dependent launch only when no trace events sit between the kernels
+  const bool pdl = g_trace.recs == nullptr;
+  return launch_gemv(p, pl, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 qlora_status run_skinny(int32_t kid, const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st) {
   const double flops = 2.0 * p.M * p.C * p.R * (p.Q1 ? 2 : 1);
   const double bytes = 2.0 * p.M * p.C;
@@ -380,7 +413,8 @@ static qlora_status check_linear(const void *x, int64_t T, const qlora_nf4_weigh
                                  const void *B, int32_t r, float s) {
   qlora_status st = check_weight(qw);
   if (st != QLORA_OK) return st;
-  if (!x || !A || !B) return QLORA_ERR_INVALID_ARG;
+  // token-sized buffers may be null (empty) when T == 0
+  if ((T > 0 && !x) || !A || !B) return QLORA_ERR_INVALID_ARG;
   if (T < 0 || r < 1 || r > 128 || !isfinite(s)) return QLORA_ERR_INVALID_ARG;
   if (qw->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
   if (T > 0x7fffffff || qw->rows > 0x7fffffff || qw->cols > 0x7fffffff) return QLORA_ERR_UNSUPPORTED;
@@ -392,7 +426,7 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
                               int32_t r, float s, void *y, void *ws, size_t ws_bytes, void *stream) {
   qlora_status cs = check_linear(x, T, qw, A, B, r, s);
   if (cs != QLORA_OK) return cs;
-  if (!y) return QLORA_ERR_INVALID_ARG;
+  if (T > 0 && !y) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(y)) return QLORA_ERR_MISALIGNED;
   const int64_t N = qw->rows, K = qw->cols;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_FWD, T, N, K, r))
@@ -415,6 +449,7 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
   pu.ldo = r64;
   qlora_status rs = run_skinny(K_LORA_U, pu, false, false, OUT_HILO, st);
   if (rs != QLORA_OK) return rs;
+  if (T <= kGemvMaxTokens) return run_gemv(qw, x, T, su_hi, r64, B, r, y, st);
   return run_gemm(0, qw, x, su_hi, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), st);
 }
 
@@ -423,7 +458,7 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
                               size_t ws_bytes, void *stream) {
   qlora_status cs = check_linear(x, T, qw, A, B, r, s);
   if (cs != QLORA_OK) return cs;
-  if (!dy || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if ((T > 0 && (!dy || !dx)) || !dA || !dB) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(dy) || !aligned16(dx) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
   const int64_t N = qw->rows, K = qw->cols;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r))

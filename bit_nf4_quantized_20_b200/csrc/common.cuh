@@ -92,16 +92,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most
 // kWaitLimitNs.  Returns false (and records DEV_TIMEOUT) if it never does.
+// Waiting threads are suspended between probes (try_wait's time hint) and
+// read the global timer only every 64 probes, so that long waits (the
+// epilogue waiting for a whole tile) take few issue slots.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      set_status(status, DEV_TIMEOUT);
-      return false;
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+    if ((i & 63u) == 0) {
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        set_status(status, DEV_TIMEOUT);
+        return false;
+      }
     }
   }
 }

@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int n_tile = tile % p.n_tiles;
+        const int n_tile = tile / p.m_tiles;
         const int t0 = n_tile * BN;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % STAGES;
@@ -294,14 +294,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       row_off = (tid >> 3) * 1024 + (tid & 7) * 128;
       phase = tid & 7;
     } else {
-      const int rho = tid >> 1, h = tid & 1;
+      const int rho = tid & 63, h = tid >> 6;   // 8 consecutive lanes: 8 swizzle phases
       row_off = ((rho >> 3) * 2 + h) * 1024 + (rho & 7) * 128;
       phase = rho & 7;
     }
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m_tile = tile / p.n_tiles;
+      const int m_tile = tile % p.m_tiles;
       // block coordinates for stage ks
       auto block_of = [&](int ks, int64_t &blk) -> bool {
         int64_t n, kb;
@@ -309,22 +309,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           n = static_cast<int64_t>(m_tile) * BM + tid;
           kb = ks;
         } else {
-          n = static_cast<int64_t>(ks) * BK + (tid >> 1);
-          kb = static_cast<int64_t>(m_tile) * (BM / 64) + (tid & 1);
+          n = static_cast<int64_t>(ks) * BK + (tid & 63);
+          kb = static_cast<int64_t>(m_tile) * (BM / 64) + (tid >> 6);
         }
         blk = n * kblocks + kb;
         return n < p.N && kb < kblocks;
       };
-      int64_t blk;
-      bool valid = block_of(0, blk);
-      BlockIn cur = load_block(p, blk, valid && p.k_main > 0);
+      // codes and scales are prefetched PF stages ahead into a register ring
+      auto fetch = [&](int ks) -> BlockIn {
+        int64_t blk = 0;
+        const bool v = ks < p.k_main && block_of(ks, blk);
+        return load_block(p, blk, v);
+      };
+      BlockIn b0 = fetch(0), b1 = fetch(1), b2 = fetch(2);
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        BlockIn nxt;
-        if (ks + 1 < p.k_main) {
-          int64_t nblk;
-          const bool nvalid = block_of(ks + 1, nblk);
-          nxt = load_block(p, nblk, nvalid);
-        }
+        const BlockIn cur = b0;
+        b0 = b1;
+        b1 = b2;
+        b2 = fetch(ks + 3);
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) { ok = false; break; }
@@ -341,8 +343,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             copy_row(src, nv, (p.r % 8) == 0, row_addr, phase);
           } else {
             // A[r, K] rows j = 64l + rho, columns k0 .. k0+63
-            const int j = l * BK + (tid >> 1);
-            const int64_t k0 = static_cast<int64_t>(m_tile) * BM + (tid & 1) * 64;
+            const int j = l * BK + (tid & 63);
+            const int64_t k0 = static_cast<int64_t>(m_tile) * BM + (tid >> 6) * 64;
             const int nv = (j < p.r && k0 < p.K) ? 64 : 0;
             const uint16_t *src = p.lora + static_cast<int64_t>(j < p.r ? j : 0) * p.K + (k0 < p.K ? k0 : 0);
             copy_row(src, nv, true, row_addr, phase);
@@ -350,7 +352,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(sm.full_a(s));
-        cur = nxt;
       }
     }
     if (!ok) atomicExch(const_cast<int *>(&s_abort), 1);
@@ -361,8 +362,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int tc = 0, chunk_count = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-      const int m_tile = tile / p.n_tiles;
-      const int n_tile = tile % p.n_tiles;
+      const int m_tile = tile % p.m_tiles;
+      const int n_tile = tile / p.m_tiles;
       const int acc = tc & 1;
       const uint32_t acc_phase = (tc >> 1) & 1;
       const bool fail = s_abort || !mbar_wait(sm.acc_full(acc), acc_phase, p.status);

@@ -45,6 +45,34 @@ __global__ void nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                 const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
 
 // ---------------------------------------------------------------------------
+// decode-sized forward, T <= 16 (gemv_nf4.cu)
+// ---------------------------------------------------------------------------
+struct GemvParams {
+  const uint8_t *codes;
+  const uint8_t *scales;
+  const float *c2;
+  float codebook[16];
+  int64_t N, K;
+  int T;
+  const uint16_t *x;     // [T, K]
+  const uint16_t *u;     // U' = BF16(s X A^T), [T, ldu]
+  int64_t ldu;
+  const uint16_t *B;     // [N, r]
+  int r;
+  uint16_t *y;           // [T, N]
+  int units, upw, splits;  // filled from the plan
+};
+struct GemvPlan {
+  int units;       // 256-wide k units
+  int upw;         // units per warp
+  int splits;      // CTAs per row tile (thread block cluster size, <= 8)
+  int rg;          // 8-row groups per CTA
+  int row_tiles;
+};
+GemvPlan gemv_plan(int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv(const GemvParams &p, const GemvPlan &pl, cudaStream_t st, bool pdl);
+
+// ---------------------------------------------------------------------------
 // rank-r LoRA GEMMs on the legacy tensor path (skinny.cu)
 //   C[M, R] = alpha * sum_c P(m, c) * Q(c, j),  Q = Q0 (+ Q1)
 // ---------------------------------------------------------------------------

@@ -28,6 +28,7 @@ namespace {
 constexpr int SBM = 64;    // rows (m) per CTA
 constexpr int SBC = 64;    // contraction per stage
 constexpr int ST = 128;    // threads
+constexpr int SST = 4;     // cp.async pipeline stages
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
   const int n = valid ? 16 : 0;
@@ -71,7 +72,7 @@ struct Layout {
   static constexpr int STAGE_BYTES = P_BYTES + NQ * Q_BYTES;
   static constexpr int ACC_PITCH = RP + 4;
   static constexpr int ACC_BYTES = SBM * ACC_PITCH * 4;
-  static constexpr int SMEM = (2 * STAGE_BYTES > ACC_BYTES ? 2 * STAGE_BYTES : ACC_BYTES) + 16;
+  static constexpr int SMEM = (SST * STAGE_BYTES > ACC_BYTES ? SST * STAGE_BYTES : ACC_BYTES) + 16;
 };
 
 template <bool PCOL, bool QCJ, bool TWOQ, int RP>
@@ -80,6 +81,9 @@ __global__ void __launch_bounds__(ST) skinny_kernel(const SkinnyParams p, int ou
   using L = Layout<PCOL, QCJ, TWOQ, RP>;
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_last;
+  // a kernel launched after this one with programmatic dependent launch may
+  // start now; it waits (griddepcontrol.wait) before reading what we write
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_tile = blockIdx.x;
@@ -142,19 +146,20 @@ __global__ void __launch_bounds__(ST) skinny_kernel(const SkinnyParams p, int ou
 #pragma unroll
   for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
-  if (nstages > 0) {
-    load_stage(0, cbeg);
+  // SST-deep cp.async pipeline; one commit group per stage slot (possibly empty)
+#pragma unroll
+  for (int i = 0; i < SST - 1; ++i) {
+    if (i < nstages) load_stage(i, cbeg + static_cast<int64_t>(i) * SBC);
     cp_async_commit();
   }
   for (int st = 0; st < nstages; ++st) {
-    const int buf = st & 1;
-    if (st + 1 < nstages) {
-      load_stage(buf ^ 1, cbeg + static_cast<int64_t>(st + 1) * SBC);
+    const int buf = st % SST;
+    {
+      const int nxt = st + SST - 1;
+      if (nxt < nstages) load_stage(nxt % SST, cbeg + static_cast<int64_t>(nxt) * SBC);
       cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
     }
+    cp_async_wait<SST - 1>();
     __syncthreads();
     const uint32_t pb = sbase + buf * L::STAGE_BYTES;
 #pragma unroll
@@ -293,6 +298,7 @@ cudaError_t launch_rp(const SkinnyParams &p, int out_mode, int q_ncols, int q_ve
 static int rp_of(int R) { return R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128; }
 
 int skinny_splits(int64_t M, int64_t C, int num_sms) {
+  if (M <= 0 || C <= 0 || num_sms <= 0) return 1;
   const int64_t m_tiles = (M + SBM - 1) / SBM;
   int64_t want = (2 * static_cast<int64_t>(num_sms) + m_tiles - 1) / m_tiles;
   const int64_t cap = (C + 255) / 256;        // at least four stages per split

@@ -86,6 +86,9 @@ def test_workspace_bytes(L):
     assert L.qlora_workspace_bytes(1, 4096, 4096, 4096, 0) == 0
     assert L.qlora_workspace_bytes(1, 4096, 4096, 4096, 129) == 0
     assert L.qlora_workspace_bytes(7, 16, 16, 64, 8) == 0
+    # zero tokens is a valid (empty) call: the size query must not fault
+    assert L.qlora_workspace_bytes(1, 0, 4096, 4096, 16) > 0
+    assert L.qlora_workspace_bytes(2, 0, 4096, 4096, 16) > 0
     # grows with the token count
     assert L.qlora_workspace_bytes(2, 8192, 4096, 4096, 16) > b
 
@@ -150,6 +153,15 @@ def test_linear_validation(L):
     deq = L.qlora_dequantize
     assert deq(C.byref(w), None, None) == 1
     assert deq(C.byref(w), C.c_void_p(FAKE + 1), None) == 3
+
+
+def test_linear_fwd_zero_tokens_is_a_noop(L):
+    """T == 0 launches nothing; the empty token buffers may be null."""
+    w = _weight()
+    P = C.c_void_p(FAKE)
+    ws = C.c_void_p(FAKE)
+    assert L.qlora_linear_fwd(None, 0, C.byref(w), P, P, 8, 2.0, None, ws, 1 << 30, None) == 0
+    assert L.qlora_linear_fwd(None, 5, C.byref(w), P, P, 8, 2.0, None, ws, 1 << 30, None) == 1
 
 
 def test_trace_attach_validation(L):

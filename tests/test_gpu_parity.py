@@ -216,3 +216,23 @@ def test_layer_8b_q_projection_full_size_sampled():
     assert_close("dX[rows]", dx[torch.from_numpy(rows).cuda()], G[rows] @ Wf + dU[rows] @ Af)
     assert_close("dA", dA, dU.T @ Xf)
     assert_close("dB", dB, s * (G.T @ (Xf @ Af.T)))
+
+
+@pytest.mark.parametrize("T,N,K", [
+    (1, 1024, 4096),      # 8B k/v projection, single token
+    (4, 4096, 4096),      # 8B q/o projection
+    (9, 4096, 14336),     # 8B down projection: 56 k-units, 7-CTA cluster, 9..16-token variant
+    (16, 14336, 4096),    # 8B gate/up projection
+    (3, 40, 320),         # ragged rows and a k-unit with a missing block
+])
+def test_decode_forward(T, N, K):
+    """Decode-sized forward (T <= 16): rank 64, s = 1, as in the decode sweep."""
+    r, s = 64, 1.0
+    W, X, A, B, _ = inputs.layer_inputs(2, 0, 0, T, N, K, r, device="cuda")
+    q = Q()
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    y = q.linear_fwd(X, qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    assert_close("Y", y, O.linear_fwd(bits(X), wd, bits(A), bits(B), s))
