@@ -315,24 +315,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         blk = n * kblocks + kb;
         return n < p.N && kb < kblocks;
       };
-      // codes and scales are prefetched PF stages ahead into a register ring
+      // Codes and scales are prefetched four stages ahead into four fixed
+      // register buffers; each buffer is refilled in place right after it is
+      // consumed (no register moves of loads still in flight).
       auto fetch = [&](int ks) -> BlockIn {
         int64_t blk = 0;
         const bool v = ks < p.k_main && block_of(ks, blk);
         return load_block(p, blk, v);
       };
-      BlockIn b0 = fetch(0), b1 = fetch(1), b2 = fetch(2);
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        const BlockIn cur = b0;
-        b0 = b1;
-        b1 = b2;
-        b2 = fetch(ks + 3);
+      auto produce = [&](int ks, BlockIn &buf) -> bool {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) { ok = false; break; }
+        ++it;
+        if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) return false;
         const uint32_t row_addr = sm.a(s) + row_off;
         if (ks < p.k_main) {
-          dequant_row(cb, cur, row_addr, phase);
+          dequant_row(cb, buf, row_addr, phase);
         } else {
           const int l = ks - p.k_main;
           if (!bwd) {
@@ -352,6 +350,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(sm.full_a(s));
+        buf = fetch(ks + 4);
+        return true;
+      };
+      BlockIn r0 = fetch(0), r1 = fetch(1), r2 = fetch(2), r3 = fetch(3);
+      for (int ks = 0; ks < ksteps && ok; ks += 4) {
+        ok = produce(ks, r0);
+        if (ok && ks + 1 < ksteps) ok = produce(ks + 1, r1);
+        if (ok && ks + 2 < ksteps) ok = produce(ks + 2, r2);
+        if (ok && ks + 3 < ksteps) ok = produce(ks + 3, r3);
       }
     }
     if (!ok) atomicExch(const_cast<int *>(&s_abort), 1);

@@ -277,8 +277,12 @@ template <bool PCOL, bool QCJ, bool TWOQ, int RP>
 cudaError_t launch_t(const SkinnyParams &p, int out_mode, int q_ncols, int q_vec, cudaStream_t st) {
   using L = Layout<PCOL, QCJ, TWOQ, RP>;
   auto kern = skinny_kernel<PCOL, QCJ, TWOQ, RP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;   // once per instantiation (keeps calls capturable in CUDA graphs)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   const int64_t m_tiles = (p.M + SBM - 1) / SBM;
   dim3 grid(static_cast<unsigned>(m_tiles), static_cast<unsigned>(p.splits));
   kern<<<grid, ST, L::SMEM, st>>>(p, out_mode, q_ncols, q_vec);
