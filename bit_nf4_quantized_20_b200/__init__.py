@@ -20,7 +20,7 @@ from . import _lib
 from ._lib import OP_BWD, OP_FWD, OP_QUANTIZE, NF4Weight, QLoraError, check, lib
 
 __all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "linear_fwd",
-           "linear_bwd", "workspace", "workspace_bytes", "get_error", "QLoraError", "lib"]
+           "linear_bwd", "linear_fwd_noalloc", "workspace", "workspace_bytes", "get_error", "QLoraError", "lib"]
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -163,6 +163,20 @@ def linear_fwd(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tens
         C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()), C.c_void_p(B.data_ptr()), r,
         float(s), C.c_void_p(y.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
     return y
+
+
+def linear_fwd_noalloc(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
+                       out: torch.Tensor) -> torch.Tensor:
+    """Forward through the entry point that uses the library's fixed device
+    scratch instead of a workspace (for callers that cannot allocate device
+    memory); `out` must be preallocated [T, N] bf16."""
+    T, r = _check_linear(x, qw, A, B)
+    _need_cuda("out", out)
+    st = qw.struct()
+    check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(
+        C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()), C.c_void_p(B.data_ptr()), r,
+        float(s), C.c_void_p(out.data_ptr()), _stream(x.device)))
+    return out
 
 
 def linear_bwd(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,

@@ -53,6 +53,8 @@ SIGNATURES = {
     "qlora_linear_bwd": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p,
                                    C.c_void_p, C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
                                    C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qlora_linear_fwd_noalloc": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
+                                           C.c_int32, C.c_float, C.c_void_p, C.c_void_p]),
     "qlora_trace_attach": (C.c_int, [C.POINTER(TraceRec), C.c_int32, C.POINTER(C.c_int32)]),
     "qlora_kernel_name": (C.c_char_p, [C.c_int32]),
 }

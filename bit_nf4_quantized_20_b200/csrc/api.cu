@@ -527,6 +527,42 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   return run_skinny(K_LORA_DA, pa, true, true, OUT_T, st);
 }
 
+// ---------------------------------------------------------------------------
+// Forward without a caller workspace.  Its scratch (status word, split
+// counters, the U' planes and the split partial sums) lives in this fixed
+// device array; each GPU that loads the library reserves it until exit.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+static void *noalloc_scratch_ptr() {
+  // the symbol's device address, looked up once per device with that device current
+  static void *ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+qlora_status qlora_linear_fwd_noalloc(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                                      const void *B, int32_t r, float s, void *y, void *stream) {
+  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
+  if (cs != QLORA_OK) return cs;
+  const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, T, qw->rows, qw->cols, r);
+  if (need == 0 || need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_WORKSPACE;
+  void *ws = noalloc_scratch_ptr();
+  if (!ws) return QLORA_ERR_CUDA;
+  // the status word and the split counters must start at zero
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + kWsCounterBytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  return qlora_linear_fwd(x, T, qw, A, B, r, s, y, ws, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 qlora_status qlora_trace_attach(qlora_trace_rec *recs, int32_t capacity, int32_t *count) {
   if (recs && (!count || capacity < 0)) return QLORA_ERR_INVALID_ARG;
   g_trace.recs = recs;

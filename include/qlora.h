@@ -182,6 +182,36 @@ QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T
                               void *dB, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Forward without a caller-supplied workspace (no counterpart on the pages: a
+ * deployment aid).  For callers that cannot allocate device memory: code that
+ * runs under a host framework which owns every device allocation (a serving
+ * runtime's plugin interface that hands in only input and output buffers), or
+ * that must not allocate at call time.  Computes exactly what qlora_linear_fwd
+ * computes; the caller still passes x, the weight, A, B and y.
+ *
+ * Scratch: a fixed array of QLORA_NOALLOC_SCRATCH_BYTES (4 MiB) in the
+ * library's device memory, reserved on every GPU that loads the library until
+ * the process exits.  The call allocates and frees nothing.  Sizes whose
+ * qlora_workspace_bytes(QLORA_OP_FWD, T, N, K, r) exceeds the array are
+ * rejected with QLORA_ERR_WORKSPACE (e.g. T = 4096 fits at r = 16 on a
+ * 14336 x 4096 weight, but not at r = 64).
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (make it before any stream capture).  Every call zeroes the array's
+ * status word and counters on `stream`, then reuses it; all calls share the
+ * one array, so calls that may overlap on the GPU (different streams, or
+ * concurrent host threads) race and must be serialized by the caller.
+ * A device-side failure (a bounded wait that ran out) is recorded in the
+ * array's status word, which the next call clears; this entry point has no
+ * separate status query.
+ * Errors: as qlora_linear_fwd; QLORA_ERR_WORKSPACE for sizes beyond the array.
+ */
+#define QLORA_NOALLOC_SCRATCH_BYTES (4u << 20)
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const void *x, int64_t T, const qlora_nf4_weight *qw,
+                                                const void *A, const void *B, int32_t r, float s, void *y,
+                                                void *stream);
+
+/*
  * Launch trace (profiling hook).  While attached, every kernel the library
  * launches records recs[i].start before and recs[i].stop after it on the
  * call's stream (cudaEvent_t handles the caller created), and fills kernel id,
