@@ -29,6 +29,7 @@ namespace qlora {
 namespace {
 
 constexpr int GW = 8;              // warps per CTA
+constexpr int kMaxRank = 128;
 constexpr int GT = GW * 32;
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -74,9 +75,11 @@ struct Blk {
 };
 
 template <int TT, int RG>
-__global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
   __shared__ float s_red[GW][TT][8 * RG];
   __shared__ float s_part[TT][8 * RG];
+  __shared__ __align__(16) uint16_t s_B[8 * RG][kMaxRank + 8];
+  __shared__ __align__(16) uint16_t s_U[TT][kMaxRank + 8];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
     Blk b;
     const int64_t n = row0 + rg * 8 + g;
     const int64_t kb = static_cast<int64_t>(u) * 4 + t;
-    if (n < p.N && kb < kblocks) {
+    if (u < p.units && n < p.N && kb < kblocks) {
       const int64_t blk = n * kblocks + kb;
       const uint8_t *cp = p.codes + blk * 32;
       b.c0 = ldg_stream(cp);
@@ -112,9 +115,22 @@ __global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
     return b;
   };
 
+  // Units of this warp: u_j = (split * upw + j) * GW + warp.  The codes of
+  // unit j + 1 are requested before unit j is computed (two register sets).
+  auto unit_of = [&](int j) { return (split * p.upw + j) * GW + warp; };
+  Blk cur[RG], nxt[RG];
+  {
+    const int u0 = unit_of(0);
+#pragma unroll
+    for (int rg = 0; rg < RG; ++rg) cur[rg] = load_blk(u0 < p.units ? u0 : p.units, rg);
+  }
   for (int j = 0; j < p.upw; ++j) {
-    const int u = (split * p.upw + j) * GW + warp;
+    const int u = unit_of(j);
     if (u >= p.units) break;
+    const int un = unit_of(j + 1);
+    const bool more = (j + 1 < p.upw) && (un < p.units);
+#pragma unroll
+    for (int rg = 0; rg < RG; ++rg) nxt[rg] = load_blk(more ? un : p.units, rg);
     // X fragments for this unit: token rows g (and g + 8), k = 64t .. 64t + 63
     uint32_t xa[32], xb[TT == 16 ? 32 : 1];
     {
@@ -145,13 +161,11 @@ __global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
         }
       }
     }
-    Blk nxt = load_blk(u, 0);
 #pragma unroll
     for (int rg = 0; rg < RG; ++rg) {
-      const Blk cur = nxt;
-      if (rg + 1 < RG) nxt = load_blk(u, rg + 1);
-      const Lut16 lut = make_lut16(cb, cur.scale);
-      const uint32_t w[8] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w, cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
+      const Lut16 lut = make_lut16(cb, cur[rg].scale);
+      const uint32_t w[8] = {cur[rg].c0.x, cur[rg].c0.y, cur[rg].c0.z, cur[rg].c0.w,
+                             cur[rg].c1.x, cur[rg].c1.y, cur[rg].c1.z, cur[rg].c1.w};
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         uint32_t b0, b1;
@@ -161,6 +175,8 @@ __global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
         mma16816(acc[rg], xa[2 * i], a1, xa[2 * i + 1], a3, b0, b1);
       }
     }
+#pragma unroll
+    for (int rg = 0; rg < RG; ++rg) cur[rg] = nxt[rg];
   }
 
   // accumulator fragment: c0/c1 = (token g, rows 2t, 2t+1), c2/c3 = (token g+8, ...)
@@ -188,20 +204,39 @@ __global__ void __launch_bounds__(GT) nf4_gemv_kernel(const GemvParams p) {
   else __syncthreads();
 
   if (split == 0) {
+    // rank-r term sum_j U'[tok, j] B[n, j] from shared memory: this CTA's rows of
+    // B (independent of the preceding kernel) first, U' after the dependency wait
+    const int nrows = static_cast<int>(min(static_cast<int64_t>(8 * RG), p.N - row0));
+    const int rv = p.r;
+    const uint16_t *bsrc = p.B + row0 * rv;
+    const int nb = nrows * rv;
+    if ((rv % 8) == 0) {
+      for (int c = threadIdx.x; c < nb / 8; c += GT) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(bsrc) + c);
+        const int e = c * 8, row = e / rv, j = e % rv;
+        *reinterpret_cast<uint4 *>(&s_B[row][j]) = v;
+      }
+    } else {
+      for (int e = threadIdx.x; e < nb; e += GT) s_B[e / rv][e % rv] = bsrc[e];
+    }
     grid_dep_wait();   // U' is written by the preceding kernel
+    const int ucols = static_cast<int>((rv + 7) / 8 * 8);      // the U' plane is zero-padded to ldu >= this
+    for (int c = threadIdx.x; c < p.T * (ucols / 8); c += GT) {
+      const int tok = c / (ucols / 8), j = (c % (ucols / 8)) * 8;
+      *reinterpret_cast<uint4 *>(&s_U[tok][j]) =
+          __ldg(reinterpret_cast<const uint4 *>(p.u + static_cast<int64_t>(tok) * p.ldu + j));
+    }
+    __syncthreads();
     for (int idx = threadIdx.x; idx < TT * 8 * RG; idx += GT) {
       const int tok = idx / (8 * RG), row = idx % (8 * RG);
       const int64_t n = row0 + row;
-      if (tok >= p.T || n >= p.N) continue;
+      if (tok >= p.T || row >= nrows) continue;
       float v = 0.f;
       for (int r = 0; r < S; ++r) v += (r == 0) ? s_part[tok][row] : ld_dsmem_f32(&s_part[tok][row], r);
-      // rank-r term: sum_j U'[tok, j] B[n, j]
       float l = 0.f;
-      const uint16_t *ur = p.u + static_cast<int64_t>(tok) * p.ldu;
-      const uint16_t *br = p.B + n * p.r;
-      for (int jj = 0; jj < p.r; ++jj) {
-        l = fmaf(__uint_as_float(static_cast<uint32_t>(ur[jj]) << 16),
-                 __uint_as_float(static_cast<uint32_t>(br[jj]) << 16), l);
+      for (int jj = 0; jj < rv; ++jj) {
+        l = fmaf(__uint_as_float(static_cast<uint32_t>(s_U[tok][jj]) << 16),
+                 __uint_as_float(static_cast<uint32_t>(s_B[row][jj]) << 16), l);
       }
       const __nv_bfloat16 o = __float2bfloat16_rn(v + l);
       p.y[static_cast<int64_t>(tok) * p.N + n] = *reinterpret_cast<const uint16_t *>(&o);
@@ -239,18 +274,23 @@ cudaError_t launch_tr(const GemvParams &p, int row_tiles, cudaStream_t st, bool 
 GemvPlan gemv_plan(int64_t N, int64_t K, int num_sms) {
   GemvPlan pl;
   pl.units = static_cast<int>((K + 255) / 256);
-  pl.upw = (pl.units + 8 * GW - 1) / (8 * GW);       // keeps the cluster at <= 8 CTAs
-  pl.splits = (pl.units + GW * pl.upw - 1) / (GW * pl.upw);
-  pl.rg = 1;
-  const int rgs[3] = {4, 2, 1};
-  for (int i = 0; i < 3; ++i) {
-    const int64_t tiles = (N + 8 * rgs[i] - 1) / (8 * rgs[i]);
-    if (tiles * pl.splits >= (3 * static_cast<int64_t>(num_sms)) / 2 || rgs[i] == 1) {
-      pl.rg = rgs[i];
-      pl.row_tiles = static_cast<int>(tiles);
-      break;
-    }
+  // 16-row tiles (8-row tiles for small N); split k over a cluster only when the
+  // row tiles alone cannot give every SM two CTAs
+  pl.rg = 2;
+  int64_t tiles = (N + 15) / 16;
+  if (tiles < 2 * static_cast<int64_t>(num_sms)) {
+    pl.rg = 1;
+    tiles = (N + 7) / 8;
   }
+  int splits = 1;
+  while (splits < 8 && tiles * splits < 2 * static_cast<int64_t>(num_sms) &&
+         pl.units >= GW * (splits + 1)) {
+    ++splits;
+  }
+  // every split gets whole rounds of GW units; at most 8 CTAs per cluster
+  pl.upw = (pl.units + GW * splits - 1) / (GW * splits);
+  pl.splits = (pl.units + GW * pl.upw - 1) / (GW * pl.upw);
+  pl.row_tiles = static_cast<int>(tiles);
   return pl;
 }
 
@@ -260,7 +300,6 @@ cudaError_t launch_gemv(const GemvParams &p_in, const GemvPlan &pl, cudaStream_t
   p.upw = pl.upw;
   p.splits = pl.splits;
   const bool t16 = p.T > 8;
-  if (pl.rg == 4) return t16 ? launch_tr<16, 4>(p, pl.row_tiles, st, pdl) : launch_tr<8, 4>(p, pl.row_tiles, st, pdl);
   if (pl.rg == 2) return t16 ? launch_tr<16, 2>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2>(p, pl.row_tiles, st, pdl);
   return t16 ? launch_tr<16, 1>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1>(p, pl.row_tiles, st, pdl);
 }
