@@ -3,6 +3,7 @@
 
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -203,14 +204,28 @@ SkinnyParams skinny_base(int64_t M, int64_t C, int R, uint8_t *ws, const WsLayou
   return p;
 }
 
+// The one-CTA GEMM kernel is kept for comparison measurements; setting
+// QLORA_GEMM_ONE_CTA=1 in the environment selects it.
+bool use_one_cta_gemm() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("QLORA_GEMM_ONE_CTA");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, const void *lact, int64_t r64,
                       const void *lora, int r, void *out, int64_t T, uint32_t *status, cudaStream_t st) {
   const int64_t N = qw->rows, K = qw->cols;
   const int64_t Mside = mode == 0 ? N : K;     // weight-side extent
   const int64_t Cext = mode == 0 ? K : N;      // contraction extent
+  // the CTA-pair kernel (default) loads 128 tokens per CTA; the one-CTA kernel 256
+  const bool pair = !use_one_cta_gemm();
+  const int act_rows = pair ? 128 : 256;
   CUtensorMap m_act, m_lact, m_out;
-  if (!make_map_bf16(&m_act, act, T, Cext, Cext, 256, 64, true)) return QLORA_ERR_CUDA;
-  if (!make_map_bf16(&m_lact, lact, T, r64, r64, 256, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&m_act, act, T, Cext, Cext, act_rows, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&m_lact, lact, T, r64, r64, act_rows, 64, true)) return QLORA_ERR_CUDA;
   if (!make_map_bf16(&m_out, out, T, Mside, Mside, 32, 128, false)) return QLORA_ERR_CUDA;
   GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -224,11 +239,40 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   p.mode = mode;
   p.lora = static_cast<const uint16_t *>(lora);
   p.r = r;
-  p.m_tiles = static_cast<int>((Mside + 127) / 128);
+  p.m_tiles = static_cast<int>((Mside + (pair ? 255 : 127)) / (pair ? 256 : 128));
   p.n_tiles = static_cast<int>((T + 255) / 256);
   p.k_main = static_cast<int>((Cext + 63) / 64);
   p.k_lora = static_cast<int>(r64 / 64);
   p.status = status;
+  const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
+  const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int sms = num_sms_current();
+  if (pair) {
+    static bool attr2 = false;
+    if (!attr2) {
+      if (cudaFuncSetAttribute(nf4_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               gemm_2sm_smem_bytes()) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+      attr2 = true;
+    }
+    const int64_t clusters = tiles < sms / 2 ? tiles : sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(448, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(gemm_2sm_smem_bytes());
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TraceScope ts(mode == 0 ? K_GEMM_FWD : K_GEMM_BWD, flops, bytes, st);
+    return cudaLaunchKernelEx(&cfg, nf4_gemm_2sm_kernel, m_act, m_lact, m_out, p) == cudaSuccess ? QLORA_OK
+                                                                                                  : QLORA_ERR_CUDA;
+  }
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(nf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes()) !=
@@ -236,10 +280,7 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
       return QLORA_ERR_CUDA;
     attr_set = true;
   }
-  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  const int grid = static_cast<int>(tiles < num_sms_current() ? tiles : num_sms_current());
-  const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
-  const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   TraceScope ts(mode == 0 ? K_GEMM_FWD : K_GEMM_BWD, flops, bytes, st);
   nf4_gemm_kernel<<<grid, 320, gemm_smem_bytes(), st>>>(m_act, m_lact, m_out, p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;

@@ -26,9 +26,12 @@
 // stops issuing work, drains what it issued and frees tensor memory.
 
 #include "common.cuh"
+#include "gemm_common.cuh"
 #include "kernels.h"
 
 namespace qlora {
+
+using namespace gemm;
 
 namespace {
 
@@ -65,104 +68,6 @@ struct Smem {
   __device__ uint32_t drain() const { return base + OFF_BAR + 8 * (3 * STAGES + 4); }
   __device__ uint32_t tmem_slot() const { return base + OFF_BAR + 8 * NUM_BARS; }
 };
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// bar.red.or over `count` threads of named barrier `id`: every thread gets the OR.
-__device__ __forceinline__ bool named_bar_any(int id, int count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred P, Q;\n\t"
-      "setp.ne.u32 P, %1, 0;\n\t"
-      "bar.red.or.pred Q, %2, %3, P;\n\t"
-      "selp.u32 %0, 1, 0, Q;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// One 64-weight block's inputs for a dequantizing thread.
-struct BlockIn {
-  uint4 c0, c1;    // 32 code bytes
-  float scale;     // s_b = RN32(fp8 * c2), or 0 for a row outside the matrix
-};
-
-__device__ __forceinline__ BlockIn load_block(const GemmParams &p, int64_t blk, bool valid) {
-  BlockIn in;
-  if (valid) {
-    const uint8_t *cp = p.codes + blk * 32;
-    in.c0 = ldg_nc_v4(cp);
-    in.c1 = ldg_nc_v4(cp + 16);
-    const float f = e4m3_to_float(__ldg(p.scales + blk));
-    in.scale = __fmul_rn(f, __ldg(p.c2 + (blk >> 8)));
-  } else {
-    in.c0 = make_uint4(0, 0, 0, 0);
-    in.c1 = in.c0;
-    in.scale = 0.f;
-  }
-  return in;
-}
-
-// Dequantize one block into one 128-byte swizzled shared-memory row.
-__device__ __forceinline__ void dequant_row(const float (&cb)[16], const BlockIn &in, uint32_t row_addr,
-                                            uint32_t phase) {
-  const Lut16 lut = make_lut16(cb, in.scale);
-  const uint32_t w[8] = {in.c0.x, in.c0.y, in.c0.z, in.c0.w, in.c1.x, in.c1.y, in.c1.z, in.c1.w};
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t o0, o1, o2, o3;
-    lut16_lookup4(lut, w[c], o0, o1);
-    lut16_lookup4(lut, w[c] >> 16, o2, o3);
-    st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
-  }
-}
-
-// Copy up to 64 BF16 values (zero-padded) into one swizzled shared-memory row.
-__device__ __forceinline__ void copy_row(const uint16_t *src, int n_valid, bool aligned16, uint32_t row_addr,
-                                         uint32_t phase) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t v[4] = {0, 0, 0, 0};
-    const int e0 = c * 8;
-    if (aligned16 && e0 + 8 <= n_valid) {
-      const uint4 q = *reinterpret_cast<const uint4 *>(src + e0);
-      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t h = (e0 + i < n_valid) ? static_cast<uint32_t>(src[e0 + i]) : 0u;
-        v[i >> 1] |= h << ((i & 1) * 16);
-      }
-    }
-    st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), v[0], v[1], v[2], v[3]);
-  }
-}
 
 }  // namespace
 

@@ -1,0 +1,337 @@
+// gemm_nf4_2sm.cu -- the fused NF4 dequantization + tcgen05 GEMM on CTA pairs
+// (2-SM UMMA, cta_group::2), forward and backward-dX.
+//
+//   forward   Y[T, N]  = X[T, K] W'[N, K]^T + (s X A^T)[T, r] B[N, r]^T
+//   backward  dX[T, K] = dY[T, N] W'[N, K] + (s dY B)[T, r] A[r, K]
+//
+// ("QLoRA: Efficient Fine-Tuning", Step 3 eq. 3 and Step 4; W' is produced in
+// shared memory by dequantization warps, "converted to BF16 on the fly for each
+// matrix multiplication", "What is QLoRA?".)
+//
+// A cluster of two CTAs on two SMs owns a 256-weight-row x 256-token tile.
+// Each CTA dequantizes its own 128 weight rows (the MMA's A operand) and
+// TMA-loads its own 128 tokens (half of the B operand); the even CTA issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256), which reads both CTAs' halves
+// and accumulates each CTA's 128 rows x 256 tokens in that CTA's tensor memory.
+// Compared with one CTA per 128 x 256 tile this halves the token operand each
+// SM streams from L2 per FLOP.
+//
+// Warp roles (448 threads per CTA, one CTA per SM, persistent over tiles):
+//   warps 0-3   epilogue: tensor memory -> BF16 -> shared memory -> TMA store
+//   warps 4-7   dequantization, even pipeline stages
+//   warps 8-11  dequantization, odd pipeline stages
+//   warp 12     TMA loads of this CTA's token half (X / dY, then s*U / dU)
+//   warp 13     paired tensor-memory allocation; on the even CTA, the MMA issue
+// Pipeline barriers: full[s] lives in the even CTA and counts both CTAs' TMA
+// bytes (armed by the even CTA) and both CTAs' dequantization warps; empty[s] and acc_full are signalled in both
+// CTAs by a multicast tcgen05.commit; acc_empty (even CTA) counts both CTAs'
+// epilogue warps.  Every wait is bounded; after a timeout each role stops
+// issuing work, drains what it issued, and both CTAs meet at the final cluster
+// barrier before the tensor memory is freed.
+
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+using namespace gemm;
+
+namespace {
+
+constexpr int PM = 128;                        // weight rows per CTA (256 per pair)
+constexpr int PN = 256;                        // tokens per tile
+constexpr int HN = 128;                        // tokens loaded by each CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = PM * BK * 2;           // 16 KiB
+constexpr int B_BYTES = HN * BK * 2;           // 16 KiB
+constexpr int EPI_ROWS = 32;
+constexpr int EPI_BYTES = EPI_ROWS * PM * 2;   // 8 KiB
+constexpr int NUM_THREADS = 448;
+constexpr int TMEM_COLS = 512;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_EPI = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_EPI + 2 * EPI_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 5;       // full[S], empty[S], acc_full[2], acc_empty[2], drain
+constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+// full[s]: the leader's TMA producer (arrive.expect_tx for both CTAs' bytes)
+// + 2 x 4 dequantization warps
+constexpr uint32_t FULL_ARRIVALS = 1 + 8;
+// acc_empty: 2 x 4 epilogue warps
+constexpr uint32_t ACC_EMPTY_ARRIVALS = 8;
+
+struct Smem {
+  uint32_t base;
+  __device__ uint32_t a(int s) const { return base + OFF_A + s * A_BYTES; }
+  __device__ uint32_t b(int s) const { return base + OFF_B + s * B_BYTES; }
+  __device__ uint32_t epi(int i) const { return base + OFF_EPI + i * EPI_BYTES; }
+  __device__ uint32_t full(int s) const { return base + OFF_BAR + 8 * s; }
+  __device__ uint32_t empty(int s) const { return base + OFF_BAR + 8 * (STAGES + s); }
+  __device__ uint32_t acc_full(int i) const { return base + OFF_BAR + 8 * (2 * STAGES + i); }
+  __device__ uint32_t acc_empty(int i) const { return base + OFF_BAR + 8 * (2 * STAGES + 2 + i); }
+  __device__ uint32_t drain() const { return base + OFF_BAR + 8 * (2 * STAGES + 4); }
+  __device__ uint32_t tmem_slot() const { return base + OFF_BAR + 8 * NUM_BARS; }
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lact,
+                        const __grid_constant__ CUtensorMap tmap_out, const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem sm;
+  sm.base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  const bool bwd = p.mode != 0;
+  const uint32_t rank = cluster_ctarank();          // 0: leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+  const int ksteps = p.k_main + p.k_lora;
+  const int m_pairs = p.m_tiles;                     // 256-row weight tiles
+  const int num_tiles = m_pairs * p.n_tiles;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(sm.full(s), FULL_ARRIVALS);
+      mbar_init(sm.empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(sm.acc_full(i), 1);
+      mbar_init(sm.acc_empty(i), ACC_EMPTY_ARRIVALS);
+    }
+    mbar_init(sm.drain(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 12 && lane == 0) {
+    tma_prefetch_desc(&tmap_act);
+    tma_prefetch_desc(&tmap_lact);
+    tma_prefetch_desc(&tmap_out);
+  }
+  if (warp == 13) {
+    tmem_alloc_pair(sm.tmem_slot(), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive_wait();   // the leader's barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = ld_shared_u32(sm.tmem_slot());
+  auto lead = [&](uint32_t local_addr) { return mapa_shared(local_addr, 0); };
+
+  if (warp == 13) {
+    // ---------------- MMA issuer (even CTA) ----------------
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, bwd, false);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
+        const int acc = tc & 1;
+        const uint32_t acc_phase = (tc >> 1) & 1;
+        if (!mbar_wait(sm.acc_empty(acc), acc_phase ^ 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PN);
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(sm.full(s), ph, p.status)) { ok = false; break; }
+          tc_fence_after();
+          int nk = 4;
+          if (ks >= p.k_main) nk = min(4, (p.r - (ks - p.k_main) * BK + 15) / 16);
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t adesc = !bwd ? smem_desc_sw128(sm.a(s) + kk * 32, 16, 1024)        // K-major
+                                        : smem_desc_sw128(sm.a(s) + kk * 4096, 1024, 2048);   // MN-major
+            const uint64_t bdesc = smem_desc_sw128(sm.b(s) + kk * 32, 16, 1024);
+            tc_mma_ss_pair(d_tmem, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(sm.empty(s), 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(sm.acc_full(acc), 0x3);
+      }
+      if (!ok) s_abort = 1;
+      tc_commit_pair_mc(sm.drain(), 0x1);     // every MMA issued so far has completed
+      mbar_wait(sm.drain(), 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp == 12) {
+    // ---------------- TMA producer: this CTA's token half ----------------
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        const int n_tile = tile / m_pairs;
+        const int t0 = n_tile * PN + static_cast<int>(rank) * HN;
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) { ok = false; break; }
+          // the leader arms its full barrier for both CTAs' bytes; the peer's
+          // load only completes transactions on it
+          const uint32_t fb = lead(sm.full(s));
+          if (leader) mbar_arrive_expect_tx(sm.full(s), 2 * B_BYTES);
+          if (ks < p.k_main) tma_load_2d_pair(sm.b(s), &tmap_act, fb, ks * BK, t0);
+          else tma_load_2d_pair(sm.b(s), &tmap_lact, fb, (ks - p.k_main) * BK, t0);
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        // loads still in flight land in this CTA's shared memory; give them time to
+        // finish (their completion is counted in the leader's barrier, which this
+        // CTA cannot wait on)
+        const uint64_t t_end = globaltimer() + 2000000ull;
+        while (globaltimer() < t_end) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- dequantization: two groups, alternating stages ----------------
+    const int grp = (warp - 4) >> 2;          // 0: even stages, 1: odd stages
+    const int tid = threadIdx.x - 128 - 128 * grp;   // 0..127
+    float cb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cb[i] = p.codebook[i];
+    const int64_t kblocks = p.K / 64;
+    uint32_t row_off, phase;
+    if (!bwd) {
+      row_off = (tid >> 3) * 1024 + (tid & 7) * 128;
+      phase = tid & 7;
+    } else {
+      const int rho = tid & 63, h = tid >> 6;
+      row_off = ((rho >> 3) * 2 + h) * 1024 + (rho & 7) * 128;
+      phase = rho & 7;
+    }
+    int it_base = 0;
+    bool ok = true;
+    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+      const int m_pair = tile % m_pairs;
+      const int64_t row0 = static_cast<int64_t>(m_pair) * 2 * PM + static_cast<int64_t>(rank) * PM;
+      auto block_of = [&](int ks, int64_t &blk) -> bool {
+        int64_t n, kb;
+        if (!bwd) {
+          n = row0 + tid;
+          kb = ks;
+        } else {
+          n = static_cast<int64_t>(ks) * BK + (tid & 63);
+          kb = row0 / 64 + (tid >> 6);
+        }
+        blk = n * kblocks + kb;
+        return n < p.N && kb < kblocks;
+      };
+      auto fetch = [&](int ks) -> BlockIn {
+        int64_t blk = 0;
+        const bool v = ks < p.k_main && block_of(ks, blk);
+        return load_block(p, blk, v);
+      };
+      auto produce = [&](int ks, BlockIn &buf) -> bool {
+        const int it = it_base + ks;
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) return false;
+        const uint32_t row_addr = sm.a(s) + row_off;
+        if (ks < p.k_main) {
+          dequant_row(cb, buf, row_addr, phase);
+        } else {
+          const int l = ks - p.k_main;
+          if (!bwd) {
+            const int64_t n = row0 + tid;
+            const int nv = (n < p.N) ? max(0, min(BK, p.r - l * BK)) : 0;
+            const uint16_t *src = p.lora + (n < p.N ? n : 0) * p.r + l * BK;
+            copy_row(src, nv, (p.r % 8) == 0, row_addr, phase);
+          } else {
+            const int j = l * BK + (tid & 63);
+            const int64_t k0 = row0 + (tid >> 6) * 64;
+            const int nv = (j < p.r && k0 < p.K) ? 64 : 0;
+            const uint16_t *src = p.lora + static_cast<int64_t>(j < p.r ? j : 0) * p.K + (k0 < p.K ? k0 : 0);
+            copy_row(src, nv, true, row_addr, phase);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead(sm.full(s)));
+        buf = fetch(ks + 6);
+        return true;
+      };
+      // this group's stages of the tile: ks0, ks0 + 2, ks0 + 4, ... (three
+      // register buffers, each refilled in place six stages ahead)
+      const int ks0 = (grp - (it_base & 1)) & 1;
+      BlockIn r0 = fetch(ks0), r1 = fetch(ks0 + 2), r2 = fetch(ks0 + 4);
+      for (int ks = ks0; ks < ksteps && ok; ks += 6) {
+        ok = produce(ks, r0);
+        if (ok && ks + 2 < ksteps) ok = produce(ks + 2, r1);
+        if (ok && ks + 4 < ksteps) ok = produce(ks + 4, r2);
+      }
+      it_base += ksteps;
+    }
+    if (!ok) s_abort = 1;
+  } else {
+    // ---------------- epilogue (warps 0-3) ----------------
+    const int q = warp;
+    const bool issuer = (threadIdx.x == 0);
+    int tc = 0, chunk_count = 0;
+    bool ok = true;
+    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
+      const int m_pair = tile % m_pairs;
+      const int n_tile = tile / m_pairs;
+      const int acc = tc & 1;
+      const uint32_t acc_phase = (tc >> 1) & 1;
+      const bool fail = s_abort || !mbar_wait(sm.acc_full(acc), acc_phase, p.status);
+      if (named_bar_any(2, 128, fail)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * PN);
+      const int m_local = q * 32 + static_cast<int>(lane);
+      const int feat0 = m_pair * 2 * PM + static_cast<int>(rank) * PM;
+      for (int ch = 0; ch < PN / EPI_ROWS; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + ch * EPI_ROWS, r);
+        tc_wait_ld();
+        if (ch == PN / EPI_ROWS - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead(sm.acc_empty(acc)));
+        }
+        if (static_cast<int64_t>(n_tile) * PN + ch * EPI_ROWS >= p.T) continue;   // uniform
+        const int buf = chunk_count & 1;
+        if (issuer) tma_store_wait_read<1>();
+        named_bar_sync(1, 128);
+        const uint32_t stg = sm.epi(buf);
+#pragma unroll
+        for (int j = 0; j < EPI_ROWS; ++j) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+          st_shared_u16(stg + (j * PM + m_local) * 2, *reinterpret_cast<const uint16_t *>(&v));
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+          tma_store_2d(&tmap_out, stg, feat0, n_tile * PN + ch * EPI_ROWS);
+          tma_store_commit();
+        }
+        ++chunk_count;
+      }
+    }
+    if (!ok) s_abort = 1;
+    if (issuer) tma_store_wait_all<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive_wait();   // both CTAs are done with the pair's tensor memory
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+int gemm_2sm_smem_bytes() { return SMEM_ALLOC; }
+
+}  // namespace qlora

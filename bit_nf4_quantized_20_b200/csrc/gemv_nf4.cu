@@ -69,9 +69,11 @@ __device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank)
 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// a block as loaded; its scale is formed at use so that loads never wait
 struct Blk {
   uint4 c0, c1;
-  float scale;
+  uint32_t fbyte;
+  float c2;
 };
 
 template <int TT, int RG>
@@ -106,11 +108,13 @@ __global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
       const uint8_t *cp = p.codes + blk * 32;
       b.c0 = ldg_stream(cp);
       b.c1 = ldg_stream(cp + 16);
-      b.scale = __fmul_rn(e4m3_to_float(__ldg(p.scales + blk)), __ldg(p.c2 + (blk >> 8)));
+      b.fbyte = __ldg(p.scales + blk);
+      b.c2 = __ldg(p.c2 + (blk >> 8));
     } else {
       b.c0 = make_uint4(0, 0, 0, 0);
       b.c1 = b.c0;
-      b.scale = 0.f;
+      b.fbyte = 0u;
+      b.c2 = 0.f;
     }
     return b;
   };
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
     }
 #pragma unroll
     for (int rg = 0; rg < RG; ++rg) {
-      const Lut16 lut = make_lut16(cb, cur[rg].scale);
+      const Lut16 lut = make_lut16(cb, __fmul_rn(e4m3_to_float(cur[rg].fbyte), cur[rg].c2));
       const uint32_t w[8] = {cur[rg].c0.x, cur[rg].c0.y, cur[rg].c0.z, cur[rg].c0.w,
                              cur[rg].c1.x, cur[rg].c1.y, cur[rg].c1.z, cur[rg].c1.w};
 #pragma unroll

@@ -40,6 +40,11 @@ struct GemmParams {
   uint32_t *status;
 };
 int gemm_smem_bytes();
+int gemm_2sm_smem_bytes();
+// CTA-pair variant: m_tiles counts 256-row weight tiles; launched as clusters of 2.
+__global__ void nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                                    const __grid_constant__ CUtensorMap tmap_lact,
+                                    const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
 __global__ void nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                 const __grid_constant__ CUtensorMap tmap_lact,
                                 const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
