@@ -152,12 +152,38 @@ qlora_status check_weight(const qlora_nf4_weight *qw) {
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
+// codebook[15 - i] == -codebook[i] bit for bit (with codebook[7] < 0 < codebook[8])
+bool codebook_symmetric(const float *cb) {
+  for (int i = 0; i < 8; ++i) {
+    const float a = cb[i], b = -cb[15 - i];
+    if (memcmp(&a, &b, sizeof(float)) != 0) return false;
+  }
+  return cb[7] < 0.f && cb[8] > 0.f;
+}
+
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
+// Up to this many tokens the forward runs the decode GEMV, and U = s X A^T
+// runs on the mma.sync kernel (a handful of rows: latency, not bandwidth).
+constexpr int64_t kGemvMaxTokens = 16;
+
 struct WsLayout {
-  size_t counters = 0, su_hi = 0, su_lo = 0, du_hi = 0, du_lo = 0, partials = 0, total = 0;
+  size_t counters = 0;
+  size_t su_row = 0;                 // forward: sU [T, ceil64(r)] (rank-r operand of the GEMM / GEMV)
+  size_t suT_hi = 0, suT_lo = 0;     // backward: sU^T planes [r, ceil8(T)]
+  size_t du_row = 0;                 // backward: dU hi [T, ceil64(r)] (rank-r operand of the dX GEMM)
+  size_t duT_hi = 0, duT_lo = 0;     // backward: dU^T planes [r, ceil8(T)]
+  size_t bpad = 0;                   // backward: B copied to [N, ceil64(r)] when TMA cannot read it in place
+  size_t partials = 0, total = 0;
 };
+
+// The split geometry of each tensor-core rank-r product (sized for kSplitSms,
+// whatever the current device, so that workspace sizes are device-independent).
+SkinnyTcGeom geom_u(int64_t T, int64_t K, int r) { return skinny_tc_geom(T, K, r, 1, false, kSplitSms); }
+SkinnyTcGeom geom_du(int64_t T, int64_t N, int r) { return skinny_tc_geom(T, N, r, 1, true, kSplitSms); }
+SkinnyTcGeom geom_db(int64_t T, int64_t N, int r) { return skinny_tc_geom(N, T, r, 2, false, kSplitSms); }
+SkinnyTcGeom geom_da(int64_t T, int64_t K, int r) { return skinny_tc_geom(K, T, r, 2, false, kSplitSms); }
 
 WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   WsLayout L;
@@ -169,19 +195,25 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     return L;
   }
   const int64_t r64 = round_up(r, 64);
-  const size_t plane = static_cast<size_t>(round_up(T * r64 * 2, 256));
-  L.su_hi = off; off += plane;
-  L.su_lo = off; off += plane;
-  size_t part = skinny_partials_bytes(T, K, r, kSplitSms);
-  if (op == QLORA_OP_BWD) {
-    L.du_hi = off; off += plane;
-    L.du_lo = off; off += plane;
-    const size_t p2 = skinny_partials_bytes(T, N, r, kSplitSms);
-    const size_t p3 = skinny_partials_bytes(N, T, r, kSplitSms);
-    const size_t p4 = skinny_partials_bytes(K, T, r, kSplitSms);
-    if (p2 > part) part = p2;
-    if (p3 > part) part = p3;
-    if (p4 > part) part = p4;
+  const size_t row_plane = static_cast<size_t>(round_up(T * r64 * 2, 256));
+  const size_t t_plane = static_cast<size_t>(round_up(r * round_up(T, 8) * 2, 256));
+  size_t part = 0;
+  if (op == QLORA_OP_FWD) {
+    L.su_row = off; off += row_plane;
+    part = T <= kGemvMaxTokens ? skinny_partials_bytes(T, K, r, kSplitSms)
+                               : skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
+  } else {
+    L.suT_hi = off; off += t_plane;
+    L.suT_lo = off; off += t_plane;
+    L.du_row = off; off += row_plane;
+    L.duT_hi = off; off += t_plane;
+    L.duT_lo = off; off += t_plane;
+    L.bpad = off; off += static_cast<size_t>(round_up(N * r64 * 2, 256));
+    const size_t p[4] = {skinny_tc_partials_bytes(geom_u(T, K, r), T, r),
+                         skinny_tc_partials_bytes(geom_du(T, N, r), T, r),
+                         skinny_tc_partials_bytes(geom_db(T, N, r), N, r),
+                         skinny_tc_partials_bytes(geom_da(T, K, r), K, r)};
+    for (size_t v : p) part = v > part ? v : part;
   }
   L.partials = off;
   off += static_cast<size_t>(round_up(static_cast<int64_t>(part), 256));
@@ -189,6 +221,7 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   return L;
 }
 
+// Parameters of the mma.sync rank-r kernel (decode-sized U only).
 SkinnyParams skinny_base(int64_t M, int64_t C, int R, uint8_t *ws, const WsLayout &L) {
   SkinnyParams p;
   memset(&p, 0, sizeof(p));
@@ -243,6 +276,7 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   p.n_tiles = static_cast<int>((T + 255) / 256);
   p.k_main = static_cast<int>((Cext + 63) / 64);
   p.k_lora = static_cast<int>(r64 / 64);
+  p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
   p.status = status;
   const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
   const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
@@ -259,7 +293,7 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
     const int64_t clusters = tiles < sms / 2 ? tiles : sms / 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-    cfg.blockDim = dim3(448, 1, 1);
+    cfg.blockDim = dim3(576, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(gemm_2sm_smem_bytes());
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -288,7 +322,6 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
 
 // Token counts up to this use the decode-sized forward (register-fragment
 // dequantization, split-K over a thread block cluster).
-constexpr int64_t kGemvMaxTokens = 16;
 
 qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
                       const void *B, int r, void *y, cudaStream_t st) {
@@ -307,6 +340,7 @@ qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, cons
   p.B = static_cast<const uint16_t *>(B);
   p.r = r;
   p.y = static_cast<uint16_t *>(y);
+  p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
   const GemvPlan pl = gemv_plan(p.N, p.K, num_sms_current());
   const double n = static_cast<double>(p.N) * p.K;
   const double bytes = n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * T * (p.N + p.K) +
@@ -317,11 +351,60 @@ qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, cons
   return launch_gemv(p, pl, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-qlora_status run_skinny(int32_t kid, const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st) {
-  const double flops = 2.0 * p.M * p.C * p.R * (p.Q1 ? 2 : 1);
-  const double bytes = 2.0 * p.M * p.C;
-  TraceScope ts(kid, flops, bytes, st);
-  return launch_skinny(p, p_col, q_cj, out_mode, st) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+// One tensor-core rank-r product.  P: p_col ? [C rows, M cols] : [M rows, C cols]
+// (row stride ldp); Q planes: q_cj ? [C rows, R cols] : [R rows, C cols] (row
+// stride ldq).  All BF16 with TMA-legal (16-byte) row strides.
+struct TcProduct {
+  int32_t kid;
+  const void *P;
+  int64_t ldp;
+  bool p_col;
+  const void *Q0, *Q1;
+  int64_t ldq;
+  bool q_cj;
+  SkinnyTcGeom g;
+};
+
+qlora_status run_skinny_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
+  a.nq = t.Q1 ? 2 : 1;
+  a.p_col = t.p_col ? 1 : 0;
+  a.q_cj = t.q_cj ? 1 : 0;
+  a.nb = t.g.nb;
+  a.stages = t.g.stages;
+  a.splits = t.g.splits;
+  a.c_per_split = t.g.c_per_split;
+  a.partials = reinterpret_cast<float *>(ws + L.partials);
+  a.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+  a.status = reinterpret_cast<uint32_t *>(ws);
+  CUtensorMap tp, tq0, tq1;
+  const bool okp = t.p_col ? make_map_bf16(&tp, t.P, a.C, a.M, t.ldp, 64, 64, true)
+                           : make_map_bf16(&tp, t.P, a.M, a.C, t.ldp, 128, 64, true);
+  if (!okp) return QLORA_ERR_CUDA;
+  auto qmap = [&](CUtensorMap *m, const void *q) {
+    return t.q_cj ? make_map_bf16(m, q, a.C, a.R, t.ldq, 64, 64, true)
+                  : make_map_bf16(m, q, a.R, a.C, t.ldq, a.nb, 64, true);
+  };
+  if (!qmap(&tq0, t.Q0)) return QLORA_ERR_CUDA;
+  if (t.Q1) {
+    if (!qmap(&tq1, t.Q1)) return QLORA_ERR_CUDA;
+  } else {
+    tq1 = tq0;
+  }
+  const double flops = 2.0 * a.M * a.C * a.R * a.nq;
+  const double bytes = 2.0 * a.M * a.C;
+  const bool pdl = g_trace.recs == nullptr;
+  TraceScope ts(t.kid, flops, bytes, st);
+  return launch_skinny_tc(a, tp, tq0, tq1, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+SkinnyTcArgs tc_args(int64_t M, int64_t C, int R, float alpha) {
+  SkinnyTcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = M;
+  a.C = C;
+  a.R = R;
+  a.alpha = alpha;
+  return a;
 }
 
 }  // namespace
@@ -477,21 +560,32 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   const WsLayout L = ws_layout(QLORA_OP_FWD, T, N, K, r);
   const int64_t r64 = round_up(r, 64);
-  uint16_t *su_hi = reinterpret_cast<uint16_t *>(w8 + L.su_hi);
-  // U' = s X A^T (hi plane only: the forward reads it as the rank-r MMA operand)
-  SkinnyParams pu = skinny_base(T, K, r, w8, L);
-  pu.P = static_cast<const uint16_t *>(x);
-  pu.ldp = K;
-  pu.Q0 = static_cast<const uint16_t *>(A);
-  pu.ldq = K;
-  pu.alpha = s;
-  pu.out0 = su_hi;
-  pu.out1 = nullptr;
-  pu.ldo = r64;
-  qlora_status rs = run_skinny(K_LORA_U, pu, false, false, OUT_HILO, st);
+  uint16_t *su = reinterpret_cast<uint16_t *>(w8 + L.su_row);
+  // sU = s X A^T [T, ceil64(r)]: the rank-r operand of the GEMV / GEMM
+  if (T <= kGemvMaxTokens) {
+    // a handful of rows: the mma.sync kernel (latency, not bandwidth)
+    SkinnyParams pu = skinny_base(T, K, r, w8, L);
+    pu.P = static_cast<const uint16_t *>(x);
+    pu.ldp = K;
+    pu.Q0 = static_cast<const uint16_t *>(A);
+    pu.ldq = K;
+    pu.alpha = s;
+    pu.out0 = su;
+    pu.out1 = nullptr;
+    pu.ldo = r64;
+    {
+      TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * T * K, st);
+      if (launch_skinny(pu, false, false, OUT_HILO, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return run_gemv(qw, x, T, su, r64, B, r, y, st);
+  }
+  SkinnyTcArgs au = tc_args(T, K, r, s);
+  au.row_hi = su;
+  au.ldo = r64;
+  const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, geom_u(T, K, r)};
+  qlora_status rs = run_skinny_tc(tu, au, w8, L, st);
   if (rs != QLORA_OK) return rs;
-  if (T <= kGemvMaxTokens) return run_gemv(qw, x, T, su_hi, r64, B, r, y, st);
-  return run_gemm(0, qw, x, su_hi, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), st);
+  return run_gemm(0, qw, x, su, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), st);
 }
 
 qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
@@ -514,58 +608,53 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   const WsLayout L = ws_layout(QLORA_OP_BWD, T, N, K, r);
   const int64_t r64 = round_up(r, 64);
-  uint16_t *su_hi = reinterpret_cast<uint16_t *>(w8 + L.su_hi);
-  uint16_t *su_lo = reinterpret_cast<uint16_t *>(w8 + L.su_lo);
-  uint16_t *du_hi = reinterpret_cast<uint16_t *>(w8 + L.du_hi);
-  uint16_t *du_lo = reinterpret_cast<uint16_t *>(w8 + L.du_lo);
-  // sU = s X A^T, as hi + lo planes
-  SkinnyParams pu = skinny_base(T, K, r, w8, L);
-  pu.P = static_cast<const uint16_t *>(x);
-  pu.ldp = K;
-  pu.Q0 = static_cast<const uint16_t *>(A);
-  pu.ldq = K;
-  pu.alpha = s;
-  pu.out0 = su_hi;
-  pu.out1 = su_lo;
-  pu.ldo = r64;
-  qlora_status rs = run_skinny(K_LORA_U, pu, false, false, OUT_HILO, st);
+  const int64_t Tp = round_up(T, 8);
+  auto plane = [&](size_t off) { return reinterpret_cast<uint16_t *>(w8 + off); };
+  // sU = s X A^T, transposed, as hi + lo planes [r, ceil8(T)]
+  SkinnyTcArgs au = tc_args(T, K, r, s);
+  au.t_hi = plane(L.suT_hi);
+  au.t_lo = plane(L.suT_lo);
+  au.ldt = Tp;
+  const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, geom_u(T, K, r)};
+  qlora_status rs = run_skinny_tc(tu, au, w8, L, st);
   if (rs != QLORA_OK) return rs;
-  // dU = s dY B, as hi + lo planes
-  SkinnyParams pd = skinny_base(T, N, r, w8, L);
-  pd.P = static_cast<const uint16_t *>(dy);
-  pd.ldp = N;
-  pd.Q0 = static_cast<const uint16_t *>(B);
-  pd.ldq = r;
-  pd.alpha = s;
-  pd.out0 = du_hi;
-  pd.out1 = du_lo;
-  pd.ldo = r64;
-  rs = run_skinny(K_LORA_DU, pd, false, true, OUT_HILO, st);
+  // dU = s dY B: hi plane [T, ceil64(r)] for the dX GEMM, and transposed hi + lo
+  // planes for dA.  TMA reads B in place when its rows are a multiple of 16
+  // bytes (columns past r come back as zeros); otherwise B is first copied to
+  // [N, ceil64(r)] rows.
+  const void *bq = B;
+  int64_t ldb = r;
+  if (r % 8 != 0 || !aligned16(B)) {
+    uint16_t *bpad = plane(L.bpad);
+    if (launch_pad_cols(static_cast<const uint16_t *>(B), N, r, bpad, static_cast<int>(r64), st,
+                        num_sms_current()) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    bq = bpad;
+    ldb = r64;
+  }
+  SkinnyTcArgs ad = tc_args(T, N, r, s);
+  ad.row_hi = plane(L.du_row);
+  ad.ldo = r64;
+  ad.t_hi = plane(L.duT_hi);
+  ad.t_lo = plane(L.duT_lo);
+  ad.ldt = Tp;
+  const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, geom_du(T, N, r)};
+  rs = run_skinny_tc(td, ad, w8, L, st);
   if (rs != QLORA_OK) return rs;
   // dX = dY W' + dU A
-  rs = run_gemm(1, qw, dy, du_hi, r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
+  rs = run_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
   if (rs != QLORA_OK) return rs;
-  // dB = dY^T (sU)
-  SkinnyParams pb = skinny_base(N, T, r, w8, L);
-  pb.P = static_cast<const uint16_t *>(dy);
-  pb.ldp = N;
-  pb.Q0 = su_hi;
-  pb.Q1 = su_lo;
-  pb.ldq = r64;
-  pb.alpha = 1.0f;
-  pb.out0 = static_cast<uint16_t *>(dB);
-  rs = run_skinny(K_LORA_DB, pb, true, true, OUT_ROW, st);
+  // dB = dY^T (sU) [N, r]
+  SkinnyTcArgs ab = tc_args(N, T, r, 1.0f);
+  ab.row = static_cast<uint16_t *>(dB);
+  const TcProduct tb = {K_LORA_DB, dy, N, true, plane(L.suT_hi), plane(L.suT_lo), Tp, false, geom_db(T, N, r)};
+  rs = run_skinny_tc(tb, ab, w8, L, st);
   if (rs != QLORA_OK) return rs;
-  // dA = dU^T X
-  SkinnyParams pa = skinny_base(K, T, r, w8, L);
-  pa.P = static_cast<const uint16_t *>(x);
-  pa.ldp = K;
-  pa.Q0 = du_hi;
-  pa.Q1 = du_lo;
-  pa.ldq = r64;
-  pa.alpha = 1.0f;
-  pa.out0 = static_cast<uint16_t *>(dA);
-  return run_skinny(K_LORA_DA, pa, true, true, OUT_T, st);
+  // dA = dU^T X [r, K]
+  SkinnyTcArgs aa = tc_args(K, T, r, 1.0f);
+  aa.tr = static_cast<uint16_t *>(dA);
+  const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, geom_da(T, K, r)};
+  return run_skinny_tc(ta, aa, w8, L, st);
 }
 
 // ---------------------------------------------------------------------------

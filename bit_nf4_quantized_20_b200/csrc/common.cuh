@@ -253,6 +253,15 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // ---------------------------------------------------------------------------
 // Thread block clusters and the 2-SM (cta_group::2) forms
 // ---------------------------------------------------------------------------
@@ -425,6 +434,47 @@ __device__ __forceinline__ void lut16_lookup4(const Lut16 &t, uint32_t sel, uint
   const uint32_t m = prmt(sel << 4, sel, 0xD9C8u);
   const uint32_t lo = lop3_select(prmt(t.lo[0], t.lo[1], idx), prmt(t.lo[2], t.lo[3], idx), m);
   const uint32_t hi = lop3_select(prmt(t.hi[0], t.hi[1], idx), prmt(t.hi[2], t.hi[3], idx), m);
+  out0 = prmt(lo, hi, 0x5140u);
+  out1 = prmt(lo, hi, 0x7362u);
+}
+
+// A codebook is "symmetric" when codebook[15 - i] == -codebook[i] bit for bit
+// (eq. 2's NF4 levels are).  Then BF16(RN32(q[c] * s)) for c < 8 is the exact
+// negation of the entry for 15 - c (negation and round-to-nearest-even commute),
+// so eight magnitudes and a sign bit give all sixteen entries.
+struct Lut8 {
+  uint32_t lo[2];   // low bytes of |entry(8 + j)|, j = 0..7
+  uint32_t hi[2];   // high bytes (sign bit clear)
+};
+
+__device__ __forceinline__ Lut8 make_lut8(const float (&cb)[16], float scale) {
+  uint32_t p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = pack_bf16x2(__fmul_rn(cb[8 + 2 * i], scale), __fmul_rn(cb[9 + 2 * i], scale));
+  Lut8 t;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    t.lo[i] = prmt(p[2 * i], p[2 * i + 1], 0x6420);
+    t.hi[i] = prmt(p[2 * i], p[2 * i + 1], 0x7531);
+  }
+  return t;
+}
+
+// Magnitude indices of eight codes: c >= 8 -> c - 8, c < 8 -> 7 - c.
+__device__ __forceinline__ uint32_t mag_index8(uint32_t w) {
+  const uint32_t neg = ~(w >> 3) & 0x11111111u;   // 1 in each nibble whose code is < 8
+  return (w ^ (neg * 7u)) & 0x77777777u;
+}
+
+// Four codes in bits 0-15 of `codes` (their magnitude indices in bits 0-15 of
+// `mag`): out0 = (entry(c0), entry(c1)), out1 = (entry(c2), entry(c3)).
+__device__ __forceinline__ void lut8_lookup4(const Lut8 &t, uint32_t codes, uint32_t mag, uint32_t &out0,
+                                             uint32_t &out1) {
+  const uint32_t lo = prmt(t.lo[0], t.lo[1], mag);
+  uint32_t hi = prmt(t.hi[0], t.hi[1], mag);
+  // byte i of m = 0xFF when code i >= 8 (sign-replicate mode of prmt on bit 3)
+  const uint32_t m = prmt(codes << 4, codes, 0xD9C8u);
+  hi |= ~m & 0x80808080u;   // negative entries for codes below 8
   out0 = prmt(lo, hi, 0x5140u);
   out1 = prmt(lo, hi, 0x7362u);
 }

@@ -77,16 +77,30 @@ __device__ __forceinline__ BlockIn load_block(const GemmParams &p, int64_t blk, 
 }
 
 // Dequantize one block into one 128-byte swizzled shared-memory row.
+template <bool SYM>
 __device__ __forceinline__ void dequant_row(const float (&cb)[16], const BlockIn &in, uint32_t row_addr,
                                             uint32_t phase) {
-  const Lut16 lut = make_lut16(cb, __fmul_rn(e4m3_to_float(in.fbyte), in.c2));
+  const float scale = __fmul_rn(e4m3_to_float(in.fbyte), in.c2);
   const uint32_t w[8] = {in.c0.x, in.c0.y, in.c0.z, in.c0.w, in.c1.x, in.c1.y, in.c1.z, in.c1.w};
+  if (SYM) {
+    const Lut8 lut = make_lut8(cb, scale);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t o0, o1, o2, o3;
-    lut16_lookup4(lut, w[c], o0, o1);
-    lut16_lookup4(lut, w[c] >> 16, o2, o3);
-    st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
+    for (int c = 0; c < 8; ++c) {
+      uint32_t o0, o1, o2, o3;
+      const uint32_t mag = mag_index8(w[c]);
+      lut8_lookup4(lut, w[c], mag, o0, o1);
+      lut8_lookup4(lut, w[c] >> 16, mag >> 16, o2, o3);
+      st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
+    }
+  } else {
+    const Lut16 lut = make_lut16(cb, scale);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t o0, o1, o2, o3;
+      lut16_lookup4(lut, w[c], o0, o1);
+      lut16_lookup4(lut, w[c] >> 16, o2, o3);
+      st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
+    }
   }
 }
 

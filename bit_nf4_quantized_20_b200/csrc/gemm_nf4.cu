@@ -235,7 +235,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) return false;
         const uint32_t row_addr = sm.a(s) + row_off;
         if (ks < p.k_main) {
-          dequant_row(cb, buf, row_addr, phase);
+          if (p.sym) dequant_row<true>(cb, buf, row_addr, phase);
+          else dequant_row<false>(cb, buf, row_addr, phase);
         } else {
           const int l = ks - p.k_main;
           if (!bwd) {

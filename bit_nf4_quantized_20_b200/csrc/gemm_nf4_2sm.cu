@@ -16,12 +16,12 @@
 // Compared with one CTA per 128 x 256 tile this halves the token operand each
 // SM streams from L2 per FLOP.
 //
-// Warp roles (448 threads per CTA, one CTA per SM, persistent over tiles):
+// Warp roles (576 threads per CTA, one CTA per SM, persistent over tiles):
 //   warps 0-3   epilogue: tensor memory -> BF16 -> shared memory -> TMA store
-//   warps 4-7   dequantization, even pipeline stages
-//   warps 8-11  dequantization, odd pipeline stages
-//   warp 12     TMA loads of this CTA's token half (X / dY, then s*U / dU)
-//   warp 13     paired tensor-memory allocation; on the even CTA, the MMA issue
+//   warps 4-15  dequantization in three groups of four warps; group g fills the
+//               pipeline stages it with it % 3 == g
+//   warp 16     TMA loads of this CTA's token half (X / dY, then s*U / dU)
+//   warp 17     paired tensor-memory allocation; on the even CTA, the MMA issue
 // Pipeline barriers: full[s] lives in the even CTA and counts both CTAs' TMA
 // bytes (armed by the even CTA) and both CTAs' dequantization warps; empty[s] and acc_full are signalled in both
 // CTAs by a multicast tcgen05.commit; acc_empty (even CTA) counts both CTAs'
@@ -48,7 +48,8 @@ constexpr int A_BYTES = PM * BK * 2;           // 16 KiB
 constexpr int B_BYTES = HN * BK * 2;           // 16 KiB
 constexpr int EPI_ROWS = 32;
 constexpr int EPI_BYTES = EPI_ROWS * PM * 2;   // 8 KiB
-constexpr int NUM_THREADS = 448;
+constexpr int NUM_THREADS = 576;
+constexpr int DQ_GROUPS = 3;          // STAGES is a multiple of it
 constexpr int TMEM_COLS = 512;
 
 constexpr int OFF_A = 0;
@@ -112,12 +113,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(sm.drain(), 1);
     fence_mbar_init();
   }
-  if (warp == 12 && lane == 0) {
+  if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tmap_act);
     tma_prefetch_desc(&tmap_lact);
     tma_prefetch_desc(&tmap_out);
   }
-  if (warp == 13) {
+  if (warp == 17) {
     tmem_alloc_pair(sm.tmem_slot(), TMEM_COLS);
     tmem_relinquish_pair();
   }
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = ld_shared_u32(sm.tmem_slot());
   auto lead = [&](uint32_t local_addr) { return mapa_shared(local_addr, 0); };
 
-  if (warp == 13) {
+  if (warp == 17) {
     // ---------------- MMA issuer (even CTA) ----------------
     if (leader && lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, bwd, false);
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(sm.drain(), 0, p.status);
     }
     __syncwarp();
-  } else if (warp == 12) {
+  } else if (warp == 16) {
     // ---------------- TMA producer: this CTA's token half ----------------
     if (lane == 0) {
       int it = 0;
@@ -195,8 +196,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- dequantization: two groups, alternating stages ----------------
-    const int grp = (warp - 4) >> 2;          // 0: even stages, 1: odd stages
+    // ---------------- dequantization: three groups, rotating stages ----------------
+    const int grp = (warp - 4) >> 2;                 // group g fills stages it % 3 == g
     const int tid = threadIdx.x - 128 - 128 * grp;   // 0..127
     float cb[16];
 #pragma unroll
@@ -240,7 +241,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (s_abort || !mbar_wait(sm.empty(s), ph ^ 1, p.status)) return false;
         const uint32_t row_addr = sm.a(s) + row_off;
         if (ks < p.k_main) {
-          dequant_row(cb, buf, row_addr, phase);
+          if (p.sym) dequant_row<true>(cb, buf, row_addr, phase);
+          else dequant_row<false>(cb, buf, row_addr, phase);
         } else {
           const int l = ks - p.k_main;
           if (!bwd) {
@@ -259,17 +261,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead(sm.full(s)));
-        buf = fetch(ks + 6);
+        buf = fetch(ks + 2 * DQ_GROUPS);
         return true;
       };
-      // this group's stages of the tile: ks0, ks0 + 2, ks0 + 4, ... (three
+      // this group's stages of the tile: ks0, ks0 + 3, ks0 + 6, ... (two
       // register buffers, each refilled in place six stages ahead)
-      const int ks0 = (grp - (it_base & 1)) & 1;
-      BlockIn r0 = fetch(ks0), r1 = fetch(ks0 + 2), r2 = fetch(ks0 + 4);
-      for (int ks = ks0; ks < ksteps && ok; ks += 6) {
+      const int ks0 = (grp - (it_base % DQ_GROUPS) + DQ_GROUPS) % DQ_GROUPS;
+      BlockIn r0 = fetch(ks0), r1 = fetch(ks0 + DQ_GROUPS);
+      for (int ks = ks0; ks < ksteps && ok; ks += 2 * DQ_GROUPS) {
         ok = produce(ks, r0);
-        if (ok && ks + 2 < ksteps) ok = produce(ks + 2, r1);
-        if (ok && ks + 4 < ksteps) ok = produce(ks + 4, r2);
+        if (ok && ks + DQ_GROUPS < ksteps) ok = produce(ks + DQ_GROUPS, r1);
       }
       it_base += ksteps;
     }
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   cluster_arrive_wait();   // both CTAs are done with the pair's tensor memory
-  if (warp == 13) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }

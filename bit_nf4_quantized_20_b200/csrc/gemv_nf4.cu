@@ -76,7 +76,7 @@ struct Blk {
   float c2;
 };
 
-template <int TT, int RG>
+template <int TT, int RG, bool SYM>
 __global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
   __shared__ float s_red[GW][TT][8 * RG];
   __shared__ float s_part[TT][8 * RG];
@@ -167,16 +167,33 @@ __global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
     }
 #pragma unroll
     for (int rg = 0; rg < RG; ++rg) {
-      const Lut16 lut = make_lut16(cb, __fmul_rn(e4m3_to_float(cur[rg].fbyte), cur[rg].c2));
+      const float scale = __fmul_rn(e4m3_to_float(cur[rg].fbyte), cur[rg].c2);
       const uint32_t w[8] = {cur[rg].c0.x, cur[rg].c0.y, cur[rg].c0.z, cur[rg].c0.w,
                              cur[rg].c1.x, cur[rg].c1.y, cur[rg].c1.z, cur[rg].c1.w};
+      if (SYM) {
+        const Lut8 lut = make_lut8(cb, scale);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        uint32_t b0, b1;
-        lut16_lookup4(lut, (i & 1) ? (w[i >> 1] >> 16) : w[i >> 1], b0, b1);
-        const uint32_t a1 = (TT == 16) ? xb[2 * i] : 0u;
-        const uint32_t a3 = (TT == 16) ? xb[2 * i + 1] : 0u;
-        mma16816(acc[rg], xa[2 * i], a1, xa[2 * i + 1], a3, b0, b1);
+        for (int h = 0; h < 8; ++h) {
+          const uint32_t mag = mag_index8(w[h]);
+          uint32_t b0, b1, b2, b3;
+          lut8_lookup4(lut, w[h], mag, b0, b1);
+          lut8_lookup4(lut, w[h] >> 16, mag >> 16, b2, b3);
+          const int i = 2 * h;
+          mma16816(acc[rg], xa[2 * i], (TT == 16) ? xb[2 * i] : 0u, xa[2 * i + 1], (TT == 16) ? xb[2 * i + 1] : 0u,
+                   b0, b1);
+          mma16816(acc[rg], xa[2 * i + 2], (TT == 16) ? xb[2 * i + 2] : 0u, xa[2 * i + 3],
+                   (TT == 16) ? xb[2 * i + 3] : 0u, b2, b3);
+        }
+      } else {
+        const Lut16 lut = make_lut16(cb, scale);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          uint32_t b0, b1;
+          lut16_lookup4(lut, (i & 1) ? (w[i >> 1] >> 16) : w[i >> 1], b0, b1);
+          const uint32_t a1 = (TT == 16) ? xb[2 * i] : 0u;
+          const uint32_t a3 = (TT == 16) ? xb[2 * i + 1] : 0u;
+          mma16816(acc[rg], xa[2 * i], a1, xa[2 * i + 1], a3, b0, b1);
+        }
       }
     }
 #pragma unroll
@@ -249,7 +266,7 @@ __global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
   if (S > 1) cluster_sync();   // peers keep their shared memory alive until rank 0 has read it
 }
 
-template <int TT, int RG>
+template <int TT, int RG, bool SYM>
 cudaError_t launch_tr(const GemvParams &p, int row_tiles, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(row_tiles * p.splits), 1, 1);
@@ -270,7 +287,7 @@ cudaError_t launch_tr(const GemvParams &p, int row_tiles, cudaStream_t st, bool 
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<TT, RG>, p);
+  return cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<TT, RG, SYM>, p);
 }
 
 }  // namespace
@@ -304,8 +321,12 @@ cudaError_t launch_gemv(const GemvParams &p_in, const GemvPlan &pl, cudaStream_t
   p.upw = pl.upw;
   p.splits = pl.splits;
   const bool t16 = p.T > 8;
-  if (pl.rg == 2) return t16 ? launch_tr<16, 2>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2>(p, pl.row_tiles, st, pdl);
-  return t16 ? launch_tr<16, 1>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1>(p, pl.row_tiles, st, pdl);
+  if (p.sym) {
+    if (pl.rg == 2) return t16 ? launch_tr<16, 2, true>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2, true>(p, pl.row_tiles, st, pdl);
+    return t16 ? launch_tr<16, 1, true>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1, true>(p, pl.row_tiles, st, pdl);
+  }
+  if (pl.rg == 2) return t16 ? launch_tr<16, 2, false>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2, false>(p, pl.row_tiles, st, pdl);
+  return t16 ? launch_tr<16, 1, false>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1, false>(p, pl.row_tiles, st, pdl);
 }
 
 }  // namespace qlora

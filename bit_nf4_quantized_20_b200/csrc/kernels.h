@@ -37,6 +37,7 @@ struct GemmParams {
   int r;
   int m_tiles, n_tiles;    // weight-side tiles of 128, token tiles of 256
   int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part
+  int sym;                 // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   uint32_t *status;
 };
 int gemm_smem_bytes();
@@ -65,6 +66,7 @@ struct GemvParams {
   const uint16_t *B;     // [N, r]
   int r;
   uint16_t *y;           // [T, N]
+  int sym;               // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   int units, upw, splits;  // filled from the plan
 };
 struct GemvPlan {
@@ -105,6 +107,45 @@ struct SkinnyParams {
   uint32_t *counters;  // one per 64-row tile when splits > 1 (zero on entry, zero on exit)
   uint32_t *status;
 };
+
+// The same products on tcgen05 (skinny_tc.cu): P and Q arrive by TMA, the
+// accumulator (128 rows x NB columns, FP32) lives in tensor memory.
+struct SkinnyTcGeom {
+  int nb;               // MMA N: R rounded up to 16, 32, 64 or 128 (64 or 128 for MN-major Q)
+  int stages;           // TMA pipeline depth
+  int smem;             // dynamic shared memory bytes
+  int splits;           // contraction splits (CTAs per 128-row tile)
+  int64_t c_per_split;  // multiple of 64
+};
+// nq: Q planes (1, or 2 for hi + lo); q_cj: Q stored [c][j] (MN-major) else [j][c].
+SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int num_sms);
+size_t skinny_tc_partials_bytes(const SkinnyTcGeom &g, int64_t M, int R);
+
+struct SkinnyTcArgs {
+  int64_t M, C;          // rows of the result, contraction length
+  int R;                 // result columns (<= 128)
+  int nq;                // Q planes summed into one accumulator
+  int p_col;             // P stored [c][m] (MN-major A) else [m][c] (K-major A)
+  int q_cj;              // Q stored [c][j] (MN-major B) else [j][c] (K-major B)
+  int nb, stages, splits;
+  int64_t c_per_split;
+  float alpha;
+  // outputs (nullptr = not written); v = alpha * C[m, j]
+  uint16_t *row_hi;      // [M, ldo] bf16(v), columns R..ldo-1 zero
+  int64_t ldo;
+  uint16_t *t_hi;        // [R, ldt] bf16(v) transposed
+  uint16_t *t_lo;        // [R, ldt] bf16(v - bf16(v)) transposed
+  int64_t ldt;
+  uint16_t *row;         // [M, R] bf16(v)
+  uint16_t *tr;          // [R, M] bf16(v)
+  float *partials;       // [splits][M][(R + 3) & ~3] when splits > 1
+  uint32_t *counters;    // one per 128-row tile (zero on entry, zero on exit)
+  uint32_t *status;
+};
+cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
+                             const CUtensorMap &tm_q1, cudaStream_t st, bool pdl);
+cudaError_t launch_pad_cols(const uint16_t *src, int64_t rows, int cols, uint16_t *dst, int ldd, cudaStream_t st,
+                            int num_sms);
 
 // p_col: P stored as [c][m] (else [m][c]); q_cj: Q stored as [c][j] (else [j][c]).
 cudaError_t launch_skinny(const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st);

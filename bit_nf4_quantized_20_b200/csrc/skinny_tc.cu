@@ -1,0 +1,421 @@
+// skinny_tc.cu -- the rank-r GEMMs of the LoRA adapter on the 5th-generation
+// tensor cores ("QLoRA: Efficient Fine-Tuning", Step 3 eq. 3 and Step 4 eq. 5):
+//
+//   U  = s X A^T      [T, r]   P = X  [t][k] (K-major),            Q = A     [j][k] (K-major)
+//   dU = s dY B       [T, r]   P = dY [t][n] (K-major),            Q = B     [n][j] (MN-major)
+//   dB = dY^T (sU)    [N, r]   P = dY [t][n] as [c][m] (MN-major), Q = sU^T  [j][t] planes (K-major)
+//   dA = dU^T X       [r, K]   P = X  [t][k] as [c][m] (MN-major), Q = dU^T  [j][t] planes (K-major)
+//
+// C[M, R] = alpha * sum_c P(m, c) Q(c, j): the large operand P streams from HBM
+// through a TMA pipeline in 128-row tiles (the MMA's M), the rank-r operand Q
+// (R rounded up to NB = 16, 32, 64 or 128 columns, the MMA's N; rows past R
+// arrive as zeros) rides along, and the FP32 accumulator sits in tensor
+// memory.  U and dU are also written transposed as two BF16 planes hi = bf16(v),
+// lo = bf16(v - hi), which dB and dA take as two MMAs into one accumulator.
+// The contraction is split across CTAs so that the grid fills the GPU in one
+// wave (two CTAs per SM); each split writes an FP32 partial tile and the last
+// CTA of a row tile (a workspace counter, reset by that CTA) sums the partials
+// in split order and writes the outputs.
+//
+// Launched as a programmatic dependent: the prologue (barriers, tensor memory,
+// descriptor prefetch) overlaps the previous kernel, and every global access
+// comes after griddepcontrol.wait.
+//
+// Warps: 0 TMA producer, 1 tensor-memory allocation + MMA issue, 2-5 epilogue.
+
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+using namespace gemm;
+
+namespace {
+
+constexpr int TBM = 128;                 // rows of P per CTA (MMA M)
+constexpr int TBK = 64;                  // contraction per stage
+constexpr int TMAX_STAGES = 8;
+constexpr int P_BYTES = TBM * TBK * 2;   // 16 KiB
+constexpr int TNUM_THREADS = 192;
+constexpr int kBarBytes = 8 * (2 * TMAX_STAGES + 1) + 8;   // full[], empty[], accumulator, tensor-memory slot
+constexpr int kFixedSmem = kBarBytes + 1024;               // + alignment slack for the 1 KiB swizzle atoms
+constexpr int kTwoPerSmBudget = 110 * 1024;
+constexpr int kOnePerSmBudget = 220 * 1024;
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Columns c0 .. c0 + CW - 1 of row m: v[j] is the un-scaled accumulator.
+template <int CW>
+__device__ __forceinline__ void emit_chunk(const SkinnyTcArgs &a, int64_t m, int c0, const float (&v)[CW]) {
+  if (a.row_hi) {
+    uint16_t *h = a.row_hi + m * a.ldo + c0;
+#pragma unroll
+    for (int g = 0; g < CW; g += 8) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float x0 = (c0 + g + e < a.R) ? a.alpha * v[g + e] : 0.f;
+        const float x1 = (c0 + g + e + 1 < a.R) ? a.alpha * v[g + e + 1] : 0.f;
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(x0, x1);
+        w[e / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+      }
+      *reinterpret_cast<uint4 *>(h + g) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < CW; ++j) {
+    const int c = c0 + j;
+    if (c < a.R) {
+      const float x = a.alpha * v[j];
+      const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+      const uint16_t hu = *reinterpret_cast<const uint16_t *>(&hb);
+      if (a.t_hi) {
+        a.t_hi[static_cast<int64_t>(c) * a.ldt + m] = hu;
+        const __nv_bfloat16 lb = __float2bfloat16_rn(x - __bfloat162float(hb));
+        a.t_lo[static_cast<int64_t>(c) * a.ldt + m] = *reinterpret_cast<const uint16_t *>(&lb);
+      }
+      if (a.row) a.row[m * a.R + c] = hu;
+      if (a.tr) a.tr[static_cast<int64_t>(c) * a.M + m] = hu;
+    }
+  }
+}
+
+template <int CW>
+__device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, float (&v)[CW]) {
+  uint32_t r[CW];
+  if constexpr (CW == 16) {
+    tmem_ld_32x32b_x16(taddr, r);
+  } else {
+    tmem_ld_32x32b_x32(taddr, r);
+  }
+  tc_wait_ld();
+#pragma unroll
+  for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+}  // namespace
+
+template <int NB>
+__global__ void __launch_bounds__(TNUM_THREADS, 2)
+    skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q0,
+                     const __grid_constant__ CUtensorMap tm_q1, const SkinnyTcArgs a) {
+  grid_dep_launch();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  constexpr int CW = NB < 32 ? NB : 32;                  // epilogue chunk (columns)
+  constexpr uint32_t TMEM_COLS = NB < 32 ? 32u : static_cast<uint32_t>(NB);
+  constexpr uint32_t Q_BYTES = NB * TBK * 2;
+  const int NS = a.stages;
+  const uint32_t stage_bytes = P_BYTES + a.nq * Q_BYTES;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t bar0 = base + NS * stage_bytes;
+  auto stage_p = [&](int s) { return base + s * stage_bytes; };
+  auto stage_q = [&](int s, int qi) { return base + s * stage_bytes + P_BYTES + qi * Q_BYTES; };
+  auto full = [&](int s) { return bar0 + 8 * s; };
+  auto empty = [&](int s) { return bar0 + 8 * (TMAX_STAGES + s); };
+  const uint32_t acc_bar = bar0 + 8 * (2 * TMAX_STAGES);
+  const uint32_t tmem_slot = acc_bar + 8;
+  __shared__ int s_last;
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  const int m_tile = blockIdx.x;
+  const int split = blockIdx.y;
+  const int64_t m0 = static_cast<int64_t>(m_tile) * TBM;
+  const int64_t cbeg = static_cast<int64_t>(split) * a.c_per_split;
+  const int64_t cend = min(a.C, cbeg + a.c_per_split);
+  const int nst = static_cast<int>((cend - cbeg + TBK - 1) / TBK);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(acc_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_p);
+    tma_prefetch_desc(&tm_q0);
+    if (a.nq > 1) tma_prefetch_desc(&tm_q1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ld_shared_u32(tmem_slot);
+  grid_dep_wait();
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % NS;
+        const uint32_t ph = (st / NS) & 1;
+        if (s_abort || !mbar_wait(empty(s), ph ^ 1, a.status)) {
+          s_abort = 1;
+          break;
+        }
+        const int32_t c0 = static_cast<int32_t>(cbeg + static_cast<int64_t>(st) * TBK);
+        mbar_arrive_expect_tx(full(s), stage_bytes);
+        if (!a.p_col) {
+          tma_load_2d(stage_p(s), &tm_p, full(s), c0, static_cast<int32_t>(m0));                     // [128 m][64 c]
+        } else {
+          tma_load_2d(stage_p(s), &tm_p, full(s), static_cast<int32_t>(m0), c0);                     // m 0-63
+          tma_load_2d(stage_p(s) + P_BYTES / 2, &tm_p, full(s), static_cast<int32_t>(m0) + 64, c0);  // m 64-127
+        }
+        for (int qi = 0; qi < a.nq; ++qi) {
+          const CUtensorMap *tq = qi ? &tm_q1 : &tm_q0;
+          if (!a.q_cj) {
+            tma_load_2d(stage_q(s, qi), tq, full(s), c0, 0);                                          // [NB j][64 c]
+          } else {
+            for (int h = 0; h < NB / 64; ++h)
+              tma_load_2d(stage_q(s, qi) + h * (TBK * 128), tq, full(s), h * 64, c0);                 // [64 c][64 j]
+          }
+        }
+        issued = st + 1;
+      }
+      if (s_abort) {
+        for (int st = max(0, issued - NS); st < issued; ++st)
+          mbar_wait(full(st % NS), (st / NS) & 1, a.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issue ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(TBM, static_cast<uint32_t>(NB), a.p_col != 0, a.q_cj != 0);
+      bool ok = true;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % NS;
+        const uint32_t ph = (st / NS) & 1;
+        if (!mbar_wait(full(s), ph, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = !a.p_col ? smem_desc_sw128(stage_p(s) + kk * 32, 16, 1024)
+                                       : smem_desc_sw128(stage_p(s) + kk * 2048, P_BYTES / 2, 1024);
+          for (int qi = 0; qi < a.nq; ++qi) {
+            const uint64_t bd = !a.q_cj ? smem_desc_sw128(stage_q(s, qi) + kk * 32, 16, 1024)
+                                        : smem_desc_sw128(stage_q(s, qi) + kk * 2048, TBK * 128, 1024);
+            tc_mma_ss(tmem, ad, bd, idesc, (st > 0 || kk > 0 || qi > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(empty(s));
+      }
+      if (!ok) s_abort = 1;
+      tc_commit(acc_bar);   // also drains: arrives once everything issued has completed
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: row m of the tile per thread ----------------
+    const int q = warp & 3;                       // tensor-memory lane quarter
+    const int row = q * 32 + static_cast<int>(lane);
+    const int64_t m = m0 + row;
+    const bool fail = !mbar_wait(acc_bar, 0, a.status) || s_abort;
+    // tcgen05.ld is warp-collective: the decision must be uniform within the warp
+    const bool have = __all_sync(0xffffffffu, !fail && nst > 0);
+    tc_fence_after();
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int pw = (a.R + 3) & ~3;      // partial row width (the R meaningful columns, float4 granular)
+    float v[CW];
+    if (a.splits > 1) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < NB; c0 += CW) {
+        if (have) {
+          tmem_load_chunk<CW>(trow + c0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] = 0.f;
+        }
+        if (m < a.M) {
+          float4 *dst = reinterpret_cast<float4 *>(a.partials + (static_cast<int64_t>(split) * a.M + m) * pw + c0);
+#pragma unroll
+          for (int g = 0; g < CW / 4; ++g)
+            if (c0 + 4 * g < pw) dst[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) {
+        const uint32_t old = atomicAdd(a.counters + m_tile, 1u);
+        s_last = (old == static_cast<uint32_t>(a.splits - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (s_last) {
+        __threadfence();
+        if (m < a.M) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < NB; c0 += CW) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) v[j] = 0.f;
+            for (int sp = 0; sp < a.splits; ++sp) {
+              const float4 *src =
+                  reinterpret_cast<const float4 *>(a.partials + (static_cast<int64_t>(sp) * a.M + m) * pw + c0);
+#pragma unroll
+              for (int g = 0; g < CW / 4; ++g) {
+                if (c0 + 4 * g < pw) {
+                  const float4 t4 = __ldcg(src + g);
+                  v[4 * g] += t4.x;
+                  v[4 * g + 1] += t4.y;
+                  v[4 * g + 2] += t4.z;
+                  v[4 * g + 3] += t4.w;
+                }
+              }
+            }
+            emit_chunk<CW>(a, m, c0, v);
+          }
+        }
+        if (threadIdx.x == 64) a.counters[m_tile] = 0u;
+      }
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < NB; c0 += CW) {
+        if (have) {   // warp-uniform
+          tmem_load_chunk<CW>(trow + c0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] = 0.f;
+        }
+        if (m < a.M) emit_chunk<CW>(a, m, c0, v);
+      }
+    }
+    // the rest of a padded row of the hi plane (columns NB .. ldo - 1) is zero
+    if (a.row_hi && m < a.M && (a.splits == 1 || s_last)) {
+      for (int64_t c = NB; c < a.ldo; c += 8)
+        *reinterpret_cast<uint4 *>(a.row_hi + m * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// One thread writes 8 consecutive outputs (one 16-byte store); ldd is a
+// multiple of 8.
+__global__ void pad_cols_kernel(const uint16_t *__restrict__ src, int64_t rows, int cols, uint16_t *__restrict__ dst,
+                                int ldd) {
+  const int per_row = ldd >> 3;
+  const int64_t n = rows * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / per_row;
+    const int c0 = static_cast<int>(i - r * per_row) << 3;
+    const uint16_t *s = src + r * cols;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c0 + 2 * e;
+      const uint32_t lo = c < cols ? s[c] : 0u;
+      const uint32_t hi = c + 1 < cols ? s[c + 1] : 0u;
+      w[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst + r * ldd + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int num_sms) {
+  SkinnyTcGeom g;
+  if (q_cj) {
+    g.nb = R <= 64 ? 64 : 128;
+  } else {
+    g.nb = R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128;
+  }
+  const int stage = P_BYTES + nq * g.nb * TBK * 2;
+  int per_sm = 2;
+  int stages = (kTwoPerSmBudget - kFixedSmem) / stage;
+  if (stages < 3) {
+    per_sm = 1;
+    stages = (kOnePerSmBudget - kFixedSmem) / stage;
+  }
+  if (stages > TMAX_STAGES) stages = TMAX_STAGES;
+  g.stages = stages;
+  g.smem = stages * stage + kFixedSmem;
+  g.splits = 1;
+  g.c_per_split = TBK;
+  if (M <= 0 || C <= 0 || num_sms <= 0) return g;
+  // one wave: m_tiles x splits <= the CTAs the GPU holds at once
+  const int64_t m_tiles = (M + TBM - 1) / TBM;
+  int64_t s = static_cast<int64_t>(per_sm) * num_sms / m_tiles;
+  const int64_t cap = (C + 2 * TBK - 1) / (2 * TBK);      // at least two stages per split
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  int64_t per = (C + s - 1) / s;
+  per = (per + TBK - 1) / TBK * TBK;
+  g.c_per_split = per;
+  g.splits = static_cast<int>((C + per - 1) / per);
+  return g;
+}
+
+size_t skinny_tc_partials_bytes(const SkinnyTcGeom &g, int64_t M, int R) {
+  if (g.splits <= 1 || M <= 0) return 0;
+  return static_cast<size_t>(g.splits) * static_cast<size_t>(M) * static_cast<size_t>((R + 3) & ~3) * sizeof(float);
+}
+
+namespace {
+template <int NB>
+cudaError_t launch_nb(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
+                      const CUtensorMap &tm_q1, cudaStream_t st, bool pdl) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(skinny_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kOnePerSmBudget);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int stage = P_BYTES + a.nq * NB * TBK * 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((a.M + TBM - 1) / TBM), static_cast<unsigned>(a.splits), 1);
+  cfg.blockDim = dim3(TNUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(a.stages * stage + kFixedSmem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, skinny_tc_kernel<NB>, tm_p, tm_q0, tm_q1, a);
+}
+}  // namespace
+
+cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
+                             const CUtensorMap &tm_q1, cudaStream_t st, bool pdl) {
+  if (a.M <= 0 || a.C <= 0 || a.R <= 0) return cudaSuccess;
+  if (a.stages < 1 || a.stages > TMAX_STAGES || a.splits < 1 || (a.nq != 1 && a.nq != 2))
+    return cudaErrorInvalidValue;
+  if (a.q_cj && a.nb < 64) return cudaErrorInvalidValue;
+  switch (a.nb) {
+    case 16: return launch_nb<16>(a, tm_p, tm_q0, tm_q1, st, pdl);
+    case 32: return launch_nb<32>(a, tm_p, tm_q0, tm_q1, st, pdl);
+    case 64: return launch_nb<64>(a, tm_p, tm_q0, tm_q1, st, pdl);
+    case 128: return launch_nb<128>(a, tm_p, tm_q0, tm_q1, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_pad_cols(const uint16_t *src, int64_t rows, int cols, uint16_t *dst, int ldd, cudaStream_t st,
+                            int num_sms) {
+  if (ldd % 8 != 0 || (reinterpret_cast<uintptr_t>(dst) & 15u)) return cudaErrorInvalidValue;
+  const int64_t n = rows * (ldd / 8);
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4 * static_cast<int64_t>(num_sms)) blocks = 4 * static_cast<int64_t>(num_sms);
+  if (blocks < 1) blocks = 1;
+  pad_cols_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, cols, dst, ldd);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -236,3 +236,33 @@ def test_decode_forward(T, N, K):
     torch.cuda.synchronize()
     wd = O.dequantize_nf4(codes, scales, c2, N, K)
     assert_close("Y", y, O.linear_fwd(bits(X), wd, bits(A), bits(B), s))
+
+
+# equally spaced 4-bit levels ("QLoRA & 4-bit Fine-Tuning", Innovation 1: the
+# INT4 contrast to NF4); not symmetric (-1 .. 7/8), so the kernels take their
+# general 16-entry lookup instead of the sign-symmetric one
+INT4_LEVELS = [(i - 8) / 8.0 for i in range(16)]
+
+
+@pytest.mark.parametrize("T,N,K,r,s", [(300, 384, 320, 24, 0.5), (4, 1024, 4096, 64, 1.0), (16, 512, 512, 8, 2.0)])
+def test_layer_asymmetric_codebook(T, N, K, r, s):
+    q = Q()
+    W, X, A, B, dY = inputs.layer_inputs(93, 0, 0, T, N, K, r, device="cuda")
+    cb = np.array(INT4_LEVELS, dtype=np.float32)
+    qw = q.quantize_nf4(W, codebook=[float(v) for v in cb])
+    torch.cuda.synchronize()
+    codes, scales, c2 = O.quantize_nf4(bits(W), cb)
+    assert np.array_equal(qw.codes.cpu().numpy(), codes)
+    assert np.array_equal(qw.scales.cpu().numpy(), scales)
+    wd = O.dequantize_nf4(codes, scales, c2, N, K, cb)
+    assert np.array_equal(bits(q.dequantize(qw)), wd)
+    y = q.linear_fwd(X, qw, A, B, s)
+    dx, dA, dB = q.linear_bwd(dY, X, qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    assert_close("Y", y, O.linear_fwd(xb, wd, ab, bb, s))
+    rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    assert_close("dX", dx, rdx)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
