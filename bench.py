@@ -365,7 +365,14 @@ def bench_secondary(dev, peaks):
         del W
         adapters.append((inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(2, 0, i, "A"), dev),
                          inputs.normal_bf16((N, r), 0.01, inputs.seed_of(2, 0, i, "B"), dev)))
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # L2 flush between timed replays: a 256 MB read (a write would leave the
+    # 126 MB L2 full of dirty lines that the timed kernels then write back)
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        torch.sum(flush, dim=0, dtype=torch.float32, out=flush_sink)
+
     for T in (1, 4, 16):
         xs = [inputs.normal_bf16((T, K), 1.0, inputs.seed_of(2, 0, i, "X") + T, dev)
               for i, (_, N, K) in enumerate(shapes)]
@@ -378,7 +385,7 @@ def bench_secondary(dev, peaks):
                 q.linear_fwd(xs[i], qws[i], adapters[i][0], adapters[i][1], 1.0, out=ys[i])
 
         # the seven-projection sweep is replayed as one CUDA graph (no host launch gaps);
-        # the L2 is flushed (256 MB write) before every replay
+        # the L2 is flushed (256 MB read) before every replay
         sweep()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -392,7 +399,7 @@ def bench_secondary(dev, peaks):
         torch.cuda.current_stream(dev).wait_stream(s_cap)
         times = []
         for rep in range(13):
-            flush.zero_()
+            flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             g.replay()
@@ -405,7 +412,7 @@ def bench_secondary(dev, peaks):
         out[f"decode_T{T}"] = {"us_per_sweep": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
                                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                "bytes_per_sweep": int(nbytes), "timing": "CUDA graph of the 7-projection sweep, "
-                               "L2 flushed before each replay, median of 10"}
+                               "L2 flushed (256 MB read) before each replay, median of 10"}
     # quantize / dequantize of one gate-shaped weight (58.7 M weights)
     N, K = 14336, 4096
     W = inputs.normal_bf16((N, K), 0.02, 7, dev)
@@ -415,7 +422,7 @@ def bench_secondary(dev, peaks):
     for name, fn in (("quantize", lambda: q.quantize_nf4(W)), ("dequantize", lambda: q.dequantize(qw))):
         times = []
         for rep in range(6):
-            flush.zero_()
+            flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()

@@ -147,6 +147,7 @@ qlora_status check_weight(const qlora_nf4_weight *qw) {
   if (qw->blocksize != 64 || qw->dq_block != 256 || (qw->cols % 64) != 0) return QLORA_ERR_UNSUPPORTED;
   if (!aligned16(qw->codes)) return QLORA_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(qw->c2) & 3u) != 0) return QLORA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(qw->scales) & 3u) != 0) return QLORA_ERR_MISALIGNED;
   return check_codebook(qw->codebook);
 }
 
@@ -167,6 +168,11 @@ bool codebook_symmetric(const float *cb) {
 // Up to this many tokens the forward runs the decode GEMV, and U = s X A^T
 // runs on the mma.sync kernel (a handful of rows: latency, not bandwidth).
 constexpr int64_t kGemvMaxTokens = 16;
+
+bool decode_path(int64_t T, int64_t N) {
+  (void)N;
+  return T <= kGemvMaxTokens;
+}
 
 struct WsLayout {
   size_t counters = 0;
@@ -200,8 +206,11 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   size_t part = 0;
   if (op == QLORA_OP_FWD) {
     L.su_row = off; off += row_plane;
-    part = T <= kGemvMaxTokens ? skinny_partials_bytes(T, K, r, kSplitSms)
-                               : skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
+    if (decode_path(T, N)) {
+      part = skinny_partials_bytes(T, K, r, kSplitSms);
+    } else {
+      part = skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
+    }
   } else {
     L.suT_hi = off; off += t_plane;
     L.suT_lo = off; off += t_plane;
@@ -320,11 +329,9 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// Token counts up to this use the decode-sized forward (register-fragment
-// dequantization, split-K over a thread block cluster).
 
 qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
-                      const void *B, int r, void *y, cudaStream_t st) {
+                      const void *B, int r, void *y, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
   GemvParams p;
   memset(&p, 0, sizeof(p));
   p.codes = qw->codes;
@@ -341,14 +348,13 @@ qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, cons
   p.r = r;
   p.y = static_cast<uint16_t *>(y);
   p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
-  const GemvPlan pl = gemv_plan(p.N, p.K, num_sms_current());
   const double n = static_cast<double>(p.N) * p.K;
   const double bytes = n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * T * (p.N + p.K) +
                        2.0 * static_cast<double>(p.N) * r;
   TraceScope ts(K_GEMV_FWD, 0.0, bytes, st);
   // programmatic dependent launch only when no trace events sit between the kernels
   const bool pdl = g_trace.recs == nullptr;
-  return launch_gemv(p, pl, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launch_gemv(p, num_sms_current(), st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 // One tensor-core rank-r product.  P: p_col ? [C rows, M cols] : [M rows, C cols]
@@ -562,8 +568,27 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
   const int64_t r64 = round_up(r, 64);
   uint16_t *su = reinterpret_cast<uint16_t *>(w8 + L.su_row);
   // sU = s X A^T [T, ceil64(r)]: the rank-r operand of the GEMV / GEMM
-  if (T <= kGemvMaxTokens) {
-    // a handful of rows: the mma.sync kernel (latency, not bandwidth)
+  if (decode_path(T, N)) {
+    // a handful of rows: a latency-bound product, on a cluster kernel (one
+    // wave, partial sums in distributed shared memory) where its slice fits
+    const bool pdl = g_trace.recs == nullptr;
+    if (lora_u_decode_smem_bytes(K, static_cast<int>(T)) <= kLoraUDecodeMaxSmem) {
+      LoraUDecodeParams pu;
+      pu.x = static_cast<const uint16_t *>(x);
+      pu.A = static_cast<const uint16_t *>(A);
+      pu.u = su;
+      pu.K = K;
+      pu.ldu = r64;
+      pu.T = static_cast<int>(T);
+      pu.r = r;
+      pu.kc = 0;
+      pu.alpha = s;
+      {
+        TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * r * K, st);
+        if (launch_lora_u_decode(pu, st, pdl) != cudaSuccess) return QLORA_ERR_CUDA;
+      }
+      return run_gemv(qw, x, T, su, r64, B, r, y, w8, L, st);
+    }
     SkinnyParams pu = skinny_base(T, K, r, w8, L);
     pu.P = static_cast<const uint16_t *>(x);
     pu.ldp = K;
@@ -577,7 +602,7 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
       TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * T * K, st);
       if (launch_skinny(pu, false, false, OUT_HILO, st) != cudaSuccess) return QLORA_ERR_CUDA;
     }
-    return run_gemv(qw, x, T, su, r64, B, r, y, st);
+    return run_gemv(qw, x, T, su, r64, B, r, y, w8, L, st);
   }
   SkinnyTcArgs au = tc_args(T, K, r, s);
   au.row_hi = su;

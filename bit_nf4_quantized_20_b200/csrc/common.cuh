@@ -479,4 +479,26 @@ __device__ __forceinline__ void lut8_lookup4(const Lut8 &t, uint32_t codes, uint
   out1 = prmt(lo, hi, 0x7362u);
 }
 
+// Eight codes of `w` (code i in bits 4i..4i+3): o0 = (entry(c0), entry(c1)),
+// o1 = (entry(c2), entry(c3)), o2 = (entry(c4), entry(c5)), o3 = (entry(c6), entry(c7)).
+// The sign masks of both halves come from one shifted copy of the word: byte i
+// of m_lo (m_hi) is 0xFF when code i (4 + i) is >= 8, by prmt's sign-replicate
+// mode on the byte whose bit 7 holds that code's bit 3.
+__device__ __forceinline__ void lut8_lookup8(const Lut8 &t, uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2,
+                                             uint32_t &o3) {
+  const uint32_t mag = mag_index8(w);
+  const uint32_t magh = mag >> 16;
+  const uint32_t w4 = w << 4;
+  const uint32_t m_lo = prmt(w4, w, 0xD9C8u);
+  const uint32_t m_hi = prmt(w4, w, 0xFBEAu);
+  const uint32_t lo0 = prmt(t.lo[0], t.lo[1], mag);
+  const uint32_t hi0 = prmt(t.hi[0], t.hi[1], mag) | (~m_lo & 0x80808080u);
+  const uint32_t lo1 = prmt(t.lo[0], t.lo[1], magh);
+  const uint32_t hi1 = prmt(t.hi[0], t.hi[1], magh) | (~m_hi & 0x80808080u);
+  o0 = prmt(lo0, hi0, 0x5140u);
+  o1 = prmt(lo0, hi0, 0x7362u);
+  o2 = prmt(lo1, hi1, 0x5140u);
+  o3 = prmt(lo1, hi1, 0x7362u);
+}
+
 }  // namespace qlora

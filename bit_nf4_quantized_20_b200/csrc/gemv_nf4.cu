@@ -4,22 +4,33 @@
 //
 //   Y[T, N] = X[T, K] W'[N, K]^T + U'[T, r] B[N, r]^T,   U' = BF16(s X A^T)
 //
-// Each lane dequantizes whole 64-weight blocks straight into mma.sync B
-// fragments (no shared-memory staging): lane (g, t) of a warp owns block t of a
-// 256-wide k-unit for weight row g of an 8-row group.  The MMA's k-slots are
-// permuted consistently for both operands (a sum does not depend on the order
-// of its terms): slot 2t+j of k16-step i holds k = 64t + 4i + j and slot
-// 2t+8+j holds k = 64t + 4i + 2 + j, so the four codes a lane feeds one MMA
-// are four consecutive codes of its block, and the X fragments are eight
-// consecutive bytes of one token row.
+// Each lane dequantizes whole 64-weight blocks straight into mma.sync A
+// fragments (no shared-memory tiles): the MMA's M is 16 weight rows and its N
+// is 8 tokens (a second MMA for tokens 8-15), and lane (g, t) of a warp owns
+// block t of a 256-wide k-unit for rows g and g + 8 of the warp's 16-row tile.
+// The MMA's k-slots are permuted consistently for both operands (a sum does
+// not depend on the order of its terms): slot 2t+j of k16-step i holds
+// k = 64t + 4i + j and slot 2t+8+j holds k = 64t + 4i + 2 + j, so the four
+// codes a lane feeds one MMA per row are four consecutive codes of its block,
+// and its X fragments are eight consecutive bytes of one token row.
 //
-// Work split: a CTA (8 warps) owns 8*RG weight rows and a range of k-units,
-// one unit per warp at a time; the CTAs that share a row tile form a thread
-// block cluster and their partial sums are added in rank order through
-// distributed shared memory by rank 0, which adds the rank-r term and writes
-// BF16 Y.  Launched with programmatic dependent launch: the weight stream
-// starts while the kernel computing U' still runs; U' is read only after
-// griddepcontrol.wait.
+// Weight stream: every lane copies its own blocks (32 code bytes, the aligned
+// word holding its scale byte, and its c2) with cp.async into a private ring
+// of GD items in shared memory, so each warp keeps GD - 1 items in flight with
+// no register cost and no cross-lane synchronisation.
+//
+// Work split: a CTA is one 16-row tile; its S warps split the k-units, and
+// their accumulators are added in warp order through shared memory by warp 0,
+// which adds the rank-r term B U'^T as extra MMA k-steps and writes BF16 Y.  S
+// is the largest split count whose grid of N/16 CTAs is resident in one wave.
+// Launched with programmatic dependent launch: the first GD - 1 units of the
+// weight stream are requested while the preceding kernel (the one computing
+// U') still runs; X, U' and Y are touched only after griddepcontrol.wait.
+//
+// lora_u_decode_kernel computes U' itself for these token counts: a cluster of
+// 8 CTAs per 16 columns of U' splits K, each CTA requests its whole slice of A
+// (and, after the dependency wait, of X) at once, and the partial sums meet
+// in rank 0's shared memory.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -28,9 +39,11 @@ namespace qlora {
 
 namespace {
 
-constexpr int GW = 8;              // warps per CTA
-constexpr int kMaxRank = 128;
-constexpr int GT = GW * 32;
+constexpr int GD = 3;              // units in the per-warp ring
+constexpr int kGemvMaxWarps = 8;   // warps per CTA (k-splits of one 16-row tile)
+// one item of one warp: codes [2 rows][2 halves][32 lanes][16 B], then per row
+// [32 lanes] scale words and [32 lanes] c2
+constexpr int kItemBytes = 2048 + 512;
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -41,292 +54,487 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+// cp.async with a source size: bytes past src_bytes are zero-filled (0 reads nothing)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
 }
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// a block as loaded; its scale is formed at use so that loads never wait
-struct Blk {
-  uint4 c0, c1;
-  uint32_t fbyte;
-  float c2;
-};
-
-template <int TT, int RG, bool SYM>
-__global__ void __launch_bounds__(GT, 2) nf4_gemv_kernel(const GemvParams p) {
-  __shared__ float s_red[GW][TT][8 * RG];
-  __shared__ float s_part[TT][8 * RG];
-  __shared__ __align__(16) uint16_t s_B[8 * RG][kMaxRank + 8];
-  __shared__ __align__(16) uint16_t s_U[TT][kMaxRank + 8];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int S = p.splits;
-  const int split = static_cast<int>(cluster_rank());
-  const int rt = blockIdx.x / S;
-  const int64_t row0 = static_cast<int64_t>(rt) * 8 * RG;
-  const int64_t kblocks = p.K / 64;
-
-  float cb[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) cb[i] = p.codebook[i];
-
-  float acc[RG][4];
-#pragma unroll
-  for (int r = 0; r < RG; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-
-  auto load_blk = [&](int u, int rg) -> Blk {
-    Blk b;
-    const int64_t n = row0 + rg * 8 + g;
-    const int64_t kb = static_cast<int64_t>(u) * 4 + t;
-    if (u < p.units && n < p.N && kb < kblocks) {
-      const int64_t blk = n * kblocks + kb;
-      const uint8_t *cp = p.codes + blk * 32;
-      b.c0 = ldg_stream(cp);
-      b.c1 = ldg_stream(cp + 16);
-      b.fbyte = __ldg(p.scales + blk);
-      b.c2 = __ldg(p.c2 + (blk >> 8));
-    } else {
-      b.c0 = make_uint4(0, 0, 0, 0);
-      b.c1 = b.c0;
-      b.fbyte = 0u;
-      b.c2 = 0.f;
-    }
-    return b;
-  };
-
-  // Units of this warp: u_j = (split * upw + j) * GW + warp.  The codes of
-  // unit j + 1 are requested before unit j is computed (two register sets).
-  auto unit_of = [&](int j) { return (split * p.upw + j) * GW + warp; };
-  Blk cur[RG], nxt[RG];
-  {
-    const int u0 = unit_of(0);
-#pragma unroll
-    for (int rg = 0; rg < RG; ++rg) cur[rg] = load_blk(u0 < p.units ? u0 : p.units, rg);
-  }
-  for (int j = 0; j < p.upw; ++j) {
-    const int u = unit_of(j);
-    if (u >= p.units) break;
-    const int un = unit_of(j + 1);
-    const bool more = (j + 1 < p.upw) && (un < p.units);
-#pragma unroll
-    for (int rg = 0; rg < RG; ++rg) nxt[rg] = load_blk(more ? un : p.units, rg);
-    // X fragments for this unit: token rows g (and g + 8), k = 64t .. 64t + 63
-    uint32_t xa[32], xb[TT == 16 ? 32 : 1];
-    {
-      const int64_t k0 = static_cast<int64_t>(u) * 256 + 64 * t;
-      const bool kv = k0 < p.K;
-      if (g < p.T && kv) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(g) * p.K + k0);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 v = __ldg(src + q);
-          xa[4 * q] = v.x; xa[4 * q + 1] = v.y; xa[4 * q + 2] = v.z; xa[4 * q + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) xa[q] = 0u;
-      }
-      if (TT == 16) {
-        if (g + 8 < p.T && kv) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(g + 8) * p.K + k0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 v = __ldg(src + q);
-            xb[4 * q] = v.x; xb[4 * q + 1] = v.y; xb[4 * q + 2] = v.z; xb[4 * q + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < (TT == 16 ? 32 : 1); ++q) xb[q] = 0u;
-        }
-      }
-    }
-#pragma unroll
-    for (int rg = 0; rg < RG; ++rg) {
-      const float scale = __fmul_rn(e4m3_to_float(cur[rg].fbyte), cur[rg].c2);
-      const uint32_t w[8] = {cur[rg].c0.x, cur[rg].c0.y, cur[rg].c0.z, cur[rg].c0.w,
-                             cur[rg].c1.x, cur[rg].c1.y, cur[rg].c1.z, cur[rg].c1.w};
-      if (SYM) {
-        const Lut8 lut = make_lut8(cb, scale);
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          const uint32_t mag = mag_index8(w[h]);
-          uint32_t b0, b1, b2, b3;
-          lut8_lookup4(lut, w[h], mag, b0, b1);
-          lut8_lookup4(lut, w[h] >> 16, mag >> 16, b2, b3);
-          const int i = 2 * h;
-          mma16816(acc[rg], xa[2 * i], (TT == 16) ? xb[2 * i] : 0u, xa[2 * i + 1], (TT == 16) ? xb[2 * i + 1] : 0u,
-                   b0, b1);
-          mma16816(acc[rg], xa[2 * i + 2], (TT == 16) ? xb[2 * i + 2] : 0u, xa[2 * i + 3],
-                   (TT == 16) ? xb[2 * i + 3] : 0u, b2, b3);
-        }
-      } else {
-        const Lut16 lut = make_lut16(cb, scale);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          uint32_t b0, b1;
-          lut16_lookup4(lut, (i & 1) ? (w[i >> 1] >> 16) : w[i >> 1], b0, b1);
-          const uint32_t a1 = (TT == 16) ? xb[2 * i] : 0u;
-          const uint32_t a3 = (TT == 16) ? xb[2 * i + 1] : 0u;
-          mma16816(acc[rg], xa[2 * i], a1, xa[2 * i + 1], a3, b0, b1);
-        }
-      }
-    }
-#pragma unroll
-    for (int rg = 0; rg < RG; ++rg) cur[rg] = nxt[rg];
-  }
-
-  // accumulator fragment: c0/c1 = (token g, rows 2t, 2t+1), c2/c3 = (token g+8, ...)
-#pragma unroll
-  for (int rg = 0; rg < RG; ++rg) {
-    const int r0 = rg * 8 + 2 * t;
-    if (g < TT) {
-      s_red[warp][g][r0] = acc[rg][0];
-      s_red[warp][g][r0 + 1] = acc[rg][1];
-    }
-    if (TT == 16) {
-      s_red[warp][(g + 8) % TT][r0] = acc[rg][2];
-      s_red[warp][(g + 8) % TT][r0 + 1] = acc[rg][3];
-    }
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < TT * 8 * RG; idx += GT) {
-    const int tok = idx / (8 * RG), row = idx % (8 * RG);
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < GW; ++w) v += s_red[w][tok][row];
-    s_part[tok][row] = v;
-  }
-  if (S > 1) cluster_sync();
-  else __syncthreads();
-
-  if (split == 0) {
-    // rank-r term sum_j U'[tok, j] B[n, j] from shared memory: this CTA's rows of
-    // B (independent of the preceding kernel) first, U' after the dependency wait
-    const int nrows = static_cast<int>(min(static_cast<int64_t>(8 * RG), p.N - row0));
-    const int rv = p.r;
-    const uint16_t *bsrc = p.B + row0 * rv;
-    const int nb = nrows * rv;
-    if ((rv % 8) == 0) {
-      for (int c = threadIdx.x; c < nb / 8; c += GT) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(bsrc) + c);
-        const int e = c * 8, row = e / rv, j = e % rv;
-        *reinterpret_cast<uint4 *>(&s_B[row][j]) = v;
-      }
-    } else {
-      for (int e = threadIdx.x; e < nb; e += GT) s_B[e / rv][e % rv] = bsrc[e];
-    }
-    grid_dep_wait();   // U' is written by the preceding kernel
-    const int ucols = static_cast<int>((rv + 7) / 8 * 8);      // the U' plane is zero-padded to ldu >= this
-    for (int c = threadIdx.x; c < p.T * (ucols / 8); c += GT) {
-      const int tok = c / (ucols / 8), j = (c % (ucols / 8)) * 8;
-      *reinterpret_cast<uint4 *>(&s_U[tok][j]) =
-          __ldg(reinterpret_cast<const uint4 *>(p.u + static_cast<int64_t>(tok) * p.ldu + j));
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < TT * 8 * RG; idx += GT) {
-      const int tok = idx / (8 * RG), row = idx % (8 * RG);
-      const int64_t n = row0 + row;
-      if (tok >= p.T || row >= nrows) continue;
-      float v = 0.f;
-      for (int r = 0; r < S; ++r) v += (r == 0) ? s_part[tok][row] : ld_dsmem_f32(&s_part[tok][row], r);
-      float l = 0.f;
-      for (int jj = 0; jj < rv; ++jj) {
-        l = fmaf(__uint_as_float(static_cast<uint32_t>(s_U[tok][jj]) << 16),
-                 __uint_as_float(static_cast<uint32_t>(s_B[row][jj]) << 16), l);
-      }
-      const __nv_bfloat16 o = __float2bfloat16_rn(v + l);
-      p.y[static_cast<int64_t>(tok) * p.N + n] = *reinterpret_cast<const uint16_t *>(&o);
-    }
-  }
-  if (S > 1) cluster_sync();   // peers keep their shared memory alive until rank 0 has read it
-}
-
-template <int TT, int RG, bool SYM>
-cudaError_t launch_tr(const GemvParams &p, int row_tiles, cudaStream_t st, bool pdl) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(row_tiles * p.splits), 1, 1);
-  cfg.blockDim = dim3(GT, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attrs[2];
-  int na = 0;
-  attrs[na].id = cudaLaunchAttributeClusterDimension;
-  attrs[na].val.clusterDim.x = static_cast<unsigned>(p.splits);
-  attrs[na].val.clusterDim.y = 1;
-  attrs[na].val.clusterDim.z = 1;
-  ++na;
-  if (pdl) {
-    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attrs[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-  }
-  cfg.attrs = attrs;
-  cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<TT, RG, SYM>, p);
+__device__ __forceinline__ uint32_t ldg_pair_bf16(const uint16_t *p, int64_t i0, int64_t i1, bool v0, bool v1) {
+  const uint32_t lo = v0 ? static_cast<uint32_t>(__ldg(p + i0)) : 0u;
+  const uint32_t hi = v1 ? static_cast<uint32_t>(__ldg(p + i1)) : 0u;
+  return lo | (hi << 16);
 }
 
 }  // namespace
 
-GemvPlan gemv_plan(int64_t N, int64_t K, int num_sms) {
-  GemvPlan pl;
-  pl.units = static_cast<int>((K + 255) / 256);
-  // 16-row tiles (8-row tiles for small N); split k over a cluster only when the
-  // row tiles alone cannot give every SM two CTAs
-  pl.rg = 2;
-  int64_t tiles = (N + 15) / 16;
-  if (tiles < 2 * static_cast<int64_t>(num_sms)) {
-    pl.rg = 1;
-    tiles = (N + 7) / 8;
+// Fragments of one item for lane (g, t): weight rows r0 = 16 * tile + g and
+// r0 + 8 are the MMA's A operand (M = 16 rows), X is the B operand (N = 8
+// tokens, a second MMA for tokens 8-15).  Accumulator: c0/c1 = (row r0, tokens
+// 2t, 2t + 1), c2/c3 = (row r0 + 8, tokens 2t, 2t + 1).
+
+// rank-r term and store for 16-row tile `tile`: v += B U'^T (k16-steps over r), Y = BF16(v)
+template <int TT>
+__device__ __forceinline__ void gemv_finish(const GemvParams &p, int64_t tile, int g, int t, float (&v)[TT / 8][4]) {
+  const int64_t r0 = tile * 16 + g, r1 = r0 + 8;
+  const bool v0 = r0 < p.N, v1 = r1 < p.N;
+  const int rv = p.r;
+  for (int j0 = 0; j0 < rv; j0 += 16) {
+    const int ja = j0 + 2 * t, jb = j0 + 2 * t + 8;
+    const uint32_t a0 = ldg_pair_bf16(p.B, r0 * rv + ja, r0 * rv + ja + 1, v0 && ja < rv, v0 && ja + 1 < rv);
+    const uint32_t a1 = ldg_pair_bf16(p.B, r1 * rv + ja, r1 * rv + ja + 1, v1 && ja < rv, v1 && ja + 1 < rv);
+    const uint32_t a2 = ldg_pair_bf16(p.B, r0 * rv + jb, r0 * rv + jb + 1, v0 && jb < rv, v0 && jb + 1 < rv);
+    const uint32_t a3 = ldg_pair_bf16(p.B, r1 * rv + jb, r1 * rv + jb + 1, v1 && jb < rv, v1 && jb + 1 < rv);
+#pragma unroll
+    for (int h = 0; h < TT / 8; ++h) {
+      const int tok = 8 * h + g;
+      uint32_t b0 = 0u, b1 = 0u;
+      if (tok < p.T) {
+        const uint16_t *ur = p.u + static_cast<int64_t>(tok) * p.ldu;   // zero-padded to ldu >= ceil16(r)
+        b0 = *reinterpret_cast<const uint32_t *>(ur + ja);
+        b1 = *reinterpret_cast<const uint32_t *>(ur + jb);
+      }
+      mma16816(v[h], a0, a1, a2, a3, b0, b1);
+    }
   }
-  int splits = 1;
-  while (splits < 8 && tiles * splits < 2 * static_cast<int64_t>(num_sms) &&
-         pl.units >= GW * (splits + 1)) {
-    ++splits;
+#pragma unroll
+  for (int h = 0; h < TT / 8; ++h) {
+    const int ta = 8 * h + 2 * t, tb = ta + 1;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v[h][0], v[h][1]);   // row r0, tokens ta, tb
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(v[h][2], v[h][3]);   // row r1
+    if (v0 && ta < p.T) p.y[static_cast<int64_t>(ta) * p.N + r0] = __bfloat16_as_ushort(lo.x);
+    if (v0 && tb < p.T) p.y[static_cast<int64_t>(tb) * p.N + r0] = __bfloat16_as_ushort(lo.y);
+    if (v1 && ta < p.T) p.y[static_cast<int64_t>(ta) * p.N + r1] = __bfloat16_as_ushort(hi.x);
+    if (v1 && tb < p.T) p.y[static_cast<int64_t>(tb) * p.N + r1] = __bfloat16_as_ushort(hi.y);
   }
-  // every split gets whole rounds of GW units; at most 8 CTAs per cluster
-  pl.upw = (pl.units + GW * splits - 1) / (GW * splits);
-  pl.splits = (pl.units + GW * pl.upw - 1) / (GW * pl.upw);
-  pl.row_tiles = static_cast<int>(tiles);
-  return pl;
 }
 
-cudaError_t launch_gemv(const GemvParams &p_in, const GemvPlan &pl, cudaStream_t st, bool pdl) {
-  GemvParams p = p_in;
+// X fragments of k16-steps 4c .. 4c + 3 for the lane's token rows (8 registers per token half)
+template <int NH>
+__device__ __forceinline__ void load_x_chunk(const uint16_t *const (&xrow)[NH], bool kv, int c, uint32_t (&xf)[NH][8]) {
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    if (kv) {
+      const uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(xrow[h]) + 2 * c);
+      const uint4 v1 = __ldg(reinterpret_cast<const uint4 *>(xrow[h]) + 2 * c + 1);
+      xf[h][0] = v0.x; xf[h][1] = v0.y; xf[h][2] = v0.z; xf[h][3] = v0.w;
+      xf[h][4] = v1.x; xf[h][5] = v1.y; xf[h][6] = v1.z; xf[h][7] = v1.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xf[h][q] = 0u;
+    }
+  }
+}
+
+template <int TT, bool SYM>
+__global__ void __launch_bounds__(kGemvMaxWarps * 32) nf4_gemv_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) uint8_t gsm[];
+  constexpr int NH = TT / 8;   // token halves
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int S = p.splits;
+  const int64_t tile = blockIdx.x;
+  const int64_t KB = p.K / 64;
+  const int u_beg = warp * p.upw;
+  const int nu = max(0, min(p.units, u_beg + p.upw) - u_beg);
+  const uint32_t ring = smem_u32(gsm) + warp * GD * kItemBytes;
+  const uintptr_t scales_addr = reinterpret_cast<uintptr_t>(p.scales);
+  const int64_t r0 = tile * 16 + g;
+  bool rok[2];
+  int64_t rowblk[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    rok[h] = r0 + 8 * h < p.N;
+    rowblk[h] = (r0 + 8 * h) * KB;
+  }
+
+  // unit u_beg + i into ring slot i % GD (one commit group per unit, empty past the end)
+  auto issue = [&](int i) {
+    if (i < nu) {
+      const int64_t kb = static_cast<int64_t>(u_beg + i) * 4 + t;
+      const uint32_t base = ring + (i % GD) * kItemBytes;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const bool ok = kb < KB && rok[h];
+        const int64_t blk = ok ? rowblk[h] + kb : 0;
+        const uint32_t d = base + h * 1024 + lane * 16;
+        const uint8_t *src = p.codes + blk * 32;
+        cp_async16(d, src, ok ? 16u : 0u);
+        cp_async16(d + 512, src + 16, ok ? 16u : 0u);
+        const uint32_t da = base + 2048 + h * 256 + lane * 4;
+        cp_async4(da, reinterpret_cast<const void *>((scales_addr + blk) & ~static_cast<uintptr_t>(3)), ok ? 4u : 0u);
+        cp_async4(da + 128, p.c2 + (blk >> 8), ok ? 4u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll 1
+  for (int i = 0; i < GD - 1; ++i) issue(i);   // the weights do not depend on the preceding kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dep_wait();                               // X, U' and Y may
+
+  // token rows this lane feeds to the MMA (rows past T repeat row T - 1; their
+  // accumulator columns are never stored)
+  const uint16_t *xrow0[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) xrow0[h] = p.x + static_cast<int64_t>(min(8 * h + g, p.T - 1)) * p.K + 64 * t;
+  float acc[NH][4], acc2[NH][4];   // even / odd k16-steps (two independent MMA chains)
+#pragma unroll
+  for (int h = 0; h < NH; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[h][e] = acc2[h][e] = 0.f;
+#pragma unroll 1
+  for (int i = 0; i < nu; ++i) {
+    issue(i + GD - 1);
+    const int u = u_beg + i;
+    const bool kv = static_cast<int64_t>(u) * 256 + 64 * t < p.K;   // false past K (codes zero-filled too)
+    const uint16_t *xrow[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) xrow[h] = xrow0[h] + static_cast<int64_t>(u) * 256;
+    uint32_t xf[NH][8], xn[NH][8];
+    load_x_chunk<NH>(xrow, kv, 0, xf);
+    cp_async_wait<GD - 1>();      // this lane's copies of unit i have landed
+    const uint32_t base = ring + (i % GD) * kItemBytes;
+    float scale[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t sword = lds32(base + 2048 + h * 256 + lane * 4);
+      const float c2v = __uint_as_float(lds32(base + 2048 + h * 256 + 128 + lane * 4));
+      const int64_t blk = rowblk[h] + static_cast<int64_t>(u) * 4 + t;
+      const uint32_t fbyte = (sword >> (8u * static_cast<uint32_t>((scales_addr + blk) & 3u))) & 0xffu;
+      scale[h] = __fmul_rn(e4m3_to_float(fbyte), c2v);
+    }
+    // four chunks of 16 codes per row (k16-steps 4c .. 4c + 3); X of the next chunk is loaded ahead
+    if constexpr (SYM) {
+      const Lut8 l0 = make_lut8(p.codebook, scale[0]);
+      const Lut8 l1 = make_lut8(p.codebook, scale[1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c < 3) load_x_chunk<NH>(xrow, kv, c + 1, xn);
+        const uint2 w0 = lds64(base + (c >> 1) * 512 + lane * 16 + (c & 1) * 8);
+        const uint2 w1 = lds64(base + 1024 + (c >> 1) * 512 + lane * 16 + (c & 1) * 8);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          uint32_t a[4], b[4];
+          lut8_lookup8(l0, e ? w0.y : w0.x, a[0], a[1], a[2], a[3]);
+          lut8_lookup8(l1, e ? w1.y : w1.x, b[0], b[1], b[2], b[3]);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            mma16816(acc[h], a[0], b[0], a[1], b[1], xf[h][4 * e], xf[h][4 * e + 1]);
+            mma16816(acc2[h], a[2], b[2], a[3], b[3], xf[h][4 * e + 2], xf[h][4 * e + 3]);
+          }
+        }
+        if (c < 3) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xf[h][q] = xn[h][q];
+        }
+      }
+    } else {
+      const Lut16 l0 = make_lut16(p.codebook, scale[0]);
+      const Lut16 l1 = make_lut16(p.codebook, scale[1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c < 3) load_x_chunk<NH>(xrow, kv, c + 1, xn);
+        const uint2 w0 = lds64(base + (c >> 1) * 512 + lane * 16 + (c & 1) * 8);
+        const uint2 w1 = lds64(base + 1024 + (c >> 1) * 512 + lane * 16 + (c & 1) * 8);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t s0 = (k & 2) ? w0.y : w0.x, s1 = (k & 2) ? w1.y : w1.x;
+          uint32_t a0, a2, a1, a3;
+          lut16_lookup4(l0, (k & 1) ? (s0 >> 16) : s0, a0, a2);
+          lut16_lookup4(l1, (k & 1) ? (s1 >> 16) : s1, a1, a3);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            if (k & 1) mma16816(acc2[h], a0, a1, a2, a3, xf[h][2 * k], xf[h][2 * k + 1]);
+            else mma16816(acc[h], a0, a1, a2, a3, xf[h][2 * k], xf[h][2 * k + 1]);
+          }
+        }
+        if (c < 3) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xf[h][q] = xn[h][q];
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int h = 0; h < NH; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[h][e] += acc2[h][e];
+
+  // the warps' partial sums over their k-units, added in warp order by warp 0;
+  // each warp's slot is the start of its own ring, whose copies have all landed
+  if (S > 1) {
+    if (warp > 0) {
+      float4 *red = reinterpret_cast<float4 *>(gsm + warp * GD * kItemBytes);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) red[h * 32 + lane] = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int w2 = 1; w2 < S; ++w2) {
+        const float4 *red = reinterpret_cast<const float4 *>(gsm + w2 * GD * kItemBytes);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const float4 o = red[h * 32 + lane];
+          acc[h][0] += o.x; acc[h][1] += o.y; acc[h][2] += o.z; acc[h][3] += o.w;
+        }
+      }
+    }
+  }
+  if (warp == 0) gemv_finish<TT>(p, tile, g, t, acc);
+}
+
+// ---------------------------------------------------------------------------
+// U' = BF16(s X A^T) for T <= 16 tokens.  Grid: 8 x (ldu / 16) CTAs in clusters
+// of 8; cluster c owns columns 16c .. 16c + 15 of U' (A rows past r arrive as
+// zeros, so the padding columns come out zero), rank k owns the k-th slice of
+// the contraction.  Four warps split the slice; each runs mma.sync with
+// A = X [tokens][k] and B = A^T.
+// ---------------------------------------------------------------------------
+constexpr int kUCluster = 8;
+constexpr int kUThreads = 128;
+
+template <int TT>
+__global__ void __launch_bounds__(kUThreads, 1) lora_u_decode_kernel(const LoraUDecodeParams p) {
+  extern __shared__ __align__(16) uint8_t usm[];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t rank = cluster_ctarank();
+  const int cg = blockIdx.x / kUCluster;
+  const int pitch = p.kc + 8;                      // BF16 elements per shared row (conflict-free fragments)
+  uint16_t *sa = reinterpret_cast<uint16_t *>(usm);            // [16 j][pitch]
+  uint16_t *sx = sa + 16 * pitch;                              // [TT tok][pitch]
+  float4 *red = reinterpret_cast<float4 *>(sx + TT * pitch);   // [4 warps][2][32]
+  const int64_t kbeg = static_cast<int64_t>(rank) * p.kc;
+  const int64_t klen = max(static_cast<int64_t>(0), min(static_cast<int64_t>(p.kc), p.K - kbeg));
+  const int chunks = static_cast<int>(p.kc / 8);               // 16-byte pieces per row
+
+  // A rows 16cg .. 16cg + 15 of this slice (static: requested before the dependency wait)
+  for (int c = threadIdx.x; c < 16 * chunks; c += kUThreads) {
+    const int j = c / chunks, q = c % chunks;
+    const int64_t jr = static_cast<int64_t>(cg) * 16 + j;
+    const bool ok = jr < p.r && 8 * q < klen;
+    const uint16_t *src = ok ? p.A + jr * p.K + kbeg + 8 * q : p.A;
+    const uint32_t d = smem_u32(sa + j * pitch + 8 * q);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(ok ? 16 : 0) : "memory");
+  }
+  grid_dep_wait();   // X may be written by the preceding kernel, U' read by it
+  for (int c = threadIdx.x; c < TT * chunks; c += kUThreads) {
+    const int tok = c / chunks, q = c % chunks;
+    const bool ok = tok < p.T && 8 * q < klen;
+    const uint16_t *src = ok ? p.x + static_cast<int64_t>(tok) * p.K + kbeg + 8 * q : p.x;
+    const uint32_t d = smem_u32(sx + tok * pitch + 8 * q);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(ok ? 16 : 0) : "memory");
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  const int steps = p.kc / 16;
+  for (int st = warp; st < steps; st += 4) {
+    const int k0 = st * 16;
+    auto ld32 = [&](const uint16_t *row, int k) { return *reinterpret_cast<const uint32_t *>(row + k); };
+    const uint32_t a0 = ld32(sx + g * pitch, k0 + 2 * t);
+    const uint32_t a2 = ld32(sx + g * pitch, k0 + 2 * t + 8);
+    const uint32_t a1 = TT == 16 ? ld32(sx + (g + 8) * pitch, k0 + 2 * t) : 0u;
+    const uint32_t a3 = TT == 16 ? ld32(sx + (g + 8) * pitch, k0 + 2 * t + 8) : 0u;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint16_t *arow = sa + (nt * 8 + g) * pitch;
+      mma16816(acc[nt], a0, a1, a2, a3, ld32(arow, k0 + 2 * t), ld32(arow, k0 + 2 * t + 8));
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) red[(warp * 2 + nt) * 32 + lane] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float4 v = red[nt * 32 + lane];
+      for (int w = 1; w < 4; ++w) {
+        const float4 o = red[(w * 2 + nt) * 32 + lane];
+        v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+      }
+      red[nt * 32 + lane] = v;   // this CTA's partial sum, in warp 0's slots
+    }
+  }
+  cluster_arrive_wait();
+  if (rank == 0 && warp == 0) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float4 v = red[nt * 32 + lane];
+      for (uint32_t k = 1; k < kUCluster; ++k) {
+        const uint32_t ra = mapa_shared(smem_u32(&red[nt * 32 + lane]), k);
+        float4 o;
+        asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(o.x), "=f"(o.y), "=f"(o.z), "=f"(o.w)
+                     : "r"(ra)
+                     : "memory");
+        v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+      }
+      // fragment: (token g, columns 2t, 2t+1) and (token g + 8, ...)
+      const int64_t col = static_cast<int64_t>(cg) * 16 + nt * 8 + 2 * t;
+      if (g < p.T)
+        *reinterpret_cast<__nv_bfloat162 *>(p.u + static_cast<int64_t>(g) * p.ldu + col) =
+            __floats2bfloat162_rn(p.alpha * v.x, p.alpha * v.y);
+      if (TT == 16 && g + 8 < p.T)
+        *reinterpret_cast<__nv_bfloat162 *>(p.u + static_cast<int64_t>(g + 8) * p.ldu + col) =
+            __floats2bfloat162_rn(p.alpha * v.z, p.alpha * v.w);
+    }
+  }
+  cluster_arrive_wait();   // the peers keep their shared memory until rank 0 has read it
+}
+
+int gemv_smem_bytes(int splits) { return splits * GD * kItemBytes; }
+
+namespace {
+
+// CTAs of `splits` warps that one SM holds at once (cached per kernel and split count)
+template <int TT, bool SYM>
+int gemv_occupancy(int splits) {
+  static int occ[kGemvMaxWarps + 1] = {0};
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(nf4_gemv_kernel<TT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv_smem_bytes(kGemvMaxWarps)) != cudaSuccess)
+      return -1;
+    attr_set = true;
+  }
+  if (occ[splits] == 0) {
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, nf4_gemv_kernel<TT, SYM>, 32 * splits,
+                                                      gemv_smem_bytes(splits)) != cudaSuccess)
+      return -1;
+    occ[splits] = o > 0 ? o : -1;
+  }
+  return occ[splits];
+}
+
+// The most k-splits per 16-row tile whose grid still fits in one wave (all
+// tiles resident at once); one split if even that does not fit.
+template <int TT, bool SYM>
+cudaError_t gemv_plan(int64_t N, int64_t K, int num_sms, GemvPlan &pl) {
+  pl.units = static_cast<int>((K + 255) / 256);
+  pl.tiles = static_cast<int>((N + 15) / 16);
+  int best = 1;
+  for (int s = 1; s <= kGemvMaxWarps && s <= pl.units; ++s) {
+    const int upw = (pl.units + s - 1) / s;
+    const int splits = (pl.units + upw - 1) / upw;
+    if (splits != s) continue;
+    const int occ = gemv_occupancy<TT, SYM>(s);
+    if (occ < 0) return cudaErrorInvalidConfiguration;
+    if (static_cast<int64_t>(occ) * num_sms >= pl.tiles) best = s;
+  }
+  pl.upw = (pl.units + best - 1) / best;
+  pl.splits = (pl.units + pl.upw - 1) / pl.upw;
+  return cudaSuccess;
+}
+
+template <int TT, bool SYM>
+cudaError_t launch_t(GemvParams p, int num_sms, cudaStream_t st, bool pdl) {
+  GemvPlan pl;
+  cudaError_t e = gemv_plan<TT, SYM>(p.N, p.K, num_sms, pl);
+  if (e != cudaSuccess) return e;
   p.units = pl.units;
   p.upw = pl.upw;
   p.splits = pl.splits;
-  const bool t16 = p.T > 8;
-  if (p.sym) {
-    if (pl.rg == 2) return t16 ? launch_tr<16, 2, true>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2, true>(p, pl.row_tiles, st, pdl);
-    return t16 ? launch_tr<16, 1, true>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1, true>(p, pl.row_tiles, st, pdl);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.tiles), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(32 * pl.splits), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(gemv_smem_bytes(pl.splits));
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<TT, SYM>, p);
+}
+
+}  // namespace
+
+int lora_u_decode_smem_bytes(int64_t K, int T) {
+  const int64_t kc = ((K + kUCluster - 1) / kUCluster + 63) / 64 * 64;
+  const int tt = T > 8 ? 16 : 8;
+  return static_cast<int>((16 + tt) * (kc + 8) * 2 + 4 * 2 * 32 * 16);
+}
+
+namespace {
+template <int TT>
+cudaError_t launch_u(const LoraUDecodeParams &p, int smem, cudaStream_t st, bool pdl) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(lora_u_decode_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kLoraUDecodeMaxSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
   }
-  if (pl.rg == 2) return t16 ? launch_tr<16, 2, false>(p, pl.row_tiles, st, pdl) : launch_tr<8, 2, false>(p, pl.row_tiles, st, pdl);
-  return t16 ? launch_tr<16, 1, false>(p, pl.row_tiles, st, pdl) : launch_tr<8, 1, false>(p, pl.row_tiles, st, pdl);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(kUCluster * (p.ldu / 16)), 1, 1);
+  cfg.blockDim = dim3(kUThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = kUCluster;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, lora_u_decode_kernel<TT>, p);
+}
+}  // namespace
+
+cudaError_t launch_lora_u_decode(const LoraUDecodeParams &p_in, cudaStream_t st, bool pdl) {
+  LoraUDecodeParams p = p_in;
+  if (p.T < 1 || p.T > 16 || p.r < 1 || p.ldu % 16 != 0 || p.ldu < p.r || p.K % 64 != 0)
+    return cudaErrorInvalidValue;
+  p.kc = static_cast<int>(((p.K + kUCluster - 1) / kUCluster + 63) / 64 * 64);
+  const int smem = lora_u_decode_smem_bytes(p.K, p.T);
+  if (smem > kLoraUDecodeMaxSmem) return cudaErrorInvalidValue;
+  return p.T > 8 ? launch_u<16>(p, smem, st, pdl) : launch_u<8>(p, smem, st, pdl);
+}
+
+cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl) {
+  if (p.T < 1 || p.T > 16 || p.N % 8 != 0 || p.K % 64 != 0 || num_sms < 1) return cudaErrorInvalidValue;
+  const bool t16 = p.T > 8;
+  if (p.sym) return t16 ? launch_t<16, true>(p, num_sms, st, pdl) : launch_t<8, true>(p, num_sms, st, pdl);
+  return t16 ? launch_t<16, false>(p, num_sms, st, pdl) : launch_t<8, false>(p, num_sms, st, pdl);
 }
 
 }  // namespace qlora

@@ -70,14 +70,28 @@ struct GemvParams {
   int units, upw, splits;  // filled from the plan
 };
 struct GemvPlan {
-  int units;       // 256-wide k units
+  int units;       // 256-wide k-units per row
   int upw;         // units per warp
-  int splits;      // CTAs per row tile (thread block cluster size, <= 8)
-  int rg;          // 8-row groups per CTA
-  int row_tiles;
+  int splits;      // warps per CTA (k-splits of one 16-row tile, <= 8)
+  int tiles;       // 16-row tiles = CTAs
 };
-GemvPlan gemv_plan(int64_t N, int64_t K, int num_sms);
-cudaError_t launch_gemv(const GemvParams &p, const GemvPlan &pl, cudaStream_t st, bool pdl);
+int gemv_smem_bytes(int splits);
+cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl);
+
+// U' = BF16(alpha X A^T) [T, ldu] for T <= 16 (gemv_nf4.cu); columns r .. ldu - 1 are written as zero.
+struct LoraUDecodeParams {
+  const uint16_t *x;     // [T, K]
+  const uint16_t *A;     // [r, K]
+  uint16_t *u;           // [T, ldu], ldu a multiple of 16
+  int64_t K, ldu;
+  int T, r;
+  int kc;                // contraction per CTA (set by the launcher)
+  float alpha;
+};
+constexpr int kLoraUDecodeMaxSmem = 200 * 1024;
+// Dynamic shared memory the kernel needs for (K, T); it runs when <= kLoraUDecodeMaxSmem.
+int lora_u_decode_smem_bytes(int64_t K, int T);
+cudaError_t launch_lora_u_decode(const LoraUDecodeParams &p, cudaStream_t st, bool pdl);
 
 // ---------------------------------------------------------------------------
 // rank-r LoRA GEMMs on the legacy tensor path (skinny.cu)

@@ -74,6 +74,7 @@ typedef enum {
  *   c2      float[ceil(rows*cols/(64*256))]: one FP32 second-level scale per
  *           256 consecutive blocks in flat order (the last group may be short).
  *   codebook  the 16 ascending FP32 levels the codes index (by value).
+ * Alignment: codes 16 bytes, scales and c2 4 bytes (else QLORA_ERR_MISALIGNED).
  * Dequantized weight: s_b = RN32(fp8(scales[b]) * c2[b/256]);
  *                     W'  = BF16_RNE(RN32(codebook[code] * s_b)).
  */
