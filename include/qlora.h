@@ -21,8 +21,8 @@
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
- *     never allocates, frees or keeps device memory between calls, apart from
- *     small __constant__ tables that each call overwrites.
+ *     never allocates or frees device memory; its only device state is the
+ *     fixed scratch array of qlora_linear_fwd_noalloc (a static symbol).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).  Work
  *     is enqueued on it and the call returns after validating the arguments;
  *     results are ready when the stream reaches that point.
