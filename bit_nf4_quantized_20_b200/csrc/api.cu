@@ -287,6 +287,8 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   p.k_lora = static_cast<int>(r64 / 64);
   p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
   p.status = status;
+  p.out = static_cast<uint16_t *>(out);
+  p.ldo = Mside;
   const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
   const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;

@@ -17,7 +17,9 @@
 // SM streams from L2 per FLOP.
 //
 // Warp roles (576 threads per CTA, one CTA per SM, persistent over tiles):
-//   warps 0-3   epilogue: tensor memory -> BF16 -> shared memory -> TMA store
+//   warps 0-3   epilogue: tensor memory -> BF16 -> global memory, a pair of features
+//               per 32-bit store (each store instruction writes 64 contiguous bytes
+//               for each of two tokens)
 //   warps 4-15  dequantization in three groups of four warps; group g fills the
 //               pipeline stages it with it % 3 == g
 //   warp 16     TMA loads of this CTA's token half (X / dY, then s*U / dU)
@@ -47,15 +49,13 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = PM * BK * 2;           // 16 KiB
 constexpr int B_BYTES = HN * BK * 2;           // 16 KiB
 constexpr int EPI_ROWS = 32;
-constexpr int EPI_BYTES = EPI_ROWS * PM * 2;   // 8 KiB
 constexpr int NUM_THREADS = 576;
 constexpr int DQ_GROUPS = 3;          // STAGES is a multiple of it
 constexpr int TMEM_COLS = 512;
 
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_EPI = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_EPI + 2 * EPI_BYTES;
+constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 5;       // full[S], empty[S], acc_full[2], acc_empty[2], drain
 constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -70,7 +70,6 @@ struct Smem {
   uint32_t base;
   __device__ uint32_t a(int s) const { return base + OFF_A + s * A_BYTES; }
   __device__ uint32_t b(int s) const { return base + OFF_B + s * B_BYTES; }
-  __device__ uint32_t epi(int i) const { return base + OFF_EPI + i * EPI_BYTES; }
   __device__ uint32_t full(int s) const { return base + OFF_BAR + 8 * s; }
   __device__ uint32_t empty(int s) const { return base + OFF_BAR + 8 * (STAGES + s); }
   __device__ uint32_t acc_full(int i) const { return base + OFF_BAR + 8 * (2 * STAGES + i); }
@@ -116,7 +115,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tmap_act);
     tma_prefetch_desc(&tmap_lact);
-    tma_prefetch_desc(&tmap_out);
   }
   if (warp == 17) {
     tmem_alloc_pair(sm.tmem_slot(), TMEM_COLS);
@@ -278,8 +276,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue (warps 0-3) ----------------
     const int q = warp;
-    const bool issuer = (threadIdx.x == 0);
-    int tc = 0, chunk_count = 0;
+    const int64_t m_side = bwd ? p.K : p.N;
+    int tc = 0;
     bool ok = true;
     for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
       const int m_pair = tile % m_pairs;
@@ -292,6 +290,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * PN);
       const int m_local = q * 32 + static_cast<int>(lane);
       const int feat0 = m_pair * 2 * PM + static_cast<int>(rank) * PM;
+      // lanes 2i and 2i + 1 hold features f and f + 1 (f even); after one exchange
+      // the even lane stores both features of token j, the odd lane those of j + 1
+      const int64_t col = static_cast<int64_t>(feat0) + (m_local & ~1);
+      const bool odd = (lane & 1) != 0;
       for (int ch = 0; ch < PN / EPI_ROWS; ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + ch * EPI_ROWS, r);
@@ -301,27 +303,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(lead(sm.acc_empty(acc)));
         }
-        if (static_cast<int64_t>(n_tile) * PN + ch * EPI_ROWS >= p.T) continue;   // uniform
-        const int buf = chunk_count & 1;
-        if (issuer) tma_store_wait_read<1>();
-        named_bar_sync(1, 128);
-        const uint32_t stg = sm.epi(buf);
+        const int64_t tok0 = static_cast<int64_t>(n_tile) * PN + ch * EPI_ROWS;
+        if (tok0 >= p.T) continue;   // uniform
 #pragma unroll
-        for (int j = 0; j < EPI_ROWS; ++j) {
-          const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
-          st_shared_u16(stg + (j * PM + m_local) * 2, *reinterpret_cast<const uint16_t *>(&v));
+        for (int j = 0; j < EPI_ROWS; j += 2) {
+          const float a = __uint_as_float(r[j]), b = __uint_as_float(r[j + 1]);
+          const float recv = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
+          const int64_t tok = tok0 + j + (odd ? 1 : 0);
+          // the row stride is a multiple of 8: an even column below it has its pair too
+          if (tok < p.T && col < m_side) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(odd ? recv : a, odd ? b : recv);
+            *reinterpret_cast<__nv_bfloat162 *>(p.out + tok * p.ldo + col) = v;
+          }
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (issuer) {
-          tma_store_2d(&tmap_out, stg, feat0, n_tile * PN + ch * EPI_ROWS);
-          tma_store_commit();
-        }
-        ++chunk_count;
       }
     }
     if (!ok) s_abort = 1;
-    if (issuer) tma_store_wait_all<0>();
   }
 
   tc_fence_before();

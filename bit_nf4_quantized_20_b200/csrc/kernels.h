@@ -39,6 +39,8 @@ struct GemmParams {
   int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part
   int sym;                 // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   uint32_t *status;
+  uint16_t *out;           // CTA-pair variant: Y [T, N] or dX [T, K], stored from registers
+  int64_t ldo;             // its row stride (N or K)
 };
 int gemm_smem_bytes();
 int gemm_2sm_smem_bytes();
