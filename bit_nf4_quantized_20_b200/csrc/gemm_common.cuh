@@ -62,9 +62,11 @@ struct BlockIn {
 __device__ __forceinline__ BlockIn load_block(const GemmParams &p, int64_t blk, bool valid) {
   BlockIn in;
   if (valid) {
-    const uint8_t *cp = p.codes + blk * 32;
-    in.c0 = ldg_nc_v4(cp);
-    in.c1 = ldg_nc_v4(cp + 16);
+    // cached loads: the second half of the 32-byte sector then hits L1, and the
+    // codes, which every token tile re-reads, keep the normal L2 policy
+    const uint4 *cp = reinterpret_cast<const uint4 *>(p.codes + blk * 32);
+    in.c0 = __ldg(cp);
+    in.c1 = __ldg(cp + 1);
     in.fbyte = __ldg(p.scales + blk);
     in.c2 = __ldg(p.c2 + (blk >> 8));
   } else {
