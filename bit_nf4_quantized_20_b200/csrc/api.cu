@@ -36,12 +36,14 @@ enum KernelId : int32_t {
   K_GEMM_FWD = 6,
   K_GEMM_BWD = 7,
   K_GEMV_FWD = 8,
-  K_COUNT = 9,
+  K_LORA_U_DU = 9,      // U and dU in one grid (backward)
+  K_LORA_DB_DA = 10,    // dB and dA in one grid (backward)
+  K_COUNT = 11,
 };
 
-const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",   "lora_du",
+const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",       "lora_du",
                                      "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx",
-                                     "nf4_gemv_fwd"};
+                                     "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA"};
 
 struct TraceScope {
   cudaStream_t st;
@@ -187,9 +189,23 @@ struct WsLayout {
 // The split geometry of each tensor-core rank-r product (sized for kSplitSms,
 // whatever the current device, so that workspace sizes are device-independent).
 SkinnyTcGeom geom_u(int64_t T, int64_t K, int r) { return skinny_tc_geom(T, K, r, 1, false, kSplitSms); }
-SkinnyTcGeom geom_du(int64_t T, int64_t N, int r) { return skinny_tc_geom(T, N, r, 1, true, kSplitSms); }
-SkinnyTcGeom geom_db(int64_t T, int64_t N, int r) { return skinny_tc_geom(N, T, r, 2, false, kSplitSms); }
-SkinnyTcGeom geom_da(int64_t T, int64_t K, int r) { return skinny_tc_geom(K, T, r, 2, false, kSplitSms); }
+// backward: U with dU, then dB with dA, each pair in one grid
+struct PairGeom {
+  SkinnyTcGeom g0, g1;
+  size_t part0, part1;   // partial-buffer bytes (the second starts 256-aligned after the first)
+};
+PairGeom pair_geom(int64_t M0, int64_t C0, bool q0, int64_t M1, int64_t C1, bool q1, int r, int nq) {
+  PairGeom pg;
+  skinny_tc_pair_geom(M0, C0, q0, M1, C1, q1, r, nq, kSplitSms, pg.g0, pg.g1);
+  pg.part0 = skinny_tc_partials_bytes(pg.g0, M0, r);
+  pg.part1 = skinny_tc_partials_bytes(pg.g1, M1, r);
+  return pg;
+}
+PairGeom geom_u_du(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(T, K, false, T, N, true, r, 1); }
+PairGeom geom_db_da(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(N, T, false, K, T, false, r, 2); }
+size_t pair_partials(const PairGeom &pg) {
+  return static_cast<size_t>(round_up(static_cast<int64_t>(pg.part0), 256)) + pg.part1;
+}
 
 WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   WsLayout L;
@@ -218,10 +234,7 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     L.duT_hi = off; off += t_plane;
     L.duT_lo = off; off += t_plane;
     L.bpad = off; off += static_cast<size_t>(round_up(N * r64 * 2, 256));
-    const size_t p[4] = {skinny_tc_partials_bytes(geom_u(T, K, r), T, r),
-                         skinny_tc_partials_bytes(geom_du(T, N, r), T, r),
-                         skinny_tc_partials_bytes(geom_db(T, N, r), N, r),
-                         skinny_tc_partials_bytes(geom_da(T, K, r), K, r)};
+    const size_t p[2] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r))};
     for (size_t v : p) part = v > part ? v : part;
   }
   L.partials = off;
@@ -373,7 +386,10 @@ struct TcProduct {
   SkinnyTcGeom g;
 };
 
-qlora_status run_skinny_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
+// Fills the launch fields of `a` for product t (partials and counters at the
+// given workspace offsets) and builds its three tensor maps {P, Q0, Q1}.
+bool prepare_tc(const TcProduct &t, SkinnyTcArgs &a, uint8_t *ws, size_t part_off, size_t counter_off,
+                CUtensorMap *maps) {
   a.nq = t.Q1 ? 2 : 1;
   a.p_col = t.p_col ? 1 : 0;
   a.q_cj = t.q_cj ? 1 : 0;
@@ -381,28 +397,47 @@ qlora_status run_skinny_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, cons
   a.stages = t.g.stages;
   a.splits = t.g.splits;
   a.c_per_split = t.g.c_per_split;
-  a.partials = reinterpret_cast<float *>(ws + L.partials);
-  a.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+  a.partials = reinterpret_cast<float *>(ws + part_off);
+  a.counters = reinterpret_cast<uint32_t *>(ws + counter_off);
   a.status = reinterpret_cast<uint32_t *>(ws);
-  CUtensorMap tp, tq0, tq1;
-  const bool okp = t.p_col ? make_map_bf16(&tp, t.P, a.C, a.M, t.ldp, 64, 64, true)
-                           : make_map_bf16(&tp, t.P, a.M, a.C, t.ldp, 128, 64, true);
-  if (!okp) return QLORA_ERR_CUDA;
+  const bool okp = t.p_col ? make_map_bf16(&maps[0], t.P, a.C, a.M, t.ldp, 64, 64, true)
+                           : make_map_bf16(&maps[0], t.P, a.M, a.C, t.ldp, 128, 64, true);
+  if (!okp) return false;
   auto qmap = [&](CUtensorMap *m, const void *q) {
     return t.q_cj ? make_map_bf16(m, q, a.C, a.R, t.ldq, 64, 64, true)
                   : make_map_bf16(m, q, a.R, a.C, t.ldq, a.nb, 64, true);
   };
-  if (!qmap(&tq0, t.Q0)) return QLORA_ERR_CUDA;
-  if (t.Q1) {
-    if (!qmap(&tq1, t.Q1)) return QLORA_ERR_CUDA;
-  } else {
-    tq1 = tq0;
-  }
+  if (!qmap(&maps[1], t.Q0)) return false;
+  if (t.Q1) return qmap(&maps[2], t.Q1);
+  maps[2] = maps[1];
+  return true;
+}
+
+qlora_status run_skinny_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
+  CUtensorMap maps[3];
+  if (!prepare_tc(t, a, ws, L.partials, L.counters, maps)) return QLORA_ERR_CUDA;
   const double flops = 2.0 * a.M * a.C * a.R * a.nq;
   const double bytes = 2.0 * a.M * a.C;
   const bool pdl = g_trace.recs == nullptr;
   TraceScope ts(t.kid, flops, bytes, st);
-  return launch_skinny_tc(a, tp, tq0, tq1, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launch_skinny_tc(a, maps[0], maps[1], maps[2], st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// Two independent products in one grid; the second's partials follow the
+// first's, its counters follow the first's row tiles.
+qlora_status run_skinny_tc_pair(int32_t kid, const TcProduct &t0, SkinnyTcArgs a0, const TcProduct &t1,
+                                SkinnyTcArgs a1, const PairGeom &pg, uint8_t *ws, const WsLayout &L,
+                                cudaStream_t st) {
+  CUtensorMap m0[3], m1[3];
+  const size_t part1 = L.partials + static_cast<size_t>(round_up(static_cast<int64_t>(pg.part0), 256));
+  const size_t cnt1 = L.counters + static_cast<size_t>((a0.M + 127) / 128) * sizeof(uint32_t);
+  if (!prepare_tc(t0, a0, ws, L.partials, L.counters, m0) || !prepare_tc(t1, a1, ws, part1, cnt1, m1))
+    return QLORA_ERR_CUDA;
+  const double flops = 2.0 * (a0.M * a0.C * a0.nq + a1.M * a1.C * a1.nq) * a0.R;
+  const double bytes = 2.0 * (a0.M * a0.C + a1.M * a1.C);
+  const bool pdl = g_trace.recs == nullptr;
+  TraceScope ts(kid, flops, bytes, st);
+  return launch_skinny_tc_pair(a0, m0, a1, m1, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 SkinnyTcArgs tc_args(int64_t M, int64_t C, int R, float alpha) {
@@ -637,17 +672,8 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   const int64_t r64 = round_up(r, 64);
   const int64_t Tp = round_up(T, 8);
   auto plane = [&](size_t off) { return reinterpret_cast<uint16_t *>(w8 + off); };
-  // sU = s X A^T, transposed, as hi + lo planes [r, ceil8(T)]
-  SkinnyTcArgs au = tc_args(T, K, r, s);
-  au.t_hi = plane(L.suT_hi);
-  au.t_lo = plane(L.suT_lo);
-  au.ldt = Tp;
-  const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, geom_u(T, K, r)};
-  qlora_status rs = run_skinny_tc(tu, au, w8, L, st);
-  if (rs != QLORA_OK) return rs;
-  // dU = s dY B: hi plane [T, ceil64(r)] for the dX GEMM, and transposed hi + lo
-  // planes for dA.  TMA reads B in place when its rows are a multiple of 16
-  // bytes (columns past r come back as zeros); otherwise B is first copied to
+  // TMA reads B in place for dU when its rows are a multiple of 16 bytes
+  // (columns past r come back as zeros); otherwise B is first copied to
   // [N, ceil64(r)] rows.
   const void *bq = B;
   int64_t ldb = r;
@@ -659,29 +685,36 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
     bq = bpad;
     ldb = r64;
   }
+  // one grid: sU = s X A^T, transposed, as hi + lo planes [r, ceil8(T)]; and
+  // dU = s dY B as a hi plane [T, ceil64(r)] for the dX GEMM plus transposed hi
+  // + lo planes for dA
+  const PairGeom g1 = geom_u_du(T, N, K, r);
+  SkinnyTcArgs au = tc_args(T, K, r, s);
+  au.t_hi = plane(L.suT_hi);
+  au.t_lo = plane(L.suT_lo);
+  au.ldt = Tp;
   SkinnyTcArgs ad = tc_args(T, N, r, s);
   ad.row_hi = plane(L.du_row);
   ad.ldo = r64;
   ad.t_hi = plane(L.duT_hi);
   ad.t_lo = plane(L.duT_lo);
   ad.ldt = Tp;
-  const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, geom_du(T, N, r)};
-  rs = run_skinny_tc(td, ad, w8, L, st);
+  const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, g1.g0};
+  const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g1};
+  qlora_status rs = run_skinny_tc_pair(K_LORA_U_DU, tu, au, td, ad, g1, w8, L, st);
   if (rs != QLORA_OK) return rs;
   // dX = dY W' + dU A
   rs = run_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
   if (rs != QLORA_OK) return rs;
-  // dB = dY^T (sU) [N, r]
+  // one grid: dB = dY^T (sU) [N, r] and dA = dU^T X [r, K]
+  const PairGeom g2 = geom_db_da(T, N, K, r);
   SkinnyTcArgs ab = tc_args(N, T, r, 1.0f);
   ab.row = static_cast<uint16_t *>(dB);
-  const TcProduct tb = {K_LORA_DB, dy, N, true, plane(L.suT_hi), plane(L.suT_lo), Tp, false, geom_db(T, N, r)};
-  rs = run_skinny_tc(tb, ab, w8, L, st);
-  if (rs != QLORA_OK) return rs;
-  // dA = dU^T X [r, K]
   SkinnyTcArgs aa = tc_args(K, T, r, 1.0f);
   aa.tr = static_cast<uint16_t *>(dA);
-  const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, geom_da(T, K, r)};
-  return run_skinny_tc(ta, aa, w8, L, st);
+  const TcProduct tb = {K_LORA_DB, dy, N, true, plane(L.suT_hi), plane(L.suT_lo), Tp, false, g2.g0};
+  const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
+  return run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, st);
 }
 
 // ---------------------------------------------------------------------------

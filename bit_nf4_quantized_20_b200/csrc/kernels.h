@@ -160,6 +160,14 @@ struct SkinnyTcArgs {
 };
 cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
                              const CUtensorMap &tm_q1, cudaStream_t st, bool pdl);
+// Two independent products sharing one grid and one tile width (the larger of
+// the two), the CTA slots of one wave shared in proportion to their bytes.  Both
+// have R columns and nq Q planes; each has its own partials and counters.
+void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int64_t M1, int64_t C1, bool q_cj1, int R, int nq,
+                         int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1);
+// maps: {P, Q0, Q1} for each product
+cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
+                                  const CUtensorMap *maps1, cudaStream_t st, bool pdl);
 cudaError_t launch_pad_cols(const uint16_t *src, int64_t rows, int cols, uint16_t *dst, int ldd, cudaStream_t st,
                             int num_sms);
 

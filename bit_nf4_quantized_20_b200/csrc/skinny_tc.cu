@@ -97,11 +97,11 @@ __device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, float (&v)[CW]) 
 
 }  // namespace
 
+// One CTA of one product: 128-row tile m_tile, contraction split `split`.
 template <int NB>
-__global__ void __launch_bounds__(TNUM_THREADS, 2)
-    skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q0,
-                     const __grid_constant__ CUtensorMap tm_q1, const SkinnyTcArgs a) {
-  grid_dep_launch();
+__device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CUtensorMap *tm_q0,
+                                               const CUtensorMap *tm_q1, const SkinnyTcArgs &a, int m_tile,
+                                               int split) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   constexpr int CW = NB < 32 ? NB : 32;                  // epilogue chunk (columns)
   constexpr uint32_t TMEM_COLS = NB < 32 ? 32u : static_cast<uint32_t>(NB);
@@ -121,8 +121,6 @@ __global__ void __launch_bounds__(TNUM_THREADS, 2)
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const int m_tile = blockIdx.x;
-  const int split = blockIdx.y;
   const int64_t m0 = static_cast<int64_t>(m_tile) * TBM;
   const int64_t cbeg = static_cast<int64_t>(split) * a.c_per_split;
   const int64_t cend = min(a.C, cbeg + a.c_per_split);
@@ -142,9 +140,9 @@ __global__ void __launch_bounds__(TNUM_THREADS, 2)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_p);
-    tma_prefetch_desc(&tm_q0);
-    if (a.nq > 1) tma_prefetch_desc(&tm_q1);
+    tma_prefetch_desc(tm_p);
+    tma_prefetch_desc(tm_q0);
+    if (a.nq > 1) tma_prefetch_desc(tm_q1);
   }
   tc_fence_before();
   __syncthreads();
@@ -166,13 +164,13 @@ __global__ void __launch_bounds__(TNUM_THREADS, 2)
         const int32_t c0 = static_cast<int32_t>(cbeg + static_cast<int64_t>(st) * TBK);
         mbar_arrive_expect_tx(full(s), stage_bytes);
         if (!a.p_col) {
-          tma_load_2d(stage_p(s), &tm_p, full(s), c0, static_cast<int32_t>(m0));                     // [128 m][64 c]
+          tma_load_2d(stage_p(s), tm_p, full(s), c0, static_cast<int32_t>(m0));                      // [128 m][64 c]
         } else {
-          tma_load_2d(stage_p(s), &tm_p, full(s), static_cast<int32_t>(m0), c0);                     // m 0-63
-          tma_load_2d(stage_p(s) + P_BYTES / 2, &tm_p, full(s), static_cast<int32_t>(m0) + 64, c0);  // m 64-127
+          tma_load_2d(stage_p(s), tm_p, full(s), static_cast<int32_t>(m0), c0);                      // m 0-63
+          tma_load_2d(stage_p(s) + P_BYTES / 2, tm_p, full(s), static_cast<int32_t>(m0) + 64, c0);   // m 64-127
         }
         for (int qi = 0; qi < a.nq; ++qi) {
-          const CUtensorMap *tq = qi ? &tm_q1 : &tm_q0;
+          const CUtensorMap *tq = qi ? tm_q1 : tm_q0;
           if (!a.q_cj) {
             tma_load_2d(stage_q(s, qi), tq, full(s), c0, 0);                                          // [NB j][64 c]
           } else {
@@ -305,6 +303,34 @@ __global__ void __launch_bounds__(TNUM_THREADS, 2)
   }
 }
 
+template <int NB>
+__global__ void __launch_bounds__(TNUM_THREADS, 2)
+    skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q0,
+                     const __grid_constant__ CUtensorMap tm_q1, const SkinnyTcArgs a) {
+  grid_dep_launch();
+  skinny_tc_body<NB>(&tm_p, &tm_q0, &tm_q1, a, static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y));
+}
+
+// Two independent products in one grid (the first ctas0 CTAs run product 0):
+// their ramp-up and split-reduction tails overlap instead of following each other.
+template <int NB>
+__global__ void __launch_bounds__(TNUM_THREADS, 2)
+    skinny_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant__ CUtensorMap tm_q00,
+                          const __grid_constant__ CUtensorMap tm_q10, const __grid_constant__ CUtensorMap tm_p1,
+                          const __grid_constant__ CUtensorMap tm_q01, const __grid_constant__ CUtensorMap tm_q11,
+                          const SkinnyTcArgs a0, const SkinnyTcArgs a1) {
+  grid_dep_launch();
+  const int mt0 = static_cast<int>((a0.M + TBM - 1) / TBM);
+  const int n0 = mt0 * a0.splits;
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < n0) {
+    skinny_tc_body<NB>(&tm_p0, &tm_q00, &tm_q10, a0, b % mt0, b / mt0);
+  } else {
+    const int mt1 = static_cast<int>((a1.M + TBM - 1) / TBM);
+    skinny_tc_body<NB>(&tm_p1, &tm_q01, &tm_q11, a1, (b - n0) % mt1, (b - n0) / mt1);
+  }
+}
+
 // One thread writes 8 consecutive outputs (one 16-byte store); ldd is a
 // multiple of 8.
 __global__ void pad_cols_kernel(const uint16_t *__restrict__ src, int64_t rows, int cols, uint16_t *__restrict__ dst,
@@ -328,14 +354,14 @@ __global__ void pad_cols_kernel(const uint16_t *__restrict__ src, int64_t rows, 
   }
 }
 
-SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int num_sms) {
-  SkinnyTcGeom g;
-  if (q_cj) {
-    g.nb = R <= 64 ? 64 : 128;
-  } else {
-    g.nb = R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128;
-  }
-  const int stage = P_BYTES + nq * g.nb * TBK * 2;
+namespace {
+int tc_nb(int R, bool q_cj) {
+  if (q_cj) return R <= 64 ? 64 : 128;
+  return R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128;
+}
+// Pipeline depth and CTAs per SM for a tile width; returns the CTAs per SM.
+int tc_stages(int nb, int nq, SkinnyTcGeom &g) {
+  const int stage = P_BYTES + nq * nb * TBK * 2;
   int per_sm = 2;
   int stages = (kTwoPerSmBudget - kFixedSmem) / stage;
   if (stages < 3) {
@@ -343,14 +369,18 @@ SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int 
     stages = (kOnePerSmBudget - kFixedSmem) / stage;
   }
   if (stages > TMAX_STAGES) stages = TMAX_STAGES;
+  g.nb = nb;
   g.stages = stages;
   g.smem = stages * stage + kFixedSmem;
   g.splits = 1;
   g.c_per_split = TBK;
-  if (M <= 0 || C <= 0 || num_sms <= 0) return g;
-  // one wave: m_tiles x splits <= the CTAs the GPU holds at once
+  return per_sm;
+}
+// Contraction splits for `slots` CTAs over the 128-row tiles of an M x C product.
+void tc_splits(int64_t M, int64_t C, int64_t slots, SkinnyTcGeom &g) {
+  if (M <= 0 || C <= 0) return;
   const int64_t m_tiles = (M + TBM - 1) / TBM;
-  int64_t s = static_cast<int64_t>(per_sm) * num_sms / m_tiles;
+  int64_t s = slots / m_tiles;
   const int64_t cap = (C + 2 * TBK - 1) / (2 * TBK);      // at least two stages per split
   if (s > cap) s = cap;
   if (s < 1) s = 1;
@@ -358,7 +388,31 @@ SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int 
   per = (per + TBK - 1) / TBK * TBK;
   g.c_per_split = per;
   g.splits = static_cast<int>((C + per - 1) / per);
+}
+}  // namespace
+
+SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int num_sms) {
+  SkinnyTcGeom g;
+  const int per_sm = tc_stages(tc_nb(R, q_cj), nq, g);
+  // one wave: m_tiles x splits <= the CTAs the GPU holds at once
+  if (num_sms > 0) tc_splits(M, C, static_cast<int64_t>(per_sm) * num_sms, g);
   return g;
+}
+
+void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int64_t M1, int64_t C1, bool q_cj1, int R, int nq,
+                         int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1) {
+  const int nb = tc_nb(R, q_cj0) > tc_nb(R, q_cj1) ? tc_nb(R, q_cj0) : tc_nb(R, q_cj1);
+  const int per_sm = tc_stages(nb, nq, g0);
+  tc_stages(nb, nq, g1);
+  if (num_sms <= 0) return;
+  // one wave for both, the slots shared in proportion to the bytes each streams
+  const int64_t slots = static_cast<int64_t>(per_sm) * num_sms;
+  const double b0 = static_cast<double>(M0) * C0, b1 = static_cast<double>(M1) * C1;
+  int64_t s0 = b0 + b1 > 0 ? static_cast<int64_t>(slots * b0 / (b0 + b1) + 0.5) : slots / 2;
+  if (s0 < 1) s0 = 1;
+  if (s0 > slots - 1) s0 = slots - 1;
+  tc_splits(M0, C0, s0, g0);
+  tc_splits(M1, C1, slots - s0, g1);
 }
 
 size_t skinny_tc_partials_bytes(const SkinnyTcGeom &g, int64_t M, int R) {
@@ -403,6 +457,49 @@ cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, con
     case 32: return launch_nb<32>(a, tm_p, tm_q0, tm_q1, st, pdl);
     case 64: return launch_nb<64>(a, tm_p, tm_q0, tm_q1, st, pdl);
     case 128: return launch_nb<128>(a, tm_p, tm_q0, tm_q1, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+namespace {
+template <int NB>
+cudaError_t launch_pair_nb(const SkinnyTcArgs &a0, const CUtensorMap *m0, const SkinnyTcArgs &a1,
+                           const CUtensorMap *m1, cudaStream_t st, bool pdl) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(skinny_tc_pair_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kOnePerSmBudget);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int stage = P_BYTES + a0.nq * NB * TBK * 2;
+  const int64_t n0 = (a0.M + TBM - 1) / TBM * a0.splits, n1 = (a1.M + TBM - 1) / TBM * a1.splits;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(n0 + n1), 1, 1);
+  cfg.blockDim = dim3(TNUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(a0.stages * stage + kFixedSmem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, skinny_tc_pair_kernel<NB>, m0[0], m0[1], m0[2], m1[0], m1[1], m1[2], a0, a1);
+}
+}  // namespace
+
+cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
+                                  const CUtensorMap *maps1, cudaStream_t st, bool pdl) {
+  if (a0.M <= 0 || a0.C <= 0 || a1.M <= 0 || a1.C <= 0 || a0.R <= 0) return cudaErrorInvalidValue;
+  if (a0.nb != a1.nb || a0.nq != a1.nq || a0.stages != a1.stages) return cudaErrorInvalidValue;
+  if (a0.stages < 1 || a0.stages > TMAX_STAGES || a0.splits < 1 || a1.splits < 1 || (a0.nq != 1 && a0.nq != 2))
+    return cudaErrorInvalidValue;
+  if ((a0.q_cj || a1.q_cj) && a0.nb < 64) return cudaErrorInvalidValue;
+  switch (a0.nb) {
+    case 16: return launch_pair_nb<16>(a0, maps0, a1, maps1, st, pdl);
+    case 32: return launch_pair_nb<32>(a0, maps0, a1, maps1, st, pdl);
+    case 64: return launch_pair_nb<64>(a0, maps0, a1, maps1, st, pdl);
+    case 128: return launch_pair_nb<128>(a0, maps0, a1, maps1, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
