@@ -170,6 +170,8 @@ bool codebook_symmetric(const float *cb) {
 // Up to this many tokens the forward runs the decode GEMV, and U = s X A^T
 // runs on the mma.sync kernel (a handful of rows: latency, not bandwidth).
 constexpr int64_t kGemvMaxTokens = 16;
+// the split counters of the decode GEMV are the workspace's tile counters
+constexpr int kGemvMaxCounterTiles = static_cast<int>(kWsCounterBytes / sizeof(uint32_t));
 
 bool decode_path(int64_t T, int64_t N) {
   (void)N;
@@ -223,7 +225,9 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   if (op == QLORA_OP_FWD) {
     L.su_row = off; off += row_plane;
     if (decode_path(T, N)) {
-      part = skinny_partials_bytes(T, K, r, kSplitSms);
+      // the U' fallback's partials, then (after it has finished) the GEMV's split partials
+      part = std::max(skinny_partials_bytes(T, K, r, kSplitSms),
+                      gemv_persist_partials_bytes(N, K, kGemvMaxCounterTiles));
     } else {
       part = skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
     }
@@ -345,6 +349,7 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
 }
 
 
+// The decode forward; u holds U' = BF16(s X A^T) [T, ldu].
 qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
                       const void *B, int r, void *y, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
   GemvParams p;
@@ -363,6 +368,9 @@ qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, cons
   p.r = r;
   p.y = static_cast<uint16_t *>(y);
   p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
+  p.ctas = gemv_persist_ctas(p.N, p.K, num_sms_current(), kGemvMaxCounterTiles);
+  p.part = reinterpret_cast<float *>(ws + L.partials);
+  p.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
   const double n = static_cast<double>(p.N) * p.K;
   const double bytes = n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * T * (p.N + p.K) +
                        2.0 * static_cast<double>(p.N) * r;

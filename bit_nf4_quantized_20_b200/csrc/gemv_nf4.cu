@@ -32,6 +32,8 @@
 // (and, after the dependency wait, of X) at once, and the partial sums meet
 // in rank 0's shared memory.
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,9 +95,9 @@ __device__ __forceinline__ uint32_t ldg_pair_bf16(const uint16_t *p, int64_t i0,
 // tokens, a second MMA for tokens 8-15).  Accumulator: c0/c1 = (row r0, tokens
 // 2t, 2t + 1), c2/c3 = (row r0 + 8, tokens 2t, 2t + 1).
 
-// rank-r term and store for 16-row tile `tile`: v += B U'^T (k16-steps over r), Y = BF16(v)
+// rank-r term for 16-row tile `tile`: v += B U'^T (k16-steps over r)
 template <int TT>
-__device__ __forceinline__ void gemv_finish(const GemvParams &p, int64_t tile, int g, int t, float (&v)[TT / 8][4]) {
+__device__ __forceinline__ void gemv_lora(const GemvParams &p, int64_t tile, int g, int t, float (&v)[TT / 8][4]) {
   const int64_t r0 = tile * 16 + g, r1 = r0 + 8;
   const bool v0 = r0 < p.N, v1 = r1 < p.N;
   const int rv = p.r;
@@ -117,6 +119,13 @@ __device__ __forceinline__ void gemv_finish(const GemvParams &p, int64_t tile, i
       mma16816(v[h], a0, a1, a2, a3, b0, b1);
     }
   }
+}
+
+// Y = BF16(v) for the rows and tokens of tile `tile` that exist
+template <int TT>
+__device__ __forceinline__ void gemv_store(const GemvParams &p, int64_t tile, int g, int t, const float (&v)[TT / 8][4]) {
+  const int64_t r0 = tile * 16 + g, r1 = r0 + 8;
+  const bool v0 = r0 < p.N, v1 = r1 < p.N;
 #pragma unroll
   for (int h = 0; h < TT / 8; ++h) {
     const int ta = 8 * h + 2 * t, tb = ta + 1;
@@ -307,7 +316,339 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32) nf4_gemv_kernel(const Gemv
       }
     }
   }
-  if (warp == 0) gemv_finish<TT>(p, tile, g, t, acc);
+  if (warp == 0) {
+    gemv_lora<TT>(p, tile, g, t, acc);
+    gemv_store<TT>(p, tile, g, t, acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent GEMV for K a multiple of 256: the same per-code work as the kernel
+// above (each lane converts whole 64-weight blocks with a per-block register
+// table of BF16(RN32(codebook[j] * scale)), so W' is the dequantization's to
+// the bit), with the work spread for bandwidth rather than one CTA per tile.
+//
+// The 16 x 256 units are numbered tile-major (unit = tile * KU + k-unit) and
+// cut into C equal contiguous ranges, one per CTA, each cut again into
+// contiguous chunks, one per warp.  A warp streams its chunk through a private
+// cp.async ring of kPGD units (the 16 x 128-byte code tile stored with a
+// 128-byte swizzle, so that each lane's 32-byte block loads without bank
+// conflicts) and keeps one tile's sums at a time.  When a tile ends:
+//   - a tile inside the warp's chunk is finished by the warp: rank-r term
+//     B U'^T, then BF16 Y;
+//   - a tile shared with other warps of the CTA leaves its sums in the warp's
+//     shared-memory slot (slot 0 for the chunk's first tile, 1 for its last);
+//     the last of those warps to arrive (a shared-memory counter) adds the
+//     slots in warp order and, if the tile lies inside the CTA's range,
+//     finishes it;
+//   - a tile shared with another CTA leaves the CTA's sum in the split
+//     workspace (slot 0 / 1 as above, per CTA); the last CTA to arrive (a
+//     workspace counter per tile, zeroed again after use) adds them in CTA
+//     order and finishes the tile.
+// Every sum is taken in a fixed order, so a launch's result does not depend on
+// timing.  No thread waits on another warp or CTA.  U' (from the preceding
+// kernel) is copied to shared memory once per CTA after the dependency wait.
+// ---------------------------------------------------------------------------
+// A CTA is 8 warps with about 86 KB of shared memory and 32K registers, so that
+// two CTAs fit on an SM: those of one launch, or one of this launch and one of
+// the next (which then requests its weights while this one runs).
+#ifndef QLORA_PERSIST_CTAS_PER_SM
+#define QLORA_PERSIST_CTAS_PER_SM 2
+#endif
+constexpr int kPWarps = 8;
+constexpr int kPThreads = 32 * kPWarps;
+constexpr int kPGD = 4;                            // units per warp ring (3 in flight)
+constexpr int kPStage = 2048 + 64 + 64;            // codes [16][128] swizzled, scale words [16], c2 [16]
+constexpr int kPRing = kPWarps * kPGD * kPStage;
+constexpr int kPSlotFloats = 16 * 16;              // one tile's sums: [T <= 16][16 rows]
+constexpr int kPUBytes = 16 * 128 * 2;             // U' [T <= 16][ldu <= 128] BF16
+constexpr int kPSmem = kPRing + kPWarps * 2 * kPSlotFloats * 4 + kPWarps * 2 * 4 + kPUBytes;
+constexpr int kPCtasPerSm = QLORA_PERSIST_CTAS_PER_SM;
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// lane (g, t) values of one tile's sums in a [T][16] float array: v[h][e] is
+// (row g + 8 (e >> 1), token 8 h + 2 t + (e & 1))
+template <int NH, typename F>
+__device__ __forceinline__ void for_tile_values(int T, int g, int t, F &&f) {
+#pragma unroll
+  for (int h = 0; h < NH; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = 8 * h + 2 * t + (e & 1), row = g + 8 * (e >> 1);
+      if (tok < T) f(h, e, tok * 16 + row);
+    }
+}
+
+template <int TT, bool SYM>
+__global__ void __launch_bounds__(kPThreads, 2) nf4_gemv_persist_kernel(const GemvParams p) {
+  extern __shared__ __align__(128) uint8_t psm[];
+  constexpr int NH = TT / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  float *slots = reinterpret_cast<float *>(psm + kPRing);                          // [warp][2][kPSlotFloats]
+  // one counter per (first contributing warp, that warp's slot) of each shared tile
+  uint32_t *scnt = reinterpret_cast<uint32_t *>(psm + kPRing + kPWarps * 2 * kPSlotFloats * 4);   // [warp][2]
+  uint16_t *su = reinterpret_cast<uint16_t *>(psm + kPRing + kPWarps * 2 * kPSlotFloats * 4 + kPWarps * 2 * 4);
+  const uint32_t ring = smem_u32(psm) + warp * (kPGD * kPStage);
+  const int KU = p.units;
+  const int64_t KB = p.K / 64, rowbytes = p.K / 2;
+  const int64_t U = static_cast<int64_t>(p.tiles) * KU, C = gridDim.x;
+  // this CTA's units [ub, ue) and this warp's chunk [wb, we)
+  auto cta_begin = [&](int64_t c) { return c * U / C; };
+  const int64_t ub = cta_begin(blockIdx.x), ue = cta_begin(blockIdx.x + 1), n = ue - ub;
+  const int64_t weff = min(static_cast<int64_t>(kPWarps), n);
+  auto warp_begin = [&](int64_t w) { return ub + w * n / weff; };
+  const int64_t wb = warp < weff ? warp_begin(warp) : ue, we = warp < weff ? warp_begin(warp + 1) : ue;
+  auto owner_warp = [&](int64_t x) { return ((x - ub + 1) * weff - 1) / n; };
+  auto owner_cta = [&](int64_t x) { return ((x + 1) * C - 1) / U; };
+
+  if (threadIdx.x < 2 * kPWarps) scnt[threadIdx.x] = 0u;
+  // Even warps walk their chunk forwards and odd warps backwards, so that of
+  // two neighbouring warps sharing a tile one reaches it first, and a CTA's
+  // last warp (odd) starts with the tile it may share with the next CTA.
+  const bool rev = (warp & 1) != 0;
+  const int64_t cnt = we - wb;
+  const int64_t x0 = rev ? we - 1 : wb;
+  auto step = [&](int64_t &tl, int &uu) {
+    if (!rev) {
+      if (++uu == KU) {
+        uu = 0;
+        ++tl;
+      }
+    } else if (--uu < 0) {
+      uu = KU - 1;
+      --tl;
+    }
+  };
+
+  // the next unit into ring slot `slot`: lane L copies 16-byte chunks L + 32 j of
+  // the code tile (row L / 8 + 4 j, column L % 8), lanes 0-15 the scale words and
+  // lanes 16-31 the c2 of rows 0-15 (one commit group per unit, empty past the end)
+  const int crow = lane >> 3, ccol = lane & 7;
+  int64_t inext = 0, itile = x0 / KU;
+  int iu = static_cast<int>(x0 - itile * KU);
+  auto issue = [&](int slot) {
+    if (inext < cnt) {
+      const uint32_t st = ring + slot * kPStage;
+      const int64_t n0 = itile * 16;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = crow + 4 * j;
+        const bool ok = n0 + row < p.N;
+        const uint8_t *src = p.codes + (ok ? (n0 + row) * rowbytes + static_cast<int64_t>(iu) * 128 + ccol * 16 : 0);
+        cp_async16(st + row * 128 + ((ccol ^ (row & 7)) << 4), src, ok ? 16u : 0u);
+      }
+      const int row = lane & 15;
+      const bool ok = n0 + row < p.N;
+      const int64_t blk = ok ? (n0 + row) * KB + 4 * static_cast<int64_t>(iu) : 0;
+      if (lane < 16) cp_async4(st + 2048 + row * 4, p.scales + blk, ok ? 4u : 0u);
+      else cp_async4(st + 2112 + row * 4, p.c2 + (blk >> 8), ok ? 4u : 0u);
+      step(itile, iu);
+    }
+    ++inext;
+    cp_async_commit();
+  };
+
+#pragma unroll 1
+  for (int s = 0; s < kPGD - 1; ++s) issue(s);   // the weights do not depend on the preceding kernel
+  __syncthreads();                                        // the shared counters are zero
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dep_wait();   // X, U', Y and the split workspace may
+  // U' into shared memory, once for all the CTA's rank-r terms
+  {
+    const int words = p.T * static_cast<int>(p.ldu) / 8;
+    for (int i = threadIdx.x; i < words; i += kPThreads)
+      reinterpret_cast<uint4 *>(su)[i] = reinterpret_cast<const uint4 *>(p.u)[i];
+  }
+  __syncthreads();
+  GemvParams pl = p;   // the rank-r term reads U' from shared memory
+  pl.u = su;
+
+  float acc[NH][4], acc2[NH][4];   // even / odd k16-steps (two independent MMA chains)
+#pragma unroll
+  for (int h = 0; h < NH; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[h][e] = acc2[h][e] = 0.f;
+  // token rows this lane feeds to the MMA (rows past T repeat row T - 1; their
+  // accumulator columns are never stored)
+  const uint16_t *xrow0[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) xrow0[h] = p.x + static_cast<int64_t>(min(8 * h + g, p.T - 1)) * p.K + 64 * t;
+
+  int64_t tile = x0 / KU;
+  int u = static_cast<int>(x0 - tile * KU);
+  int slot = 0;
+  bool seg_start = true;
+  const int64_t brow_bytes = 2 * static_cast<int64_t>(p.r) * 16;   // one tile's rows of B
+#pragma unroll 1
+  for (int64_t i = 0; i < cnt; ++i) {
+    issue((slot + kPGD - 1) % kPGD);
+    if (seg_start) {
+      // the tile's rows of B, for whichever warp finishes it
+      const int64_t off = static_cast<int64_t>(lane) * 128;
+      if (off < brow_bytes && tile * 16 + off / (2 * p.r) < p.N)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const uint8_t *>(p.B) + tile * brow_bytes + off));
+      seg_start = false;
+    }
+    const uint16_t *xrow[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) xrow[h] = xrow0[h] + static_cast<int64_t>(u) * 256;
+    uint32_t xf[NH][8], xn[NH][8];
+    load_x_chunk<NH>(xrow, true, 0, xf);
+    cp_async_wait<kPGD - 1>();   // this lane's copies of the unit have landed
+    __syncwarp();                // and every lane's
+    const uint32_t st = ring + slot * kPStage;
+    // block t of rows g and g + 8: its scale, and its 32 code bytes (chunks 2t, 2t + 1)
+    float scale[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t sword = lds32(st + 2048 + (g + 8 * h) * 4);
+      const float c2v = __uint_as_float(lds32(st + 2112 + (g + 8 * h) * 4));
+      scale[h] = __fmul_rn(e4m3_to_float((sword >> (8 * t)) & 0xffu), c2v);
+    }
+    const uint32_t r0a = st + g * 128, r1a = st + (g + 8) * 128;
+    const uint4 q0[2] = {lds128(r0a + (((2 * t) ^ g) << 4)), lds128(r0a + (((2 * t + 1) ^ g) << 4))};
+    const uint4 q1[2] = {lds128(r1a + (((2 * t) ^ g) << 4)), lds128(r1a + (((2 * t + 1) ^ g) << 4))};
+    __syncwarp();   // every lane has read the slot before it is refilled
+    slot = (slot + 1) % kPGD;
+    // four chunks of 16 codes per row (k16-steps 4c .. 4c + 3); X of the next chunk is loaded ahead
+    if constexpr (SYM) {
+      const Lut8 l0 = make_lut8(p.codebook, scale[0]);
+      const Lut8 l1 = make_lut8(p.codebook, scale[1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c < 3) load_x_chunk<NH>(xrow, true, c + 1, xn);
+        const uint4 &v0 = q0[c >> 1], &v1 = q1[c >> 1];
+        const uint32_t w0[2] = {(c & 1) ? v0.z : v0.x, (c & 1) ? v0.w : v0.y};
+        const uint32_t w1[2] = {(c & 1) ? v1.z : v1.x, (c & 1) ? v1.w : v1.y};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          uint32_t a[4], b[4];
+          lut8_lookup8(l0, w0[e], a[0], a[1], a[2], a[3]);
+          lut8_lookup8(l1, w1[e], b[0], b[1], b[2], b[3]);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            mma16816(acc[h], a[0], b[0], a[1], b[1], xf[h][4 * e], xf[h][4 * e + 1]);
+            mma16816(acc2[h], a[2], b[2], a[3], b[3], xf[h][4 * e + 2], xf[h][4 * e + 3]);
+          }
+        }
+        if (c < 3) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xf[h][q] = xn[h][q];
+        }
+      }
+    } else {
+      const Lut16 l0 = make_lut16(p.codebook, scale[0]);
+      const Lut16 l1 = make_lut16(p.codebook, scale[1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c < 3) load_x_chunk<NH>(xrow, true, c + 1, xn);
+        const uint4 &v0 = q0[c >> 1], &v1 = q1[c >> 1];
+        const uint32_t w0[2] = {(c & 1) ? v0.z : v0.x, (c & 1) ? v0.w : v0.y};
+        const uint32_t w1[2] = {(c & 1) ? v1.z : v1.x, (c & 1) ? v1.w : v1.y};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t s0 = w0[k >> 1], s1 = w1[k >> 1];
+          uint32_t a0, a2, a1, a3;
+          lut16_lookup4(l0, (k & 1) ? (s0 >> 16) : s0, a0, a2);
+          lut16_lookup4(l1, (k & 1) ? (s1 >> 16) : s1, a1, a3);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            if (k & 1) mma16816(acc2[h], a0, a1, a2, a3, xf[h][2 * k], xf[h][2 * k + 1]);
+            else mma16816(acc[h], a0, a1, a2, a3, xf[h][2 * k], xf[h][2 * k + 1]);
+          }
+        }
+        if (c < 3) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xf[h][q] = xn[h][q];
+        }
+      }
+    }
+
+    if (i + 1 == cnt || (rev ? u == 0 : u + 1 == KU)) {
+      seg_start = true;
+      // the end of this warp's part of the tile
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[h][e] += acc2[h][e];
+          acc2[h][e] = 0.f;
+        }
+      const int64_t t0 = tile * KU, t1 = t0 + KU;   // the tile's units
+      if (t0 >= wb && t1 <= we) {
+        gemv_lora<TT>(pl, tile, g, t, acc);
+        gemv_store<TT>(p, tile, g, t, acc);
+      } else {
+        float *mine = slots + (warp * 2 + (t0 <= wb ? 0 : 1)) * kPSlotFloats;
+        for_tile_values<NH>(p.T, g, t, [&](int h, int e, int i) { mine[i] = acc[h][e]; });
+        const int64_t wf = owner_warp(max(ub, t0)), wl = owner_warp(min(ue, t1) - 1);
+        __threadfence_block();
+        __syncwarp();
+        uint32_t old = 0;
+        if (lane == 0) old = atomicAdd(scnt + 2 * wf + (t0 <= warp_begin(wf) ? 0 : 1), 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == static_cast<uint32_t>(wl - wf)) {
+          // the CTA's last warp on this tile: its sum over the CTA's warps, in warp order
+          __threadfence_block();
+          float sum[NH][4];
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sum[h][e] = 0.f;
+          for (int64_t w2 = wf; w2 <= wl; ++w2) {
+            const float *src = slots + (w2 * 2 + (t0 <= warp_begin(w2) ? 0 : 1)) * kPSlotFloats;
+            for_tile_values<NH>(p.T, g, t, [&](int h, int e, int i) { sum[h][e] += src[i]; });
+          }
+          if (t0 >= ub && t1 <= ue) {
+            gemv_lora<TT>(pl, tile, g, t, sum);
+            gemv_store<TT>(p, tile, g, t, sum);
+          } else {
+            // shared with another CTA: leave the CTA's sum in the workspace
+            float *gp = p.part + (static_cast<int64_t>(blockIdx.x) * 2 + (t0 <= ub ? 0 : 1)) * kPSlotFloats;
+            for_tile_values<NH>(p.T, g, t, [&](int h, int e, int i) { gp[i] = sum[h][e]; });
+            __threadfence();
+            __syncwarp();
+            uint32_t gold = 0;
+            if (lane == 0) gold = atomicAdd(p.counters + tile, 1u);
+            gold = __shfl_sync(0xffffffffu, gold, 0);
+            const int64_t cf = owner_cta(t0), cl = owner_cta(t1 - 1);
+            if (gold == static_cast<uint32_t>(cl - cf)) {
+              // the last CTA on this tile: the CTAs' sums in CTA order
+              __threadfence();
+              float tot[NH][4];
+#pragma unroll
+              for (int h = 0; h < NH; ++h)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) tot[h][e] = 0.f;
+              for (int64_t c2 = cf; c2 <= cl; ++c2) {
+                const float *src = p.part + (c2 * 2 + (t0 <= cta_begin(c2) ? 0 : 1)) * kPSlotFloats;
+                for_tile_values<NH>(p.T, g, t, [&](int h, int e, int i) { tot[h][e] += __ldcg(src + i); });
+              }
+              gemv_lora<TT>(pl, tile, g, t, tot);
+              gemv_store<TT>(p, tile, g, t, tot);
+              if (lane == 0) p.counters[tile] = 0u;   // zero again for the next call
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+    }
+    step(tile, u);
+  }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -525,9 +866,58 @@ cudaError_t launch_lora_u_decode(const LoraUDecodeParams &p_in, cudaStream_t st,
   return p.T > 8 ? launch_u<16>(p, smem, st, pdl) : launch_u<8>(p, smem, st, pdl);
 }
 
-cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl) {
+int gemv_persist_ctas(int64_t N, int64_t K, int num_sms, int max_tiles) {
+  if (K % 256 != 0 || K <= 0 || N <= 0) return 0;
+  const int64_t tiles = (N + 15) / 16, units = tiles * (K / 256);
+  if (tiles > max_tiles || units > (int64_t(1) << 40)) return 0;
+  // one whole tile per CTA when the tiles fit in the resident CTAs (no tile is
+  // then shared between CTAs), otherwise every resident CTA with an equal share
+  const int64_t slots = std::min<int64_t>(static_cast<int64_t>(num_sms) * kPCtasPerSm, kPersistMaxCtas);
+  return static_cast<int>(tiles <= slots ? tiles : std::min<int64_t>(units, slots));
+}
+
+size_t gemv_persist_partials_bytes(int64_t N, int64_t K, int max_tiles) {
+  if (gemv_persist_ctas(N, K, kPersistMaxCtas, max_tiles) == 0) return 0;
+  return static_cast<size_t>(kPersistMaxCtas) * 2 * kPSlotFloats * sizeof(float);
+}
+
+namespace {
+template <int TT, bool SYM>
+cudaError_t launch_persist(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(nf4_gemv_persist_kernel<TT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.ctas), 1, 1);
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, nf4_gemv_persist_kernel<TT, SYM>, p);
+}
+}  // namespace
+
+cudaError_t launch_gemv(const GemvParams &p_in, int num_sms, cudaStream_t st, bool pdl) {
+  const GemvParams &p = p_in;
   if (p.T < 1 || p.T > 16 || p.N % 8 != 0 || p.K % 64 != 0 || num_sms < 1) return cudaErrorInvalidValue;
   const bool t16 = p.T > 8;
+  if (p.ctas > 0) {
+    GemvParams q = p;
+    q.units = static_cast<int>(p.K / 256);
+    q.tiles = static_cast<int>((p.N + 15) / 16);
+    q.ctas = std::min(p.ctas, num_sms * kPCtasPerSm);
+    if (p.K % 256 != 0 || !q.part || !q.counters || p.ldu > 128 || p.ldu % 8 != 0) return cudaErrorInvalidValue;
+    if (q.sym) return t16 ? launch_persist<16, true>(q, num_sms, st, pdl) : launch_persist<8, true>(q, num_sms, st, pdl);
+    return t16 ? launch_persist<16, false>(q, num_sms, st, pdl) : launch_persist<8, false>(q, num_sms, st, pdl);
+  }
   if (p.sym) return t16 ? launch_t<16, true>(p, num_sms, st, pdl) : launch_t<8, true>(p, num_sms, st, pdl);
   return t16 ? launch_t<16, false>(p, num_sms, st, pdl) : launch_t<8, false>(p, num_sms, st, pdl);
 }

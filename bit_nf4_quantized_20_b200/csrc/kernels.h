@@ -70,6 +70,12 @@ struct GemvParams {
   uint16_t *y;           // [T, N]
   int sym;               // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   int units, upw, splits;  // filled from the plan
+  // persistent kernel (K % 256 == 0): `ctas` CTAs (0 = per-tile kernel), the
+  // sums of the tiles that straddle two CTAs [kPersistMaxCtas][2][16][16] fp32, and
+  // one counter per 16-row tile (zero between calls)
+  int tiles, ctas;
+  float *part;
+  uint32_t *counters;
 };
 struct GemvPlan {
   int units;       // 256-wide k-units per row
@@ -78,6 +84,13 @@ struct GemvPlan {
   int tiles;       // 16-row tiles = CTAs
 };
 int gemv_smem_bytes(int splits);
+// CTAs of the persistent GEMV for an N x K weight on `num_sms` SMs (0 when it
+// does not apply: K % 256 != 0 or more 16-row tiles than `max_tiles` counters),
+// and the workspace its straddling tiles need (independent of the device)
+constexpr int64_t kPersistMaxCtas = 1024;
+int gemv_persist_ctas(int64_t N, int64_t K, int num_sms, int max_tiles);
+size_t gemv_persist_partials_bytes(int64_t N, int64_t K, int max_tiles);
+// launches the persistent kernel when p.ctas > 0, else the per-tile kernel
 cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl);
 
 // U' = BF16(alpha X A^T) [T, ldu] for T <= 16 (gemv_nf4.cu); columns r .. ldu - 1 are written as zero.

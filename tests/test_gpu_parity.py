@@ -224,6 +224,10 @@ def test_layer_8b_q_projection_full_size_sampled():
     (9, 4096, 14336),     # 8B down projection: 56 k-units, 7-CTA cluster, 9..16-token variant
     (16, 14336, 4096),    # 8B gate/up projection
     (3, 40, 320),         # ragged rows and a k-unit with a missing block
+    (5, 1032, 768),       # last 16-row tile half empty (table-lookup kernel)
+    (13, 2048, 2560),     # 9..16 tokens, one k-unit per split, ten splits
+    (2, 40000, 1792),     # seven k-units in three splits of 2, 2 and 3 units
+    (2, 113664, 512),     # enough rows that each tile is one item (no split partials)
 ])
 def test_decode_forward(T, N, K):
     """Decode-sized forward (T <= 16): rank 64, s = 1, as in the decode sweep."""
