@@ -137,6 +137,45 @@ def test_nonfinite_weight_is_reported():
     q.get_error()   # cleared
 
 
+def test_stack_8b_32_layers_quantize_storage_roundtrip():
+    """Every linear weight of a 32-layer Llama-3.1-8B-shaped stack (hidden 4096,
+    ffn 14336, 8 KV heads of dim 128: 6.98e9 parameters), BF16 N(0, 0.02^2),
+    quantized on the GPU.  Storage is exactly 4 + 0.127 bits per parameter
+    ("What is QLoRA?"); dequantize then quantize gives back the same codes,
+    scale bytes and c2 on every matrix; layer 0's seven matrices match the
+    oracle bit for bit on their first, a middle and their last two 256-block
+    groups (group-aligned, so each range quantizes on its own)."""
+    q = Q()
+    G = 64 * 256                     # weights per second-level group
+    total_w = total_b = 0
+    for layer in range(32):
+        for i, (name, N, K) in enumerate(inputs.LLAMA8B_PROJ):
+            W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(3, layer, i, "W"), "cuda")
+            qw = q.quantize_nf4(W)
+            qw2 = q.quantize_nf4(q.dequantize(qw))
+            q.get_error()
+            assert torch.equal(qw2.codes, qw.codes), f"layer {layer} {name}: codes"
+            assert torch.equal(qw2.scales, qw.scales), f"layer {layer} {name}: scales"
+            assert torch.equal(qw2.c2.view(torch.int32), qw.c2.view(torch.int32)), f"layer {layer} {name}: c2"
+            n = N * K
+            total_w += n
+            total_b += qw.codes.numel() + qw.scales.numel() + 4 * qw.c2.numel()
+            if layer == 0:
+                w = bits(W).reshape(-1)
+                g_codes, g_scales = qw.codes.cpu().numpy(), qw.scales.cpu().numpy()
+                g_c2 = qw.c2.cpu().numpy().view(np.uint32)
+                for a in (0, (n // 2) // G * G, n - 2 * G):
+                    b = a + 2 * G
+                    codes, scales, c2 = O.quantize_nf4(w[a:b].reshape(-1, 64))
+                    assert np.array_equal(g_codes[a // 2:b // 2], codes), f"{name}: codes at {a}"
+                    assert np.array_equal(g_scales[a // 64:b // 64], scales), f"{name}: scales at {a}"
+                    assert np.array_equal(g_c2[a // G:b // G], c2.view(np.uint32)), f"{name}: c2 at {a}"
+            del W, qw, qw2
+    assert total_w == 32 * sum(N * K for (_, N, K) in inputs.LLAMA8B_PROJ)
+    assert round(total_w / 1e9, 2) == 6.98
+    assert total_b * 8 / total_w == O.bits_per_param()
+
+
 # --------------------------------------------------------------------------
 # forward / backward
 # --------------------------------------------------------------------------
@@ -210,6 +249,33 @@ def test_layer_8b_q_projection_full_size_sampled():
     (X, A, B, dY), wd, (y, dx, dA, dB) = run_layer(T, N, K, r, s, config=1)
     xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
     rows = np.array([0, 1, 255, 256, 1000, 2047, 2048, 3333, 4094, 4095])
+    assert_close("Y[rows]", y[torch.from_numpy(rows).cuda()], O.linear_fwd(xb[rows], wd, ab, bb, s))
+    Xf, Wf, Af, Bf, G = (O.bf16_bits_to_f32(v).astype(np.float64) for v in (xb, wd, ab, bb, dyb))
+    dU = s * (G @ Bf)
+    assert_close("dX[rows]", dx[torch.from_numpy(rows).cuda()], G[rows] @ Wf + dU[rows] @ Af)
+    assert_close("dA", dA, dU.T @ Xf)
+    assert_close("dB", dB, s * (G.T @ (Xf @ Af.T)))
+
+
+@pytest.mark.parametrize("name,N,K", [("q", 8192, 8192), ("down", 8192, 22016)])
+def test_layer_65b_shapes_full_size_sampled(name, N, K):
+    """A 65B-shaped projection (hidden 8192, ffn 22016; the q/k/v/o and down
+    shapes), fwd + bwd on 4 x 512 = 2048 tokens, rank 64, s = 0.25, as in the
+    layer-by-layer run.  Quantize in full; Y and dX on sampled tokens (every
+    output feature); dA and dB in full."""
+    T, r, s = 2048, 64, 0.25
+    i = {"q": 0, "down": 6}[name]
+    W, X, A, B, dY = inputs.layer_inputs(4, 0, i, T, N, K, r, device="cuda")
+    q = Q()
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    del W
+    y = q.linear_fwd(X, qw, A, B, s)
+    dx, dA, dB = q.linear_bwd(dY, X, qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    rows = np.array([0, 1, 511, 512, 1023, 1500, 2046, 2047])
     assert_close("Y[rows]", y[torch.from_numpy(rows).cuda()], O.linear_fwd(xb[rows], wd, ab, bb, s))
     Xf, Wf, Af, Bf, G = (O.bf16_bits_to_f32(v).astype(np.float64) for v in (xb, wd, ab, bb, dyb))
     dU = s * (G @ Bf)
