@@ -223,7 +223,9 @@ def bench_ours(args, rank, world, local_rank):
     q.get_error(dev)
     ms = start.elapsed_time(stop) / args.steps
     # per-kernel breakdown: the same steps again with an event pair around every
-    # launch (outside the timed region: the events serialise the launches)
+    # launch (outside the timed region: the events serialise the launches, and
+    # the backward's dB/dA products then run on the caller's stream instead of
+    # beside the dX GEMM, so that every pair of events times one launch alone)
     with tracer:
         for _ in range(args.steps):
             run_step(layers, s)

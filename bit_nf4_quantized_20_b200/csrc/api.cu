@@ -79,6 +79,33 @@ int num_sms_current() {
   return cache[dev];
 }
 
+// A second stream (and its fork / join events) per host thread and device: the
+// backward runs its adapter-gradient products there, beside the dX GEMM, whose
+// last partial round of tiles leaves SMs idle.  Created on first use, kept
+// until exit; nullptr if the device refuses (the caller then stays on one stream).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool tried = false;
+};
+
+SideStream *side_stream() {
+  thread_local SideStream cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream &ss = cache[dev];
+  if (!ss.tried) {
+    ss.tried = true;
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      ss.s = nullptr;
+      (void)cudaGetLastError();
+    }
+  }
+  return ss.s ? &ss : nullptr;
+}
+
 // Splits of the rank-r GEMMs are sized for a fixed CTA target so that the
 // workspace size does not depend on the device.
 constexpr int kSplitSms = 148;
@@ -711,10 +738,9 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g1};
   qlora_status rs = run_skinny_tc_pair(K_LORA_U_DU, tu, au, td, ad, g1, w8, L, st);
   if (rs != QLORA_OK) return rs;
-  // dX = dY W' + dU A
-  rs = run_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
-  if (rs != QLORA_OK) return rs;
-  // one grid: dB = dY^T (sU) [N, r] and dA = dU^T X [r, K]
+  // one grid: dB = dY^T (sU) [N, r] and dA = dU^T X [r, K]; it needs only the
+  // planes above, so it runs on the side stream beside the dX GEMM (which
+  // touches no other workspace than the status word) and joins before return
   const PairGeom g2 = geom_db_da(T, N, K, r);
   SkinnyTcArgs ab = tc_args(N, T, r, 1.0f);
   ab.row = static_cast<uint16_t *>(dB);
@@ -722,7 +748,19 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   aa.tr = static_cast<uint16_t *>(dA);
   const TcProduct tb = {K_LORA_DB, dy, N, true, plane(L.suT_hi), plane(L.suT_lo), Tp, false, g2.g0};
   const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
-  return run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, st);
+  // (with a trace attached everything stays on the caller's stream, so that each
+  // launch's events time that launch alone)
+  SideStream *side = g_trace.recs == nullptr ? side_stream() : nullptr;
+  if (side && cudaEventRecord(side->fork, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  // dX = dY W' + dU A, first in line for the SMs
+  rs = run_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
+  if (rs != QLORA_OK) return rs;
+  if (!side) return run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, st);
+  if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
+  rs = run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, side->s);
+  if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return rs;
 }
 
 // ---------------------------------------------------------------------------

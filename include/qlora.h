@@ -176,6 +176,11 @@ QLORA_API qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf
  * dy[T, N], x[T, K], A[r, K], B[N, r]; outputs dx[T, K], dA[r, K], dB[N, r]
  * (BF16, overwritten, not accumulated).  Same requirements as the forward.
  * ws: at least qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r) bytes.
+ * Streams: all work is ordered on `stream`; dB and dA are computed on a
+ * library-owned second stream (one per host thread and device, forked from and
+ * joined back into `stream` with events, so graph capture of `stream` captures
+ * it too) beside the dX GEMM.  With a trace attached everything runs on
+ * `stream`.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.
  */
 QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
@@ -215,7 +220,8 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const void *x, int64_t T, const 
 /*
  * Launch trace (profiling hook).  While attached, every kernel the library
  * launches records recs[i].start before and recs[i].stop after it on the
- * call's stream (cudaEvent_t handles the caller created), and fills kernel id,
+ * call's stream (cudaEvent_t handles the caller created; launches then run one
+ * after another on that stream), and fills kernel id,
  * units and the algorithmic work of that launch.  *count counts the launches;
  * launches beyond `capacity` are counted but not recorded.  Pass recs = NULL
  * to detach.  Process-wide; not thread-safe.

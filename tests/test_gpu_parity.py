@@ -257,6 +257,41 @@ def test_layer_8b_q_projection_full_size_sampled():
     assert_close("dB", dB, s * (G.T @ (Xf @ Af.T)))
 
 
+def test_backward_graph_capture_matches_eager():
+    """The backward forks dB/dA onto a second stream and joins it back; captured
+    in a CUDA graph and replayed it gives the eager results bit for bit, and a
+    forward queued right after it on the same stream sees the finished dA/dB."""
+    q = Q()
+    T, N, K, r, s = 512, 1024, 768, 16, 2.0
+    W, X, A, B, dY = inputs.layer_inputs(91, 0, 0, T, N, K, r, device="cuda")
+    qw = q.quantize_nf4(W)
+    ref = q.linear_bwd(dY, X, qw, A, B, s)
+    torch.cuda.synchronize()
+    outs = tuple(torch.empty_like(t) for t in ref)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        q.linear_bwd(dY, X, qw, A, B, s, outs=outs)   # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for t in outs:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        q.linear_bwd(dY, X, qw, A, B, s, outs=outs)
+    g.replay()
+    # the adapter gradients are complete once the stream reaches the next call
+    y_dA = q.linear_fwd(X, qw, outs[1], B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dX", "dA", "dB"), outs, ref):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), name
+    y_ref = q.linear_fwd(X, qw, ref[1], B, s)
+    torch.cuda.synchronize()
+    assert torch.equal(y_dA.view(torch.int16), y_ref.view(torch.int16))
+    del g
+
+
 @pytest.mark.parametrize("name,N,K", [("q", 8192, 8192), ("down", 8192, 22016)])
 def test_layer_65b_shapes_full_size_sampled(name, N, K):
     """A 65B-shaped projection (hidden 8192, ffn 22016; the q/k/v/o and down
