@@ -170,6 +170,24 @@ void snap_thresholds(const float *cb, float *thr) {
   }
 }
 
+// The same decisions without a division: for c1 > 0, RN32(w / c1) >= t_j holds
+// exactly when w / c1 is at least the real midpoint between t_j and the next
+// fp32 value below it (strictly above it when that tie rounds to the lower,
+// odd neighbour).  The midpoint and the tie side per threshold, and the code of 0.
+void snap_boundaries(SnapTable &tab) {
+  tab.incl = 0;
+  tab.snap0 = 0;
+  for (int j = 0; j < 15; ++j) {
+    const float t = tab.thr[j];
+    const float below = nextafterf(t, -INFINITY);
+    tab.mid[j] = (static_cast<double>(t) + static_cast<double>(below)) * 0.5;   // exact in double
+    uint32_t bits;
+    memcpy(&bits, &t, 4);
+    if ((bits & 1u) == 0u) tab.incl |= 1u << j;
+    if (0.0f >= t) ++tab.snap0;
+  }
+}
+
 qlora_status check_weight(const qlora_nf4_weight *qw) {
   if (!qw || !qw->codes || !qw->scales || !qw->c2) return QLORA_ERR_INVALID_ARG;
   if (qw->rows <= 0 || qw->cols <= 0) return QLORA_ERR_INVALID_ARG;
@@ -589,6 +607,7 @@ qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, 
     out->codebook[i] = codebook[i];
   }
   snap_thresholds(codebook, tab.thr);
+  snap_boundaries(tab);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nblocks = rows * cols / 64;
   const double n = static_cast<double>(rows) * cols;

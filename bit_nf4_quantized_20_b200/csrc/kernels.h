@@ -12,6 +12,11 @@ namespace qlora {
 struct SnapTable {
   float codebook[16];
   float thr[15];   // t_j = smallest fp32 >= (q_j + q_{j+1}) / 2
+  // RN32(x) >= t_j  <=>  x >= mid_j (incl bit j set) or x > mid_j (clear), with
+  // mid_j the real midpoint between t_j and the fp32 value below it (ties to even)
+  double mid[15];
+  uint32_t incl;
+  uint32_t snap0;  // the code of w_hat = 0 (all-zero blocks)
 };
 
 // ---------------------------------------------------------------------------

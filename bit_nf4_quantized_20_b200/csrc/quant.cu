@@ -13,6 +13,13 @@
 // weights): 8 lanes share a block, each loading 8 BF16 weights with one
 // 128-bit load; the block absmax is an integer max of |bits| reduced with
 // three xor-shuffles; the group max is a CTA reduction.
+//
+// The code needs no division per weight.  For c1 > 0, RN32(w / c1) >= t_j
+// exactly when w >= mid_j * c1 (or w > mid_j * c1, by the tie rule), where
+// mid_j is the real midpoint between t_j and the fp32 value below it; mid_j
+// has at most 25 significant bits and c1 8, so the product is exact in double.
+// Each block turns its 15 thresholds into the smallest BF16 weights that reach
+// them, B_j, and code = #{ j : w >= B_j } by the same 4-step search.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -23,9 +30,9 @@ namespace {
 
 constexpr int QT = 256;
 
-// Number of thresholds t_j <= x, by a branch-free binary search: the first
-// two levels select between register-held thresholds, the last two read the
-// table in shared memory.
+// Number of boundaries b_j <= x (b non-decreasing), by a branch-free binary
+// search: the first two levels select between register-held boundaries, the
+// last two read the block's table in shared memory.
 __device__ __forceinline__ uint32_t snap_code(float x, float t3, float t7, float t11, const float *s_thr) {
   uint32_t c = (x >= t7) ? 8u : 0u;
   const float th = c ? t11 : t3;
@@ -35,13 +42,28 @@ __device__ __forceinline__ uint32_t snap_code(float x, float t3, float t7, float
   return c;
 }
 
+// The smallest BF16 value w with w >= mid * c1 (incl) or w > mid * c1 (not
+// incl), for c1 > 0; +Inf when no finite BF16 value qualifies.
+__device__ __forceinline__ float snap_boundary(float c1, double mid, bool incl) {
+  const double P = mid * static_cast<double>(c1);   // exact
+  const float f = __double2float_ru(P);             // the smallest fp32 >= P
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0xFFFFu) != 0u) u = (f > 0.f) ? ((u + 0x10000u) & 0xFFFF0000u) : (u & 0xFFFF0000u);
+  float b = __uint_as_float(u);                     // the smallest BF16 >= f, hence >= P
+  if (!incl && static_cast<double>(b) == P) {       // strictly above P: the next BF16 up
+    if ((u & 0x7FFFFFFFu) == 0u) u = 0x00010000u;
+    else u = (b > 0.f) ? u + 0x10000u : u - 0x10000u;
+    b = __uint_as_float(u);
+  }
+  return b;
+}
+
 __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ w, int64_t n_blocks,
                                                       uint32_t *__restrict__ codes, uint8_t *__restrict__ scales,
                                                       float *__restrict__ c2, const SnapTable tab,
                                                       uint32_t *status) {
-  __shared__ float s_thr[16];
+  __shared__ float s_bnd[256 * 16];   // per block of the group: B_0 .. B_14
   __shared__ float s_wmax[QT / 32];
-  if (threadIdx.x < 15) s_thr[threadIdx.x] = tab.thr[threadIdx.x];
 
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * 256;
@@ -89,20 +111,37 @@ __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ 
   const float c2v = __fdiv_rn(gmax, 448.0f);
   if (tid == 0) c2[g] = c2v;
 
-  const float t3 = s_thr[3], t7 = s_thr[7], t11 = s_thr[11];
+  // the block's boundaries: lane `sub` of its 8 lanes forms B_sub and B_{sub + 8}
+  // (an all-zero block gets boundaries that give every weight the code of 0)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bl = i * 32 + bw;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = sub + 8 * h;
+      if (j < 15) {
+        float bj;
+        if (c1[i] > 0.f) bj = snap_boundary(c1[i], tab.mid[j], ((tab.incl >> j) & 1u) != 0u);
+        else bj = j < static_cast<int>(tab.snap0) ? -INFINITY : INFINITY;
+        s_bnd[bl * 16 + j] = bj;
+      }
+    }
+  }
+  __syncwarp();   // a block's 8 lanes are in one warp
+
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int bl = i * 32 + bw;
     if (bl < nb) {
       if (sub == 0) scales[b0 + bl] = static_cast<uint8_t>(c2v > 0.f ? float_to_e4m3(__fdiv_rn(c1[i], c2v)) : 0u);
       const uint32_t hw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      const float *bnd = s_bnd + bl * 16;
+      const float b3 = bnd[3], b7 = bnd[7], b11 = bnd[11];
       uint32_t word = 0;
-      const bool nz = c1[i] > 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const uint32_t bits = (e & 1) ? (hw[e >> 1] & 0xFFFF0000u) : (hw[e >> 1] << 16);
-        const float x = nz ? __fdiv_rn(__uint_as_float(bits), c1[i]) : 0.f;
-        word |= snap_code(x, t3, t7, t11, s_thr) << (4 * e);
+        word |= snap_code(__uint_as_float(bits), b3, b7, b11, bnd) << (4 * e);
       }
       codes[(b0 + bl) * 8 + sub] = word;
     }
