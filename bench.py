@@ -12,7 +12,8 @@ distributions) and resident in HBM; the step's working set (~0.8 GB) is far
 larger than the 126 MB L2, so no flush is needed between steps.
 
 The JSON line also carries: `e2e` (same metric with the step's X and dY copied
-from pinned host memory and dA, dB read back, inside the timed region),
+from pinned host memory and dA, dB read back, inside the timed region; the
+copies run on two copy streams that overlap the projections' compute),
 `roofline` of the dominant kernel (CUDA-event durations of every launch in the
 timed region, through the library's trace hook), `cpu_baseline` (the CPU
 oracle timed on a bounded token sample), `clocks` sampled with nvidia-smi
@@ -300,14 +301,38 @@ def bench_e2e(args, layers, dev, s, world, dist):
     h2d = sum(h[0].numel() * 2 + h[1].numel() * 2 for h in host)
     d2h = sum(h[2].numel() * 2 + h[3].numel() * 2 for h in host)
 
+    # The copies run on their own streams so that they overlap the projections'
+    # compute: the inputs of projection p+1 cross PCIe while p computes, and dA,
+    # dB go back on a second copy stream.  Every copy of the step is still
+    # inside the timed region: both copy streams join the compute stream at the
+    # end of the step, and a projection's buffers are refilled for the next
+    # step only after that projection's compute has consumed them.
+    compute = torch.cuda.current_stream(dev)
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = len(layers)
+    ev_in = [torch.cuda.Event() for _ in range(n)]     # inputs of p landed
+    ev_done = [torch.cuda.Event() for _ in range(n)]   # p's compute finished
+    for e in ev_done:
+        e.record(compute)
+
     def e2e_step():
-        for L, (hx, hdy, hda, hdb) in zip(layers, host):
-            L["X"].copy_(hx, non_blocking=True)
-            L["dY"].copy_(hdy, non_blocking=True)
+        with torch.cuda.stream(h2d_s):
+            for i, (L, (hx, hdy, _, _)) in enumerate(zip(layers, host)):
+                h2d_s.wait_event(ev_done[i])
+                L["X"].copy_(hx, non_blocking=True)
+                L["dY"].copy_(hdy, non_blocking=True)
+                ev_in[i].record(h2d_s)
+        for i, (L, (_, _, hda, hdb)) in enumerate(zip(layers, host)):
+            compute.wait_event(ev_in[i])
             q.linear_fwd(L["X"], L["qw"], L["A"], L["B"], s, out=L["Y"])
             q.linear_bwd(L["dY"], L["X"], L["qw"], L["A"], L["B"], s, outs=(L["dX"], L["dA"], L["dB"]))
-            hda.copy_(L["dA"], non_blocking=True)
-            hdb.copy_(L["dB"], non_blocking=True)
+            ev_done[i].record(compute)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[i])
+                hda.copy_(L["dA"], non_blocking=True)
+                hdb.copy_(L["dB"], non_blocking=True)
+        compute.wait_stream(h2d_s)
+        compute.wait_stream(d2h_s)
 
     steps = max(1, min(args.steps, 5))
     for _ in range(2):
@@ -317,6 +342,7 @@ def bench_e2e(args, layers, dev, s, world, dist):
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
+    h2d_s.wait_stream(compute)   # no copy of the timed steps starts before `a`
     for _ in range(steps):
         e2e_step()
     b.record()
