@@ -319,6 +319,15 @@ def linear_bwd(dy_bits, x_bits, w_deq_bits, a_bits, b_bits, s):
 # Llama 3.1 8B worked example; "QLoRA: Efficient Fine-Tuning", eq. 4).
 # ----------------------------------------------------------------------------
 
+def merge_adapter(w_deq_bits, a_bits, b_bits, s):
+    """The merged weight of "QLoRA: Efficient Fine-Tuning" Step 3 (h = W0 x + s B A x
+    as one matrix): W'[N, K] + s B[N, r] A[r, K], in float64 from the BF16 dequantized
+    weight and adapter.  Export rounds it to BF16 (and may quantize it again)."""
+    w = _f64(w_deq_bits)
+    a, b = _f64(a_bits), _f64(b_bits)
+    return w + float(s) * (b @ a)
+
+
 def storage_bytes(rows: int, cols: int, blocksize: int = BLOCKSIZE, dq_block: int = DQ_BLOCK):
     """(codes, scale bytes, c2 bytes) for one quantized weight."""
     n = rows * cols

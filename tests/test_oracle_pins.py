@@ -352,6 +352,21 @@ def test_forward_merged_weight_identity():
     assert np.allclose(O.linear_fwd(X, W, A, zero, s), O.linear_fwd(X, W, A, B, 0.0), rtol=0, atol=1e-14)
 
 
+def test_merge_adapter_elementwise_and_forward_identity():
+    """merge_adapter = W' + s B A: element by element as an explicit sum over the
+    rank, and X merged^T equals eq. 3's forward (the point of merging)."""
+    T, m, n, r, s = 3, 5, 64, 3, 0.75
+    X, W, A, B = _bits((T, n), 1, 15), _bits((m, n), 0.02, 16), _bits((r, n), 0.1, 17), _bits((m, r), 0.05, 18)
+    M = O.merge_adapter(W, A, B, s)
+    w, a, b = (O.bf16_bits_to_f32(v).astype(F64) for v in (W, A, B))
+    for i in range(m):
+        for k in range(n):
+            ref = w[i, k] + s * sum(b[i, j] * a[j, k] for j in range(r))
+            assert abs(M[i, k] - ref) <= 1e-15 * max(1.0, abs(ref))
+    assert np.allclose(O.bf16_bits_to_f32(X).astype(F64) @ M.T, O.linear_fwd(X, W, A, B, s), rtol=1e-12, atol=1e-12)
+    assert np.array_equal(O.merge_adapter(W, A, B, 0.0), w)
+
+
 def test_backward_eq5_per_token_outer_products():
     """eq. 5: dL/dA = B^T g x^T and dL/dB = g (A x)^T per token (times s), summed."""
     T, m, n, r, s = 3, 5, 7, 2, 0.5
