@@ -441,13 +441,16 @@ def bench_secondary(dev, peaks):
                                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                "bytes_per_sweep": int(nbytes), "timing": "CUDA graph of the 7-projection sweep, "
                                "L2 flushed (256 MB read) before each replay, median of 10"}
-    # quantize / dequantize of one gate-shaped weight (58.7 M weights)
+    # quantize / dequantize / rank-16 adapter merge of one gate-shaped weight (58.7 M weights)
     N, K = 14336, 4096
     W = inputs.normal_bf16((N, K), 0.02, 7, dev)
     qw = q.quantize_nf4(W)
     wd = torch.empty_like(W)
     per = 2.0 + 0.5 + 1 / 64
-    for name, fn in (("quantize", lambda: q.quantize_nf4(W)), ("dequantize", lambda: q.dequantize(qw))):
+    A = inputs.normal_bf16((16, K), (1.0 / K) ** 0.5, 8, dev)
+    B = inputs.normal_bf16((N, 16), 0.01, 9, dev)
+    for name, fn in (("quantize", lambda: q.quantize_nf4(W)), ("dequantize", lambda: q.dequantize(qw)),
+                     ("merge_adapter", lambda: q.merge_adapter(qw, A, B, 2.0))):
         times = []
         for rep in range(6):
             flush_l2()

@@ -133,6 +133,24 @@ def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: 
     return QuantizedNF4(codes, scales, c2, rows, cols, cb, blocksize, dq_block)
 
 
+def merge_adapter(qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float) -> torch.Tensor:
+    """BF16(W' + s B A) [rows, cols]: the adapter folded into the dequantized
+    weight for export (quantize_nf4 of the result gives an NF4 merged model)."""
+    for name, t in (("A", A), ("B", B)):
+        _need_cuda(name, t)
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor")
+    r = A.shape[0]
+    if A.dim() != 2 or A.shape[1] != qw.cols or tuple(B.shape) != (qw.rows, r):
+        raise ValueError(f"A must be [r, {qw.cols}] and B [{qw.rows}, r]")
+    out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.device)
+    st = qw.struct()
+    check("qlora_merge_adapter", lib().qlora_merge_adapter(C.byref(st), C.c_void_p(A.data_ptr()),
+                                                           C.c_void_p(B.data_ptr()), r, float(s),
+                                                           C.c_void_p(out.data_ptr()), _stream(qw.device)))
+    return out
+
+
 def dequantize(qw: QuantizedNF4) -> torch.Tensor:
     out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.device)
     s = qw.struct()

@@ -48,6 +48,8 @@ SIGNATURES = {
                                      C.POINTER(C.c_float), C.POINTER(NF4Weight), C.c_void_p, C.c_size_t,
                                      C.c_void_p]),
     "qlora_dequantize": (C.c_int, [C.POINTER(NF4Weight), C.c_void_p, C.c_void_p]),
+    "qlora_merge_adapter": (C.c_int, [C.POINTER(NF4Weight), C.c_void_p, C.c_void_p, C.c_int32, C.c_float,
+                                      C.c_void_p, C.c_void_p]),
     "qlora_linear_fwd": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
                                    C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "qlora_linear_bwd": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p,

@@ -38,12 +38,13 @@ enum KernelId : int32_t {
   K_GEMV_FWD = 8,
   K_LORA_U_DU = 9,      // U and dU in one grid (backward)
   K_LORA_DB_DA = 10,    // dB and dA in one grid (backward)
-  K_COUNT = 11,
+  K_MERGE = 11,         // adapter merge for export
+  K_COUNT = 12,
 };
 
 const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",       "lora_du",
                                      "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx",
-                                     "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA"};
+                                     "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA",   "merge_adapter"};
 
 struct TraceScope {
   cudaStream_t st;
@@ -627,6 +628,22 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *qw, void *w_bf16_out, void
   TraceScope ts(K_DEQUANTIZE, 0.0, n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + n * 2.0, st);
   cudaError_t e = launch_dequantize(qw->codes, qw->scales, qw->c2, qw->rows * qw->cols, qw->codebook,
                                     static_cast<uint16_t *>(w_bf16_out), st, num_sms_current());
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_merge_adapter(const qlora_nf4_weight *qw, const void *A, const void *B, int32_t r, float s,
+                                 void *w_out, void *stream) {
+  qlora_status cs = check_weight(qw);
+  if (cs != QLORA_OK) return cs;
+  if (!A || !B || !w_out || r < 1 || r > 128 || !isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(w_out) || (reinterpret_cast<uintptr_t>(B) & 1u)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const double n = static_cast<double>(qw->rows) * qw->cols;
+  TraceScope ts(K_MERGE, 2.0 * n * r,
+                n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * r * (qw->rows + qw->cols) + 2.0 * n, st);
+  cudaError_t e = launch_merge(qw->codes, qw->scales, qw->c2, qw->rows, qw->cols, qw->codebook,
+                               static_cast<const uint16_t *>(A), static_cast<const uint16_t *>(B), r, s,
+                               static_cast<uint16_t *>(w_out), st, num_sms_current());
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

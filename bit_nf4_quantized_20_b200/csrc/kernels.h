@@ -22,6 +22,10 @@ struct SnapTable {
 // ---------------------------------------------------------------------------
 // quantize / dequantize (quant.cu)
 // ---------------------------------------------------------------------------
+// out[N, K] = BF16(W' + s B A) (quant.cu)
+cudaError_t launch_merge(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t N, int64_t K,
+                         const float (&codebook)[16], const uint16_t *A, const uint16_t *B, int r, float s,
+                         uint16_t *out, cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
                             const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t n_weights,

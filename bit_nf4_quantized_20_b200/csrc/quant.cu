@@ -176,7 +176,74 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint2 *__restrict__ 
   }
 }
 
+// Adapter merge for export ("QLoRA: Efficient Fine-Tuning", Step 3: eq. 3's two
+// terms as one matrix W0 + s B A):
+//   out[n, k] = BF16_RNE(fma(s, d, W'[n, k])),   d = sum_j B[n, j] A[j, k] in fp32,
+// with W' formed exactly as dequant_kernel forms it (so the frozen part is the
+// BF16 dequantized weight) and j ascending.  One thread per 16 consecutive
+// weights of a row (a unit never crosses a row: K % 64 == 0).
+__global__ void __launch_bounds__(256) merge_kernel(const uint2 *__restrict__ codes,
+                                                    const uint8_t *__restrict__ scales,
+                                                    const float *__restrict__ c2, int64_t n_units, int64_t K,
+                                                    const SnapTable tab, const uint16_t *__restrict__ A,
+                                                    const uint16_t *__restrict__ B, int r, float s,
+                                                    uint4 *__restrict__ out) {
+  __shared__ float s_cb[16];
+  if (threadIdx.x < 16) s_cb[threadIdx.x] = tab.codebook[threadIdx.x];
+  __syncthreads();
+  const int64_t units_per_row = K / 16;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_units; i += stride) {
+    const int64_t n = i / units_per_row, k0 = (i - n * units_per_row) * 16;
+    const uint2 c = __ldg(codes + i);       // 16 codes
+    const int64_t blk = i >> 2;             // 4 units of 16 weights per block
+    const float sc = __fmul_rn(e4m3_to_float(__ldg(scales + blk)), __ldg(c2 + (blk >> 8)));
+    float w[16], d[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t word = e < 8 ? c.x : c.y;
+      const float q = s_cb[(word >> (4 * (e & 7))) & 15u];
+      w[e] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(q, sc)));
+      d[e] = 0.f;
+    }
+    const uint16_t *brow = B + n * r;
+    for (int j = 0; j < r; ++j) {
+      const float b = __uint_as_float(static_cast<uint32_t>(__ldg(brow + j)) << 16);
+      const uint4 *ap = reinterpret_cast<const uint4 *>(A + static_cast<int64_t>(j) * K + k0);
+      const uint4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+      const uint32_t aw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint32_t bits = (e & 1) ? (aw[e >> 1] & 0xFFFF0000u) : (aw[e >> 1] << 16);
+        d[e] = fmaf(b, __uint_as_float(bits), d[e]);
+      }
+    }
+    uint32_t o[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) o[p] = pack_bf16x2(fmaf(s, d[2 * p], w[2 * p]), fmaf(s, d[2 * p + 1], w[2 * p + 1]));
+    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_merge(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t N, int64_t K,
+                         const float (&codebook)[16], const uint16_t *A, const uint16_t *B, int r, float s,
+                         uint16_t *out, cudaStream_t st, int num_sms) {
+  const int64_t n_units = N * K / 16;
+  if (n_units <= 0) return cudaSuccess;
+  SnapTable tab;
+  for (int i = 0; i < 16; ++i) tab.codebook[i] = codebook[i];
+  for (int i = 0; i < 15; ++i) tab.thr[i] = 0.f;
+  int64_t blocks = (n_units + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(reinterpret_cast<const uint2 *>(codes), scales, c2,
+                                                               n_units, K, tab, A, B, r, s,
+                                                               reinterpret_cast<uint4 *>(out));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
                             const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms) {

@@ -158,6 +158,19 @@ QLORA_API qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int6
 QLORA_API qlora_status qlora_dequantize(const qlora_nf4_weight *qw, void *w_bf16_out, void *stream);
 
 /*
+ * Adapter merge for export ("QLoRA: Efficient Fine-Tuning", Step 3: eq. 3's
+ * two terms as one matrix):
+ *   w_out[n, k] = BF16_RNE(fma(s, d, W'[n, k])),  d = sum_j B[n, j] A[j, k] in
+ *   FP32 (j ascending), W' the BF16 dequantized weight.
+ * A[r, K] (16-byte aligned), B[N, r] (2-byte aligned): BF16, row-major;
+ * w_out[N, K]: BF16, 16-byte aligned, overwritten.  1 <= r <= 128.  The result
+ * can be quantized again with qlora_quantize_nf4.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+QLORA_API qlora_status qlora_merge_adapter(const qlora_nf4_weight *qw, const void *A, const void *B, int32_t r,
+                                           float s, void *w_out, void *stream);
+
+/*
  * Forward, eq. 3 with the PEFT scaling (Step 3):
  *   y[T, N] = x[T, K] W'^T + s (x A^T) B^T, BF16 out, FP32 accumulation,
  *   W' dequantized inside the matmul and never written to memory.

@@ -126,6 +126,35 @@ def test_code_function_sweep_over_bf16_pairs():
     assert np.array_equal(qw.codes.cpu().numpy(), codes)
 
 
+@pytest.mark.parametrize("N,K,r,s,a_std,b_std", [
+    (512, 512, 8, 2.0, 0.1, 0.05),          # adapter term comparable to W'
+    (1032, 768, 64, 0.25, 0.1, 0.05),       # ragged rows, large rank
+    (4096, 4096, 16, 2.0, None, 0.01),      # 8B q shape, trained-adapter scale
+])
+def test_merge_adapter(N, K, r, s, a_std, b_std):
+    """BF16(W' + s B A) on the GPU against the oracle's float64 merge.  The GPU
+    forms d = sum_j B A in FP32 and fma(s, d, W') before rounding to BF16, so
+    an element may differ from the oracle's value by one BF16 step (2^-7 |o|)
+    plus the FP32 error of that arithmetic, 2^-24 (r + 2) (|W'| + s sum_j |B||A|)
+    (which only matters where W' and s B A cancel)."""
+    q = Q()
+    W, _, A, B, _ = inputs.layer_inputs(95, 0, 0, 1, N, K, r, device="cuda", a_std=a_std, b_std=b_std)
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    m = q.merge_adapter(qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    o = O.merge_adapter(wd, bits(A), bits(B), s)
+    af, bf, wf = (O.bf16_bits_to_f32(v).astype(np.float64) for v in (bits(A), bits(B), wd))
+    bound = 2.0 ** -7 * np.abs(o) + 2.0 ** -24 * (r + 2) * (np.abs(wf) + abs(s) * (np.abs(bf) @ np.abs(af)))
+    g = bits(m).astype(np.uint32) << np.uint32(16)
+    err = np.abs(g.view(np.float32).astype(np.float64) - o)
+    bad = err > bound
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} elements outside the bound; worst {np.max(err - bound)!r}"
+    # the adapter really moved the weight (the term is not lost in rounding)
+    assert (g != (wd.astype(np.uint32) << np.uint32(16))).mean() > 0.01
+
+
 def test_nonfinite_weight_is_reported():
     q = Q()
     w = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
