@@ -14,18 +14,23 @@
 // codes a lane feeds one MMA per row are four consecutive codes of its block,
 // and its X fragments are eight consecutive bytes of one token row.
 //
-// Weight stream: every lane copies its own blocks (32 code bytes, the aligned
-// word holding its scale byte, and its c2) with cp.async into a private ring
-// of GD items in shared memory, so each warp keeps GD - 1 items in flight with
-// no register cost and no cross-lane synchronisation.
+// Two kernels share that per-lane work and differ in how they spread it:
 //
-// Work split: a CTA is one 16-row tile; its S warps split the k-units, and
-// their accumulators are added in warp order through shared memory by warp 0,
-// which adds the rank-r term B U'^T as extra MMA k-steps and writes BF16 Y.  S
-// is the largest split count whose grid of N/16 CTAs is resident in one wave.
-// Launched with programmatic dependent launch: the first GD - 1 units of the
-// weight stream are requested while the preceding kernel (the one computing
-// U') still runs; X, U' and Y are touched only after griddepcontrol.wait.
+// nf4_gemv_kernel (any K that is a multiple of 64): every lane copies its own
+// blocks (32 code bytes, the aligned word holding its scale byte, and its c2)
+// with cp.async into a private ring of GD items in shared memory.  A CTA is
+// one 16-row tile; its S warps split the k-units, and their accumulators are
+// added in warp order through shared memory by warp 0, which adds the rank-r
+// term B U'^T as extra MMA k-steps and writes BF16 Y.  S is the largest split
+// count whose grid of N/16 CTAs is resident in one wave.
+//
+// nf4_gemv_persist_kernel (K a multiple of 256, the default): persistent
+// stream-K over all 16 x 256 units, described where it is defined.
+//
+// Both are launched with programmatic dependent launch: the first units of
+// the weight stream are requested while the preceding kernel (the one
+// computing U') still runs; X, U' and Y are touched only after
+// griddepcontrol.wait.
 //
 // lora_u_decode_kernel computes U' itself for these token counts: a cluster of
 // 8 CTAs per 16 columns of U' splits K, each CTA requests its whole slice of A
