@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 
 from oracle import oracle as O
+from bit_nf4_quantized_20_b200 import inputs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "qlora.h")
@@ -91,6 +92,19 @@ def test_workspace_bytes(L):
     assert L.qlora_workspace_bytes(2, 0, 4096, 4096, 16) > 0
     # grows with the token count
     assert L.qlora_workspace_bytes(2, 8192, 4096, 4096, 16) > b
+
+
+def test_decode_workspace_fits_the_noalloc_scratch(L):
+    """The allocation-free forward keeps its scratch in a fixed 4 MiB array; the
+    decode shapes (1-16 tokens, rank up to 128) of the 8B and 65B projections
+    must fit in it, split partials of the persistent GEMV included."""
+    scratch = 4 << 20
+    shapes = [(n, k) for (_, n, k) in inputs.LLAMA8B_PROJ] + [(8192, 8192), (22016, 8192), (8192, 22016)]
+    for (n, k) in shapes:
+        for T in (1, 4, 16):
+            for r in (16, 64, 128):
+                need = L.qlora_workspace_bytes(1, T, n, k, r)
+                assert 0 < need <= scratch, (T, n, k, r, need)
 
 
 def _weight(rows=128, cols=128, codes=0x1000, scales=0x2000, c2=0x3000, bs=64, dq=256):
