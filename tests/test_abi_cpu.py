@@ -169,6 +169,24 @@ def test_linear_validation(L):
     assert deq(C.byref(w), C.c_void_p(FAKE + 1), None) == 3
 
 
+def test_merge_validation(L):
+    """qlora_merge_adapter rejects bad arguments before touching the GPU."""
+    w = _weight()
+    P = C.c_void_p(FAKE)
+    merge = L.qlora_merge_adapter
+    assert merge(None, P, P, 8, 2.0, P, None) == 1
+    assert merge(C.byref(w), None, P, 8, 2.0, P, None) == 1
+    assert merge(C.byref(w), P, None, 8, 2.0, P, None) == 1
+    assert merge(C.byref(w), P, P, 8, 2.0, None, None) == 1
+    assert merge(C.byref(w), P, P, 0, 2.0, P, None) == 1            # r = 0
+    assert merge(C.byref(w), P, P, 129, 2.0, P, None) == 1          # r > 128
+    assert merge(C.byref(w), P, P, 8, float("nan"), P, None) == 1
+    assert merge(C.byref(w), C.c_void_p(FAKE + 8), P, 8, 2.0, P, None) == 3   # A not 16-byte aligned
+    assert merge(C.byref(w), P, C.c_void_p(FAKE + 1), 8, 2.0, P, None) == 3   # B not 2-byte aligned
+    assert merge(C.byref(w), P, P, 8, 2.0, C.c_void_p(FAKE + 4), None) == 3   # output not 16-byte aligned
+    assert merge(C.byref(_weight(bs=128)), P, P, 8, 2.0, P, None) == 2
+
+
 def test_linear_fwd_zero_tokens_is_a_noop(L):
     """T == 0 launches nothing; the empty token buffers may be null."""
     w = _weight()
