@@ -157,6 +157,20 @@ def nf4_codebook() -> np.ndarray:
     return np.concatenate([-pos[::-1], pos]).astype(F32)
 
 
+def nf4_codebook_with_zero() -> np.ndarray:
+    """READING: a variant of eq. 2 with an exact zero level.
+
+    eq. 2 places no level at zero ("QLoRA: Efficient Fine-Tuning", Step 1), so
+    a zero weight dequantizes to +-0.042 s.  The plainest table that keeps
+    eq. 2's spacing and represents zero exactly replaces the negative level
+    nearest zero, q_8, with 0: seven negative levels, zero, eight positive
+    levels, all other entries equal to nf4_codebook()'s.  Ascending.
+    """
+    q = nf4_codebook().copy()
+    q[7] = F32(0.0)
+    return q
+
+
 def snap_thresholds(codebook: np.ndarray) -> np.ndarray:
     """READING of "snapped to the nearest NF4 quantile level".
 
@@ -242,20 +256,25 @@ def double_quantize(c1: np.ndarray, dq_block: int = DQ_BLOCK):
 
 
 def quantize_nf4(w_bits: np.ndarray, codebook: np.ndarray | None = None,
-                 blocksize: int = BLOCKSIZE, dq_block: int = DQ_BLOCK):
+                 blocksize: int = BLOCKSIZE, dq_block: int = DQ_BLOCK, snap_to_dq_scale: bool = False):
     """Quantize a BF16 weight W[rows, cols] (given as uint16 bit patterns).
 
     Returns (codes uint8[rows*cols/2], scales uint8[rows*cols/64], c2 fp32[...]).
-    Codes are snapped against the exact fp32 c1 (quantize first, then double-
-    quantize the scales, in the order the prepfeed page describes them).
+    By default codes are snapped against the exact fp32 c1 (quantize first,
+    then double-quantize the scales, in the order the prepfeed page describes
+    them).  READING, variant: with snap_to_dq_scale the scales are
+    double-quantized first and each block is normalised by the scale it will
+    be dequantized with, s_b = RN32(fp8(f_b) * c2) (w_hat = 0 where s_b = 0),
+    so that each code is the level nearest w / s_b.
     """
     if codebook is None:
         codebook = nf4_codebook()
     w_bits = np.asarray(w_bits, dtype=np.uint16)
     assert w_bits.ndim == 2 and w_bits.shape[1] % blocksize == 0
     c1 = block_absmax(w_bits, blocksize)
-    codes = snap(normalise(w_bits, c1, blocksize), codebook)
     scales, c2 = double_quantize(c1, dq_block)
+    divisor = block_scales(scales, c2, dq_block) if snap_to_dq_scale else c1
+    codes = snap(normalise(w_bits, divisor, blocksize), codebook)
     return pack_codes(codes), scales, c2
 
 
@@ -298,19 +317,34 @@ def linear_fwd(x_bits, w_deq_bits, a_bits, b_bits, s):
     return X @ W.T + float(s) * (U @ B.T)
 
 
+def lora_adapter_grads(dy_bits, x_bits, a_bits, b_bits, s):
+    """eq. 5 ("QLoRA: Efficient Fine-Tuning", Step 4) with the PEFT scaling,
+    in float64: dU = s dY B; dB = s dY^T (X A^T); dA = dU^T X.
+
+    Only the adapter gradients (they sum over every token; the gradient
+    through the frozen weight is per token and lives in linear_bwd).
+    Returns (dA[r, K], dB[N, r]).
+    """
+    dY, X, A, B = _f64(dy_bits), _f64(x_bits), _f64(a_bits), _f64(b_bits)
+    s = float(s)
+    U = X @ A.T
+    dU = s * (dY @ B)
+    dB = s * (dY.T @ U)
+    dA = dU.T @ X
+    return dA, dB
+
+
 def linear_bwd(dy_bits, x_bits, w_deq_bits, a_bits, b_bits, s):
     """eq. 5 plus the gradient through the frozen weight, in float64.
 
     dU = s dY B; dX = dY W' + dU A; dB = s dY^T (X A^T); dA = dU^T X.
-    Returns (dX[T, K], dA[r, K], dB[N, r]).
+    Returns (dX[T, K], dA[r, K], dB[N, r]).  Row t of dX depends only on row t
+    of dY, so dX of a subset of tokens is linear_bwd of those tokens' rows.
     """
-    dY, X, W, A, B = _f64(dy_bits), _f64(x_bits), _f64(w_deq_bits), _f64(a_bits), _f64(b_bits)
-    s = float(s)
-    U = X @ A.T
-    dU = s * (dY @ B)
+    dY, W, A, B = _f64(dy_bits), _f64(w_deq_bits), _f64(a_bits), _f64(b_bits)
+    dU = float(s) * (dY @ B)
     dX = dY @ W + dU @ A
-    dB = s * (dY.T @ U)
-    dA = dU.T @ X
+    dA, dB = lora_adapter_grads(dy_bits, x_bits, a_bits, b_bits, s)
     return dX, dA, dB
 
 
@@ -354,3 +388,36 @@ def lora_fraction(m: int, n: int, r: int) -> float:
 def normal_cdf(x: float) -> float:
     """Phi(x) = (1 + erf(x / sqrt 2)) / 2 -- used only to check eq. 2's spacing."""
     return 0.5 * (1.0 + math.erf(x / math.sqrt(2.0)))
+
+
+# ----------------------------------------------------------------------------
+# The adapters' optimizer step ("What is QLoRA?", "The three pieces": paged
+# optimizers keep the optimizer state in unified memory; "Worked example":
+# adapters in fp32 with gradients and Adam moments, 16 bytes each).
+# ----------------------------------------------------------------------------
+
+def adam_step(param, m, v, grad, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+              eps: float = 1e-8, weight_decay: float = 0.0):
+    """One Adam step (Kingma & Ba, 2015, Algorithm 1) with decoupled weight
+    decay (Loshchilov & Hutter, 2019), in float64:
+
+        param <- param (1 - lr wd)
+        m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2
+        param <- param - lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+
+    READING: the pages name Adam and its fp32 moments but no formula or
+    hyper-parameters; this is the published algorithm as written.  step counts
+    from 1.  grad is given as BF16 bits (the layer's dA / dB); param, m, v as
+    float arrays.  Returns (param, m, v) as new float64 arrays.
+    """
+    p = np.asarray(param, F64)
+    m = np.asarray(m, F64)
+    v = np.asarray(v, F64)
+    g = bf16_bits_to_f32(grad).astype(F64).reshape(p.shape)
+    p = p * (1.0 - lr * weight_decay)
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** step)
+    v_hat = v / (1.0 - beta2 ** step)
+    p = p - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return p, m, v

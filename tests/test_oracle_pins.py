@@ -444,3 +444,164 @@ def test_backward_is_the_derivative_of_the_forward(which):
         fd = (L(Xf, Af, Bf + e * D) - L(Xf, Af, Bf - e * D)) / (2 * e)
         an = float(np.sum(dB * D))
     assert abs(fd - an) <= 1e-8 * (1 + abs(an))
+
+
+# --------------------------------------------------------------------------
+# codebook variants ("QLoRA & 4-bit Fine-Tuning", Innovation 1 and 2)
+# --------------------------------------------------------------------------
+
+def test_codebook_with_zero_level():
+    """eq. 2 with its negative level nearest zero replaced by an exact 0: still
+    ascending, ends at -1 and +1, zero present, the other 15 entries eq. 2's."""
+    z = O.nf4_codebook_with_zero()
+    q = O.nf4_codebook()
+    assert z.dtype == F32 and z.shape == (16,)
+    assert np.all(np.diff(z.astype(F64)) > 0)
+    assert z[7] == 0.0 and not np.signbit(z[7])
+    keep = np.arange(16) != 7
+    assert np.array_equal(z[keep].view(np.uint32), q[keep].view(np.uint32))
+    assert z[0] == -1.0 and z[15] == 1.0
+    # a zero weight in a non-zero block now dequantizes to exactly zero
+    w = np.zeros((1, 64), np.uint16)
+    w[0, 3] = 0x3C00                                   # one non-zero weight (2^-7)
+    codes, scales, c2 = O.quantize_nf4(w, z)
+    wd = O.dequantize_nf4(codes, scales, c2, 1, 64, z)
+    assert np.all(wd[0, np.arange(64) != 3] == 0) and wd[0, 3] == 0x3C00
+
+
+def _scale_of_bytes(scales, c2, dq=256):
+    """s_b = RN32(fp8 * c2) with the FP8 bytes decoded by ml_dtypes."""
+    f = np.asarray(scales, np.uint8).view(ml_dtypes.float8_e4m3fn).astype(F32)
+    return (f * np.asarray(c2, F32)[np.arange(f.size) // dq]).astype(F32)
+
+
+def test_dq_scale_snapping_is_nearest_level_of_w_over_sb():
+    """The variant that snaps against the double-quantized scale: each code is
+    the level nearest RN32(w / s_b) (exact rational brute force, ties up), with
+    s_b decoded independently; the scale bytes and c2 are the default's."""
+    w = _w(4, 256, 19)
+    for cb in (O.nf4_codebook(), O.nf4_codebook_with_zero()):
+        codes, scales, c2 = O.quantize_nf4(w, cb, snap_to_dq_scale=True)
+        codes0, scales0, c20 = O.quantize_nf4(w, cb)
+        assert np.array_equal(scales, scales0) and np.array_equal(c2.view(np.uint32), c20.view(np.uint32))
+        sb = _scale_of_bytes(scales, c2)
+        c = O.unpack_codes(codes).reshape(-1, 64)
+        wf = O.bf16_bits_to_f32(w).reshape(-1, 64)
+        for b in range(wf.shape[0]):
+            for i in range(64):
+                v = F32(wf[b, i] / sb[b]) if sb[b] > 0 else F32(0.0)
+                assert c[b, i] == _brute_nearest(v, cb)
+
+
+def test_dq_scale_snapping_worked_example():
+    """A group whose largest scale is 1.0 (c2 = RN32(1/448)) and a block with
+    c1 = 0.9: 0.9 / c2 = 403.2 lies between the E4M3 values 384 and 416 and
+    rounds to 416, so that block is dequantized with s_b = RN32(416 c2) =
+    0.92857.. > c1.  A weight just above 0.9 t_14 (the threshold to the top
+    level) snaps to level 15 against c1 but to level 14 against s_b."""
+    q = O.nf4_codebook()
+    t14 = float(O.snap_thresholds(q)[14])
+    c2 = F32(F32(1.0) / F32(448.0))
+    sb = F32(F32(416.0) * c2)
+    w = np.zeros((1, 128), np.float32)
+    w[0, 0] = 1.0                                     # block 0: c1 = 1.0, the group max
+    w[0, 64] = 0.9                                    # block 1: c1 = 0.9 (BF16 0.8984375)
+    c1 = float(ml_dtypes.bfloat16(0.9))
+    # the smallest BF16 value above c1 * t14: reaches t14 against c1 ...
+    x = ml_dtypes.bfloat16(c1 * t14)
+    while float(x) < c1 * t14:
+        x = np.nextafter(x, ml_dtypes.bfloat16(1.0))
+    w[0, 65] = float(x)
+    wb = w.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert float(x) / c1 >= t14 and float(x) / float(sb) < t14   # ... but not against s_b
+    codes0, scales, c2g = O.quantize_nf4(wb, q)
+    codes1, _, _ = O.quantize_nf4(wb, q, snap_to_dq_scale=True)
+    assert c2g[0] == c2 and scales[1] == 0x7D                     # E4M3 0x7D = 1.625 * 2^8 = 416
+    assert O.unpack_codes(codes0)[65] == 15 and O.unpack_codes(codes1)[65] == 14
+    assert O.unpack_codes(codes0)[0] == O.unpack_codes(codes1)[0] == 15
+
+
+def test_dq_scale_snapping_equals_default_when_scales_are_exact():
+    """When every c1 is exactly an E4M3 multiple of c2 (here: powers of two
+    with the group max 448 * 2^-12, so c2 = 2^-12), s_b == c1 and the variant
+    gives the default's codes bit for bit."""
+    rng = np.random.default_rng(5)
+    w = rng.normal(0, 1, (4, 64 * 64)).astype(np.float32).reshape(-1, 64)
+    w /= np.max(np.abs(w), axis=1, keepdims=True)                 # each block's absmax 1 ...
+    w *= np.exp2(rng.integers(-20, -12, (w.shape[0], 1))).astype(np.float32)  # ... times 2^e
+    w[0] *= 448.0 * 2.0 ** -12 / np.max(np.abs(w[0]))              # group max 448 * 2^-12
+    wb = w.reshape(4, -1).astype(ml_dtypes.bfloat16).view(np.uint16)
+    c1 = O.block_absmax(wb)
+    _, scales, c2 = O.quantize_nf4(wb)
+    assert np.array_equal(_scale_of_bytes(scales, c2), c1)
+    assert np.array_equal(O.quantize_nf4(wb, snap_to_dq_scale=True)[0], O.quantize_nf4(wb)[0])
+
+
+def test_dq_scale_snapping_lowers_the_round_trip_error():
+    """Dequantization multiplies by s_b, so snapping against s_b picks, per
+    weight, the level whose reconstruction is nearest: on N(0, 0.02^2) weights
+    no weight's error grows and the RMS error falls, for each table."""
+    rows, cols = 64, 4096
+    wb = _bits((rows, cols), 0.02, 321)
+    w = O.bf16_bits_to_f32(wb).astype(F64)
+    tables = [O.nf4_codebook(), O.nf4_codebook_with_zero(), np.array([(i - 8) / 8.0 for i in range(16)], F32)]
+    for cb in tables:
+        errs = []
+        for dq in (False, True):
+            codes, scales, c2 = O.quantize_nf4(wb, cb, snap_to_dq_scale=dq)
+            qv = cb.astype(F64)[O.unpack_codes(codes)].reshape(rows, cols)
+            sb = _scale_of_bytes(scales, c2).astype(F64).repeat(64).reshape(rows, cols)
+            errs.append(np.abs(qv * sb - w))        # reconstruction before the final BF16 rounding
+        assert np.all(errs[1] <= errs[0] * (1 + 1e-6) + 1e-12)
+        assert np.sqrt((errs[1] ** 2).mean()) < 0.999 * np.sqrt((errs[0] ** 2).mean())
+
+
+# --------------------------------------------------------------------------
+# the adapters' optimizer step (Adam with decoupled weight decay)
+# --------------------------------------------------------------------------
+
+def test_adam_first_step_is_lr_times_sign():
+    """From zero moments the first step's bias-corrected m and v are g and g^2,
+    so each parameter moves by lr g / (|g| + eps)."""
+    g = _bits((1, 257), 0.3, 41)
+    gf = O.bf16_bits_to_f32(g).astype(F64).reshape(-1)
+    p0 = np.linspace(-1, 1, 257)
+    p, m, v = O.adam_step(p0, np.zeros(257), np.zeros(257), g, 1, lr=1e-3, eps=1e-8)
+    assert np.allclose(p, p0 - 1e-3 * gf / (np.abs(gf) + 1e-8), rtol=0, atol=1e-15)
+    assert np.allclose(m, 0.1 * gf) and np.allclose(v, 0.001 * gf * gf)
+
+
+def test_adam_constant_gradient_closed_form():
+    """With the same gradient every step the bias-corrected moments stay g and
+    g^2, so after t steps param = p0 - t lr g / (|g| + eps)."""
+    g = _bits((1, 64), 0.5, 42)
+    gf = O.bf16_bits_to_f32(g).astype(F64).reshape(-1)
+    p, m, v = np.ones(64), np.zeros(64), np.zeros(64)
+    for t in range(1, 26):
+        p, m, v = O.adam_step(p, m, v, g, t, lr=2e-3, beta1=0.8, beta2=0.95, eps=1e-6)
+    assert np.allclose(p, 1.0 - 25 * 2e-3 * gf / (np.abs(gf) + 1e-6), rtol=0, atol=1e-12)
+
+
+def test_adam_weight_decay_alone_is_geometric():
+    g = np.zeros(16, np.uint16)                       # BF16 +0.0 gradients
+    p = np.full(16, 3.0)
+    m, v = np.zeros(16), np.zeros(16)
+    for t in range(1, 11):
+        p, m, v = O.adam_step(p, m, v, g, t, lr=0.01, weight_decay=0.1)
+    assert np.allclose(p, 3.0 * (1 - 0.01 * 0.1) ** 10, rtol=1e-15)
+
+
+def test_adam_matches_torch_adamw():
+    """Seven steps against torch.optim.AdamW (an independent implementation of
+    the same published algorithm) in float64 on the CPU."""
+    n = 1000
+    p0 = np.random.default_rng(3).normal(0, 0.05, n)
+    tp = torch.nn.Parameter(torch.tensor(p0, dtype=torch.float64))
+    opt = torch.optim.AdamW([tp], lr=3e-3, betas=(0.85, 0.98), eps=1e-7, weight_decay=0.05)
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t in range(1, 8):
+        g = _bits((1, n), 0.02, 100 + t).reshape(-1)
+        tp.grad = torch.from_numpy(O.bf16_bits_to_f32(g).astype(F64))
+        opt.step()
+        p, m, v = O.adam_step(p, m, v, g, t, lr=3e-3, beta1=0.85, beta2=0.98, eps=1e-7, weight_decay=0.05)
+    assert np.allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-16)
