@@ -19,8 +19,10 @@ import torch
 from . import _lib
 from ._lib import OP_BWD, OP_FWD, OP_QUANTIZE, NF4Weight, QLoraError, check, lib
 
-__all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "linear_fwd",
-           "linear_bwd", "linear_fwd_noalloc", "workspace", "workspace_bytes", "get_error", "QLoraError", "lib"]
+__all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "merge_adapter",
+           "linear_fwd", "linear_bwd", "linear_fwd_save", "linear_bwd_saved", "saved_u_bytes",
+           "linear_fwd_noalloc", "noalloc_get_error", "wait_selftest", "workspace", "workspace_bytes",
+           "get_error", "adam_step", "PagedBuffer", "QLoraError", "lib"]
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -108,8 +110,11 @@ def get_error(device=None) -> None:
     check("qlora_get_error", lib().qlora_get_error(C.c_void_p(ws.data_ptr()), _stream(dev)))
 
 
-def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: int = 256) -> QuantizedNF4:
-    """NF4 + double quantization of a BF16 weight w[rows, cols] on the GPU."""
+def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: int = 256,
+                 snap_to_dq_scale: bool = False) -> QuantizedNF4:
+    """NF4 + double quantization of a BF16 weight w[rows, cols] on the GPU.
+    snap_to_dq_scale: snap the codes against the double-quantized block scale
+    (the one dequantization multiplies by) instead of the exact absmax."""
     _need_cuda("w", w)
     if w.dim() != 2:
         raise ValueError("w must be 2-D [rows, cols]")
@@ -127,8 +132,9 @@ def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: 
     cbuf = (C.c_float * 16)(*cb)
     wsb = workspace_bytes(OP_QUANTIZE, 0, 0, 0, 1)
     ws = workspace(dev, wsb)
-    check("qlora_quantize_nf4", lib().qlora_quantize_nf4(
-        C.c_void_p(w.data_ptr()), rows, cols, blocksize, dq_block, cbuf, C.byref(out),
+    flags = _lib.QUANT_SNAP_DQ_SCALE if snap_to_dq_scale else 0
+    check("qlora_quantize_nf4_ex", lib().qlora_quantize_nf4_ex(
+        C.c_void_p(w.data_ptr()), rows, cols, blocksize, dq_block, cbuf, flags, C.byref(out),
         C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
     return QuantizedNF4(codes, scales, c2, rows, cols, cb, blocksize, dq_block)
 
@@ -166,7 +172,25 @@ def _check_linear(x, qw, A, B):
     r = A.shape[0]
     if tuple(A.shape) != (r, qw.cols) or tuple(B.shape) != (qw.rows, r):
         raise ValueError(f"A must be [r, {qw.cols}] and B [{qw.rows}, r]")
+    for n, t in (("A", A), ("B", B), ("qw", qw.codes)):
+        if t.device != x.device:
+            raise ValueError(f"{n} is on {t.device}, x on {x.device}")
     return x.shape[0], r
+
+
+def _check_out(name, t, shape, device):
+    """An output buffer the kernels write: a contiguous bf16 CUDA tensor of
+    exactly `shape` on `device` (the epilogues write every element of it)."""
+    _need_cuda(name, t)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {list(shape)}, got {list(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def saved_u_bytes(T: int, r: int) -> int:
+    """Bytes of the U = s x A^T planes the forward saves for the backward."""
+    return int(lib().qlora_saved_u_bytes(T, r))
 
 
 def linear_fwd(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
@@ -174,6 +198,8 @@ def linear_fwd(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tens
     """y = x W'^T + s (x A^T) B^T (BF16), W' dequantized inside the kernel."""
     T, r = _check_linear(x, qw, A, B)
     dev = x.device
+    if out is not None:
+        _check_out("out", out, (T, qw.rows), dev)
     y = out if out is not None else torch.empty(T, qw.rows, dtype=torch.bfloat16, device=dev)
     ws = workspace(dev, workspace_bytes(OP_FWD, T, qw.rows, qw.cols, r))
     st = qw.struct()
@@ -183,13 +209,37 @@ def linear_fwd(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tens
     return y
 
 
+def linear_fwd_save(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
+                    out: torch.Tensor | None = None, u_save: torch.Tensor | None = None):
+    """The forward that also returns U = s x A^T (hi + lo BF16 planes, as a
+    uint8 buffer of saved_u_bytes(T, r)) for linear_bwd_saved."""
+    T, r = _check_linear(x, qw, A, B)
+    dev = x.device
+    if out is not None:
+        _check_out("out", out, (T, qw.rows), dev)
+    y = out if out is not None else torch.empty(T, qw.rows, dtype=torch.bfloat16, device=dev)
+    nbytes = saved_u_bytes(T, r)
+    if u_save is None:
+        u_save = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _need_cuda("u_save", u_save, dtype=torch.uint8)
+    if u_save.numel() < nbytes or u_save.device != dev:
+        raise ValueError(f"u_save must hold {nbytes} bytes on {dev}")
+    ws = workspace(dev, workspace_bytes(OP_FWD, T, qw.rows, qw.cols, r))
+    st = qw.struct()
+    check("qlora_linear_fwd_save", lib().qlora_linear_fwd_save(
+        C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()), C.c_void_p(B.data_ptr()), r,
+        float(s), C.c_void_p(y.data_ptr()), C.c_void_p(u_save.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(),
+        _stream(dev)))
+    return y, u_save
+
+
 def linear_fwd_noalloc(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
                        out: torch.Tensor) -> torch.Tensor:
     """Forward through the entry point that uses the library's fixed device
     scratch instead of a workspace (for callers that cannot allocate device
-    memory); `out` must be preallocated [T, N] bf16."""
+    memory); `out` must be preallocated [T, N] bf16 on x's device."""
     T, r = _check_linear(x, qw, A, B)
-    _need_cuda("out", out)
+    _check_out("out", out, (T, qw.rows), x.device)
     st = qw.struct()
     check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(
         C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()), C.c_void_p(B.data_ptr()), r,
@@ -197,20 +247,48 @@ def linear_fwd_noalloc(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: to
     return out
 
 
+def noalloc_get_error(device=None) -> None:
+    """Synchronize and raise if an allocation-free forward on `device` recorded
+    a device-side failure (reads and clears the fixed array's status word)."""
+    dev = torch.device(device if device is not None else torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        check("qlora_noalloc_get_error", lib().qlora_noalloc_get_error(_stream(dev)))
+
+
+def wait_selftest(limit_us: int, device=None, noalloc: bool = False) -> None:
+    """Run the bounded-wait self-test kernel on `device` (its wait runs out
+    after limit_us); the timeout is then reported by get_error(device), or by
+    noalloc_get_error(device) when `noalloc` puts it in the allocation-free
+    forward's fixed array."""
+    dev = torch.device(device if device is not None else torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        if noalloc:
+            st = lib().qlora_wait_selftest(None, 0, int(limit_us), _stream(dev))
+        else:
+            ws = workspace(dev, 4096)
+            st = lib().qlora_wait_selftest(C.c_void_p(ws.data_ptr()), ws.numel(), int(limit_us), _stream(dev))
+    check("qlora_wait_selftest", st)
+
+
+def _bwd_outs(outs, T, qw, r, dev):
+    if outs is None:
+        return (torch.empty(T, qw.cols, dtype=torch.bfloat16, device=dev),
+                torch.empty(r, qw.cols, dtype=torch.bfloat16, device=dev),
+                torch.empty(qw.rows, r, dtype=torch.bfloat16, device=dev))
+    dx, dA, dB = outs
+    _check_out("dx", dx, (T, qw.cols), dev)
+    _check_out("dA", dA, (r, qw.cols), dev)
+    _check_out("dB", dB, (qw.rows, r), dev)
+    return dx, dA, dB
+
+
 def linear_bwd(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,
                outs=None):
     """(dX, dA, dB) of the layer for upstream gradient dy[T, N]."""
     T, r = _check_linear(x, qw, A, B)
-    _need_cuda("dy", dy)
-    if tuple(dy.shape) != (T, qw.rows):
-        raise ValueError(f"dy must be [{T}, {qw.rows}]")
     dev = x.device
-    if outs is None:
-        dx = torch.empty(T, qw.cols, dtype=torch.bfloat16, device=dev)
-        dA = torch.empty(r, qw.cols, dtype=torch.bfloat16, device=dev)
-        dB = torch.empty(qw.rows, r, dtype=torch.bfloat16, device=dev)
-    else:
-        dx, dA, dB = outs
+    _check_out("dy", dy, (T, qw.rows), dev)
+    dx, dA, dB = _bwd_outs(outs, T, qw, r, dev)
     ws = workspace(dev, workspace_bytes(OP_BWD, T, qw.rows, qw.cols, r))
     st = qw.struct()
     check("qlora_linear_bwd", lib().qlora_linear_bwd(
@@ -218,3 +296,96 @@ def linear_bwd(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedNF4, A: torch.Ten
         C.c_void_p(B.data_ptr()), r, float(s), C.c_void_p(dx.data_ptr()), C.c_void_p(dA.data_ptr()),
         C.c_void_p(dB.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(dev)))
     return dx, dA, dB
+
+
+def linear_bwd_saved(dy: torch.Tensor, x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor,
+                     s: float, u_saved: torch.Tensor, outs=None):
+    """linear_bwd with U taken from linear_fwd_save's buffer instead of
+    recomputed from x."""
+    T, r = _check_linear(x, qw, A, B)
+    dev = x.device
+    _check_out("dy", dy, (T, qw.rows), dev)
+    _need_cuda("u_saved", u_saved, dtype=torch.uint8)
+    if u_saved.numel() < saved_u_bytes(T, r) or u_saved.device != dev:
+        raise ValueError(f"u_saved must hold {saved_u_bytes(T, r)} bytes on {dev}")
+    dx, dA, dB = _bwd_outs(outs, T, qw, r, dev)
+    ws = workspace(dev, workspace_bytes(OP_BWD, T, qw.rows, qw.cols, r))
+    st = qw.struct()
+    check("qlora_linear_bwd_saved", lib().qlora_linear_bwd_saved(
+        C.c_void_p(dy.data_ptr()), C.c_void_p(x.data_ptr()), T, C.byref(st), C.c_void_p(A.data_ptr()),
+        C.c_void_p(B.data_ptr()), r, float(s), C.c_void_p(u_saved.data_ptr()), C.c_void_p(dx.data_ptr()),
+        C.c_void_p(dA.data_ptr()), C.c_void_p(dB.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(),
+        _stream(dev)))
+    return dx, dA, dB
+
+
+# --------------------------------------------------------------------------
+# the adapters' optimizer step, with its state optionally in unified memory
+# --------------------------------------------------------------------------
+class PagedBuffer:
+    """`n` elements of unified ("paged") memory from qlora_paged_alloc: the
+    driver keeps them on the GPU while there is room and pages them out to host
+    memory under pressure.  `.ptr` is the address the kernels take; `.numpy()`
+    views the same memory from the host (synchronize first).  Freed on delete."""
+
+    _CT = {torch.float32: C.c_float, torch.bfloat16: C.c_uint16, torch.uint8: C.c_uint8}
+
+    def __init__(self, n: int, dtype=torch.float32, device=None):
+        if dtype not in self._CT:
+            raise ValueError(f"unsupported dtype {dtype}")
+        self.n, self.dtype = int(n), dtype
+        self.device = torch.device(device if device is not None else torch.cuda.current_device())
+        self.nbytes = max(16, self.n * torch.empty((), dtype=dtype).element_size())
+        p = C.c_void_p()
+        with torch.cuda.device(self.device):
+            check("qlora_paged_alloc", lib().qlora_paged_alloc(self.nbytes, C.byref(p)))
+        self.ptr = p.value
+
+    def numpy(self):
+        import numpy as np
+        arr = (self._CT[self.dtype] * self.n).from_address(self.ptr)
+        return np.ctypeslib.as_array(arr)
+
+    def prefetch(self, to_host: bool = False):
+        with torch.cuda.device(self.device):
+            check("qlora_paged_prefetch", lib().qlora_paged_prefetch(C.c_void_p(self.ptr), self.nbytes,
+                                                                     1 if to_host else 0, _stream(self.device)))
+
+    def __del__(self):
+        if getattr(self, "ptr", None):
+            try:
+                torch.cuda.synchronize(self.device)
+                lib().qlora_paged_free(C.c_void_p(self.ptr))
+            except Exception:
+                pass
+            self.ptr = None
+
+
+def _addr(name, t, dtype, n, device):
+    if isinstance(t, PagedBuffer):
+        if t.dtype != dtype or t.n < n:
+            raise ValueError(f"{name} must hold {n} {dtype}")
+        return t.ptr
+    _need_cuda(name, t, dtype=dtype)
+    if t.numel() < n or t.device != device:
+        raise ValueError(f"{name} must hold {n} elements on {device}")
+    return t.data_ptr()
+
+
+def adam_step(param, m, v, grad: torch.Tensor, param_bf16: torch.Tensor | None = None, *, step: int, lr: float,
+              beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0) -> None:
+    """One Adam step (decoupled weight decay) of the FP32 adapter parameters
+    `param` with moments `m`, `v` (torch CUDA tensors or PagedBuffers) from the
+    BF16 gradient `grad` (dA or dB); writes the BF16 copy of the new
+    parameters to `param_bf16` if given.  Elementwise over grad.numel()."""
+    n = grad.numel()
+    dev = grad.device
+    _need_cuda("grad", grad)
+    ptrs = [_addr(nm, t, torch.float32, n, dev) for nm, t in (("param", param), ("m", m), ("v", v))]
+    out = None
+    if param_bf16 is not None:
+        out = _addr("param_bf16", param_bf16, torch.bfloat16, n, dev)
+    h = _lib.AdamHParams(lr, beta1, beta2, eps, weight_decay, int(step))
+    check("qlora_adam_step", lib().qlora_adam_step(C.c_void_p(ptrs[0]), C.c_void_p(ptrs[1]), C.c_void_p(ptrs[2]),
+                                                   C.c_void_p(grad.data_ptr()), C.c_void_p(out), n, C.byref(h),
+                                                   _stream(dev)))

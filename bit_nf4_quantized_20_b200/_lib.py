@@ -18,6 +18,7 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
                 3: "QLORA_ERR_MISALIGNED", 4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA",
                 6: "QLORA_ERR_NONFINITE", 7: "QLORA_ERR_TIMEOUT"}
 OP_QUANTIZE, OP_FWD, OP_BWD = 0, 1, 2
+QUANT_SNAP_DQ_SCALE = 1
 
 
 class NF4Weight(C.Structure):
@@ -26,6 +27,12 @@ class NF4Weight(C.Structure):
                 ("rows", C.c_int64), ("cols", C.c_int64),
                 ("blocksize", C.c_int32), ("dq_block", C.c_int32),
                 ("codebook", C.c_float * 16)]
+
+
+class AdamHParams(C.Structure):
+    """Mirror of qlora_adam_hparams."""
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float), ("step", C.c_int32)]
 
 
 class TraceRec(C.Structure):
@@ -47,6 +54,9 @@ SIGNATURES = {
     "qlora_quantize_nf4": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int32, C.c_int32,
                                      C.POINTER(C.c_float), C.POINTER(NF4Weight), C.c_void_p, C.c_size_t,
                                      C.c_void_p]),
+    "qlora_quantize_nf4_ex": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_int32, C.c_int32,
+                                        C.POINTER(C.c_float), C.c_uint32, C.POINTER(NF4Weight), C.c_void_p,
+                                        C.c_size_t, C.c_void_p]),
     "qlora_dequantize": (C.c_int, [C.POINTER(NF4Weight), C.c_void_p, C.c_void_p]),
     "qlora_merge_adapter": (C.c_int, [C.POINTER(NF4Weight), C.c_void_p, C.c_void_p, C.c_int32, C.c_float,
                                       C.c_void_p, C.c_void_p]),
@@ -57,6 +67,20 @@ SIGNATURES = {
                                    C.c_void_p, C.c_size_t, C.c_void_p]),
     "qlora_linear_fwd_noalloc": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
                                            C.c_int32, C.c_float, C.c_void_p, C.c_void_p]),
+    "qlora_noalloc_get_error": (C.c_int, [C.c_void_p]),
+    "qlora_saved_u_bytes": (C.c_size_t, [C.c_int64, C.c_int32]),
+    "qlora_linear_fwd_save": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
+                                        C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
+                                        C.c_void_p]),
+    "qlora_linear_bwd_saved": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p,
+                                         C.c_void_p, C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
+                                         C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qlora_wait_selftest": (C.c_int, [C.c_void_p, C.c_size_t, C.c_uint32, C.c_void_p]),
+    "qlora_adam_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64,
+                                  C.POINTER(AdamHParams), C.c_void_p]),
+    "qlora_paged_alloc": (C.c_int, [C.c_size_t, C.POINTER(C.c_void_p)]),
+    "qlora_paged_free": (C.c_int, [C.c_void_p]),
+    "qlora_paged_prefetch": (C.c_int, [C.c_void_p, C.c_size_t, C.c_int32, C.c_void_p]),
     "qlora_trace_attach": (C.c_int, [C.POINTER(TraceRec), C.c_int32, C.POINTER(C.c_int32)]),
     "qlora_kernel_name": (C.c_char_p, [C.c_int32]),
 }

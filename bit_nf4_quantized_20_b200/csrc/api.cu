@@ -14,6 +14,33 @@
 
 using namespace qlora;
 
+namespace qlora {
+
+// Dynamic shared memory above 48 KB needs an opt-in per kernel and per device;
+// a process that drives several GPUs makes it once on each.
+cudaError_t ensure_smem_optin(const void *func, int bytes) {
+  struct Entry {
+    const void *func;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry done[256];
+  static int n_done = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].func == func && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (n_done < 256) done[n_done++] = Entry{func, dev, bytes};
+  return cudaSuccess;
+}
+
+}  // namespace qlora
+
 namespace {
 
 // ---------------------------------------------------------------------------
@@ -39,12 +66,15 @@ enum KernelId : int32_t {
   K_LORA_U_DU = 9,      // U and dU in one grid (backward)
   K_LORA_DB_DA = 10,    // dB and dA in one grid (backward)
   K_MERGE = 11,         // adapter merge for export
-  K_COUNT = 12,
+  K_LORA_DU_DB = 12,    // dU and dB in one grid (backward with the forward's saved U)
+  K_ADAM = 13,          // the adapters' optimizer step
+  K_COUNT = 14,
 };
 
 const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",       "lora_du",
                                      "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx",
-                                     "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA",   "merge_adapter"};
+                                     "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA",   "merge_adapter",
+                                     "lora_du+dB",      "adam_step"};
 
 struct TraceScope {
   cudaStream_t st;
@@ -226,9 +256,9 @@ bool decode_path(int64_t T, int64_t N) {
 
 struct WsLayout {
   size_t counters = 0;
-  size_t su_row = 0;                 // forward: sU [T, ceil64(r)] (rank-r operand of the GEMM / GEMV)
+  size_t su_row = 0;                 // forward: sU hi | lo [T, 2 ceil64(r)] (rank-r operand of the GEMM / GEMV)
   size_t suT_hi = 0, suT_lo = 0;     // backward: sU^T planes [r, ceil8(T)]
-  size_t du_row = 0;                 // backward: dU hi [T, ceil64(r)] (rank-r operand of the dX GEMM)
+  size_t du_row = 0;                 // backward: dU hi | lo [T, 2 ceil64(r)] (rank-r operand of the dX GEMM)
   size_t duT_hi = 0, duT_lo = 0;     // backward: dU^T planes [r, ceil8(T)]
   size_t bpad = 0;                   // backward: B copied to [N, ceil64(r)] when TMA cannot read it in place
   size_t partials = 0, total = 0;
@@ -242,15 +272,19 @@ struct PairGeom {
   SkinnyTcGeom g0, g1;
   size_t part0, part1;   // partial-buffer bytes (the second starts 256-aligned after the first)
 };
-PairGeom pair_geom(int64_t M0, int64_t C0, bool q0, int64_t M1, int64_t C1, bool q1, int r, int nq) {
+PairGeom pair_geom(int64_t M0, int64_t C0, bool q0, int nq0, int64_t M1, int64_t C1, bool q1, int nq1, int r) {
   PairGeom pg;
-  skinny_tc_pair_geom(M0, C0, q0, M1, C1, q1, r, nq, kSplitSms, pg.g0, pg.g1);
+  skinny_tc_pair_geom(M0, C0, q0, nq0, M1, C1, q1, nq1, r, kSplitSms, pg.g0, pg.g1);
   pg.part0 = skinny_tc_partials_bytes(pg.g0, M0, r);
   pg.part1 = skinny_tc_partials_bytes(pg.g1, M1, r);
   return pg;
 }
-PairGeom geom_u_du(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(T, K, false, T, N, true, r, 1); }
-PairGeom geom_db_da(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(N, T, false, K, T, false, r, 2); }
+// U [T, r] with dU [T, r]; dB [N, r] with dA [r, K] (written as [K, r] products)
+PairGeom geom_u_du(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(T, K, false, 1, T, N, true, 1, r); }
+PairGeom geom_db_da(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(N, T, false, 2, K, T, false, 2, r); }
+// with U saved by the forward: dU with dB (both stream dY), then dA alone
+PairGeom geom_du_db(int64_t T, int64_t N, int r) { return pair_geom(T, N, true, 1, N, T, false, 2, r); }
+SkinnyTcGeom geom_da(int64_t T, int64_t K, int r) { return skinny_tc_geom(K, T, r, 2, false, kSplitSms); }
 size_t pair_partials(const PairGeom &pg) {
   return static_cast<size_t>(round_up(static_cast<int64_t>(pg.part0), 256)) + pg.part1;
 }
@@ -265,18 +299,18 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     return L;
   }
   const int64_t r64 = round_up(r, 64);
-  const size_t row_plane = static_cast<size_t>(round_up(T * r64 * 2, 256));
+  const size_t row_plane = static_cast<size_t>(round_up(T * 2 * r64 * 2, 256));   // hi and lo per row
   const size_t t_plane = static_cast<size_t>(round_up(r * round_up(T, 8) * 2, 256));
   size_t part = 0;
   if (op == QLORA_OP_FWD) {
     L.su_row = off; off += row_plane;
-    if (decode_path(T, N)) {
-      // the U' fallback's partials, then (after it has finished) the GEMV's split partials
-      part = std::max(skinny_partials_bytes(T, K, r, kSplitSms),
-                      gemv_persist_partials_bytes(N, K, kGemvMaxCounterTiles));
-    } else {
-      part = skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
-    }
+    // the tensor-core U product (every token count when U is saved for the
+    // backward); at decode sizes also the U' fallback's partials and, after
+    // it has finished, the GEMV's split partials
+    part = skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
+    if (decode_path(T, N))
+      part = std::max(part, std::max(skinny_partials_bytes(T, K, r, kSplitSms),
+                                     gemv_persist_partials_bytes(N, K, kGemvMaxCounterTiles)));
   } else {
     L.suT_hi = off; off += t_plane;
     L.suT_lo = off; off += t_plane;
@@ -284,7 +318,8 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     L.duT_hi = off; off += t_plane;
     L.duT_lo = off; off += t_plane;
     L.bpad = off; off += static_cast<size_t>(round_up(N * r64 * 2, 256));
-    const size_t p[2] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r))};
+    const size_t p[4] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r)),
+                         pair_partials(geom_du_db(T, N, r)), skinny_tc_partials_bytes(geom_da(T, K, r), K, r)};
     for (size_t v : p) part = v > part ? v : part;
   }
   L.partials = off;
@@ -309,30 +344,26 @@ SkinnyParams skinny_base(int64_t M, int64_t C, int R, uint8_t *ws, const WsLayou
   return p;
 }
 
-// The one-CTA GEMM kernel is kept for comparison measurements; setting
-// QLORA_GEMM_ONE_CTA=1 in the environment selects it.
-bool use_one_cta_gemm() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("QLORA_GEMM_ONE_CTA");
-    v = (e && e[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
+// The fused GEMM's launch, prepared (tensor maps encoded, parameters filled)
+// before anything of the call is enqueued.
+struct GemmLaunch {
+  CUtensorMap m_act, m_lact, m_out;
+  GemmParams p;
+  int64_t clusters;
+  int32_t kid;
+  double flops, bytes;
+};
 
-qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, const void *lact, int64_t r64,
-                      const void *lora, int r, void *out, int64_t T, uint32_t *status, cudaStream_t st) {
+qlora_status prepare_gemm(int mode, const qlora_nf4_weight *qw, const void *act, const void *lact, int64_t r64,
+                          const void *lora, int r, void *out, int64_t T, uint32_t *status, GemmLaunch &g) {
   const int64_t N = qw->rows, K = qw->cols;
   const int64_t Mside = mode == 0 ? N : K;     // weight-side extent
   const int64_t Cext = mode == 0 ? K : N;      // contraction extent
-  // the CTA-pair kernel (default) loads 128 tokens per CTA; the one-CTA kernel 256
-  const bool pair = !use_one_cta_gemm();
-  const int act_rows = pair ? 128 : 256;
-  CUtensorMap m_act, m_lact, m_out;
-  if (!make_map_bf16(&m_act, act, T, Cext, Cext, act_rows, 64, true)) return QLORA_ERR_CUDA;
-  if (!make_map_bf16(&m_lact, lact, T, r64, r64, act_rows, 64, true)) return QLORA_ERR_CUDA;
-  if (!make_map_bf16(&m_out, out, T, Mside, Mside, 32, 128, false)) return QLORA_ERR_CUDA;
-  GemmParams p;
+  // each CTA of a pair loads 128 of the tile's 256 tokens
+  if (!make_map_bf16(&g.m_act, act, T, Cext, Cext, 128, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&g.m_lact, lact, T, 2 * r64, 2 * r64, 128, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&g.m_out, out, T, Mside, Mside, 32, 128, false)) return QLORA_ERR_CUDA;
+  GemmParams &p = g.p;
   memset(&p, 0, sizeof(p));
   p.codes = qw->codes;
   p.scales = qw->scales;
@@ -344,58 +375,48 @@ qlora_status run_gemm(int mode, const qlora_nf4_weight *qw, const void *act, con
   p.mode = mode;
   p.lora = static_cast<const uint16_t *>(lora);
   p.r = r;
-  p.m_tiles = static_cast<int>((Mside + (pair ? 255 : 127)) / (pair ? 256 : 128));
+  p.m_tiles = static_cast<int>((Mside + 255) / 256);
   p.n_tiles = static_cast<int>((T + 255) / 256);
   p.k_main = static_cast<int>((Cext + 63) / 64);
-  p.k_lora = static_cast<int>(r64 / 64);
+  p.k_lora_plane = static_cast<int>(r64 / 64);
+  p.k_lora = 2 * p.k_lora_plane;   // hi plane, then lo plane
   p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
   p.status = status;
   p.out = static_cast<uint16_t *>(out);
   p.ldo = Mside;
-  const double flops = 2.0 * T * N * K + 2.0 * T * r * Mside;
-  const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
+  g.flops = 2.0 * T * N * K + 2.0 * T * r * Mside;   // algorithmic: the lo plane's MMAs are not counted
+  g.bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 64) + 2.0 * T * (Cext + Mside);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   const int sms = num_sms_current();
-  if (pair) {
-    static bool attr2 = false;
-    if (!attr2) {
-      if (cudaFuncSetAttribute(nf4_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               gemm_2sm_smem_bytes()) != cudaSuccess)
-        return QLORA_ERR_CUDA;
-      attr2 = true;
-    }
-    const int64_t clusters = tiles < sms / 2 ? tiles : sms / 2;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-    cfg.blockDim = dim3(576, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(gemm_2sm_smem_bytes());
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    TraceScope ts(mode == 0 ? K_GEMM_FWD : K_GEMM_BWD, flops, bytes, st);
-    return cudaLaunchKernelEx(&cfg, nf4_gemm_2sm_kernel, m_act, m_lact, m_out, p) == cudaSuccess ? QLORA_OK
-                                                                                                  : QLORA_ERR_CUDA;
-  }
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(nf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes()) !=
-        cudaSuccess)
-      return QLORA_ERR_CUDA;
-    attr_set = true;
-  }
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  TraceScope ts(mode == 0 ? K_GEMM_FWD : K_GEMM_BWD, flops, bytes, st);
-  nf4_gemm_kernel<<<grid, 320, gemm_smem_bytes(), st>>>(m_act, m_lact, m_out, p);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  g.clusters = tiles < sms / 2 ? tiles : sms / 2;
+  g.kid = mode == 0 ? K_GEMM_FWD : K_GEMM_BWD;
+  return QLORA_OK;
+}
+
+qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
+  if (ensure_smem_optin(reinterpret_cast<const void *>(nf4_gemm_2sm_kernel), gemm_2sm_smem_bytes()) !=
+      cudaSuccess)
+    return QLORA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * g.clusters), 1, 1);
+  cfg.blockDim = dim3(576, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(gemm_2sm_smem_bytes());
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TraceScope ts(g.kid, g.flops, g.bytes, st);
+  return cudaLaunchKernelEx(&cfg, nf4_gemm_2sm_kernel, g.m_act, g.m_lact, g.m_out, g.p) == cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
 }
 
 
-// The decode forward; u holds U' = BF16(s X A^T) [T, ldu].
+// The decode forward; u holds U' = s X A^T as hi | lo BF16 planes per row [T, ldu].
 qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
                       const void *B, int r, void *y, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
   GemvParams p;
@@ -467,31 +488,49 @@ bool prepare_tc(const TcProduct &t, SkinnyTcArgs &a, uint8_t *ws, size_t part_of
   return true;
 }
 
-qlora_status run_skinny_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
-  CUtensorMap maps[3];
-  if (!prepare_tc(t, a, ws, L.partials, L.counters, maps)) return QLORA_ERR_CUDA;
-  const double flops = 2.0 * a.M * a.C * a.R * a.nq;
-  const double bytes = 2.0 * a.M * a.C;
-  const bool pdl = g_trace.recs == nullptr;
-  TraceScope ts(t.kid, flops, bytes, st);
-  return launch_skinny_tc(a, maps[0], maps[1], maps[2], st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+// A prepared tensor-core rank-r launch: one product, or two in one grid.
+struct TcLaunch {
+  int32_t kid;
+  bool pair;
+  SkinnyTcArgs a0, a1;
+  CUtensorMap m0[3], m1[3];
+  double flops, bytes;
+};
+
+qlora_status prepare_single_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L,
+                               TcLaunch &l) {
+  if (!prepare_tc(t, a, ws, L.partials, L.counters, l.m0)) return QLORA_ERR_CUDA;
+  l.kid = t.kid;
+  l.pair = false;
+  l.a0 = a;
+  l.flops = 2.0 * a.M * a.C * a.R * a.nq;
+  l.bytes = 2.0 * a.M * a.C;
+  return QLORA_OK;
 }
 
 // Two independent products in one grid; the second's partials follow the
 // first's, its counters follow the first's row tiles.
-qlora_status run_skinny_tc_pair(int32_t kid, const TcProduct &t0, SkinnyTcArgs a0, const TcProduct &t1,
-                                SkinnyTcArgs a1, const PairGeom &pg, uint8_t *ws, const WsLayout &L,
-                                cudaStream_t st) {
-  CUtensorMap m0[3], m1[3];
+qlora_status prepare_pair_tc(int32_t kid, const TcProduct &t0, SkinnyTcArgs a0, const TcProduct &t1,
+                             SkinnyTcArgs a1, const PairGeom &pg, uint8_t *ws, const WsLayout &L, TcLaunch &l) {
   const size_t part1 = L.partials + static_cast<size_t>(round_up(static_cast<int64_t>(pg.part0), 256));
   const size_t cnt1 = L.counters + static_cast<size_t>((a0.M + 127) / 128) * sizeof(uint32_t);
-  if (!prepare_tc(t0, a0, ws, L.partials, L.counters, m0) || !prepare_tc(t1, a1, ws, part1, cnt1, m1))
+  if (!prepare_tc(t0, a0, ws, L.partials, L.counters, l.m0) || !prepare_tc(t1, a1, ws, part1, cnt1, l.m1))
     return QLORA_ERR_CUDA;
-  const double flops = 2.0 * (a0.M * a0.C * a0.nq + a1.M * a1.C * a1.nq) * a0.R;
-  const double bytes = 2.0 * (a0.M * a0.C + a1.M * a1.C);
+  l.kid = kid;
+  l.pair = true;
+  l.a0 = a0;
+  l.a1 = a1;
+  l.flops = 2.0 * (a0.M * a0.C * a0.nq + a1.M * a1.C * a1.nq) * a0.R;
+  l.bytes = 2.0 * (a0.M * a0.C + a1.M * a1.C);
+  return QLORA_OK;
+}
+
+qlora_status launch_tc(const TcLaunch &l, cudaStream_t st) {
   const bool pdl = g_trace.recs == nullptr;
-  TraceScope ts(kid, flops, bytes, st);
-  return launch_skinny_tc_pair(a0, m0, a1, m1, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  TraceScope ts(l.kid, l.flops, l.bytes, st);
+  const cudaError_t e = l.pair ? launch_skinny_tc_pair(l.a0, l.m0, l.a1, l.m1, st, pdl)
+                               : launch_skinny_tc(l.a0, l.m0[0], l.m0[1], l.m0[2], st, pdl);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 SkinnyTcArgs tc_args(int64_t M, int64_t C, int R, float alpha) {
@@ -587,11 +626,12 @@ qlora_status qlora_get_error(void *ws, void *stream) {
   return QLORA_OK;
 }
 
-qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
-                                int32_t dq_block, const float codebook[16], qlora_nf4_weight *out, void *ws,
-                                size_t ws_bytes, void *stream) {
+qlora_status qlora_quantize_nf4_ex(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
+                                   int32_t dq_block, const float codebook[16], uint32_t flags, qlora_nf4_weight *out,
+                                   void *ws, size_t ws_bytes, void *stream) {
   if (!w_bf16 || !codebook || !out || !out->codes || !out->scales || !out->c2) return QLORA_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<uint32_t>(QLORA_QUANT_SNAP_DQ_SCALE)) != 0u) return QLORA_ERR_INVALID_ARG;
   if (blocksize != 64 || dq_block != 256 || cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
   if (!aligned16(w_bf16) || !aligned16(out->codes) || (reinterpret_cast<uintptr_t>(out->c2) & 3u))
     return QLORA_ERR_MISALIGNED;
@@ -614,8 +654,15 @@ qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, 
   const double n = static_cast<double>(rows) * cols;
   TraceScope ts(K_QUANTIZE, 0.0, n * 2.0 + n * (0.5 + 1.0 / 64) + 4.0 * ((nblocks + 255) / 256), st);
   cudaError_t e = launch_quantize(static_cast<const uint16_t *>(w_bf16), nblocks, out->codes, out->scales, out->c2,
-                                  tab, static_cast<uint32_t *>(ws), st, num_sms_current());
+                                  tab, (flags & QLORA_QUANT_SNAP_DQ_SCALE) != 0u, static_cast<uint32_t *>(ws), st,
+                                  num_sms_current());
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
+                                int32_t dq_block, const float codebook[16], qlora_nf4_weight *out, void *ws,
+                                size_t ws_bytes, void *stream) {
+  return qlora_quantize_nf4_ex(w_bf16, rows, cols, blocksize, dq_block, codebook, 0u, out, ws, ws_bytes, stream);
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight *qw, void *w_bf16_out, void *stream) {
@@ -660,25 +707,40 @@ static qlora_status check_linear(const void *x, int64_t T, const qlora_nf4_weigh
   return QLORA_OK;
 }
 
-qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A, const void *B,
-                              int32_t r, float s, void *y, void *ws, size_t ws_bytes, void *stream) {
+// Every argument check of the forward that does not involve the workspace.
+static qlora_status check_fwd(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A, const void *B,
+                              int32_t r, float s, const void *y, const void *u_save, bool want_save) {
   qlora_status cs = check_linear(x, T, qw, A, B, r, s);
   if (cs != QLORA_OK) return cs;
-  if (T > 0 && !y) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(y)) return QLORA_ERR_MISALIGNED;
+  if (T > 0 && (!y || (want_save && !u_save))) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(u_save)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+static bool ws_ok(const void *ws, size_t ws_bytes, int op, int64_t T, int64_t N, int64_t K, int r) {
+  return ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 && ws_bytes >= qlora_workspace_bytes(op, T, N, K, r);
+}
+
+// Offsets of the two planes of a saved U (hi, then lo) for T tokens at rank r.
+static size_t saved_plane_bytes(int64_t T, int r) {
+  return static_cast<size_t>(round_up(static_cast<int64_t>(r) * round_up(T, 8) * 2, 256));
+}
+
+// The forward after validation (T > 0).  u_save (optional): sU^T as hi + lo
+// planes [r, ceil8(T)] for the backward.
+static qlora_status linear_fwd_impl(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                                    const void *B, int32_t r, float s, void *y, void *u_save, void *ws,
+                                    cudaStream_t st) {
   const int64_t N = qw->rows, K = qw->cols;
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_FWD, T, N, K, r))
-    return QLORA_ERR_WORKSPACE;
-  if (T == 0) return QLORA_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   const WsLayout L = ws_layout(QLORA_OP_FWD, T, N, K, r);
   const int64_t r64 = round_up(r, 64);
   uint16_t *su = reinterpret_cast<uint16_t *>(w8 + L.su_row);
-  // sU = s X A^T [T, ceil64(r)]: the rank-r operand of the GEMV / GEMM
-  if (decode_path(T, N)) {
-    // a handful of rows: a latency-bound product, on a cluster kernel (one
-    // wave, partial sums in distributed shared memory) where its slice fits
+  const bool decode = decode_path(T, N);
+  if (decode && !u_save) {
+    // sU = s X A^T [T, ceil64(r)], a handful of rows: a latency-bound product,
+    // on a cluster kernel (one wave, partial sums in distributed shared
+    // memory) where its slice fits
     const bool pdl = g_trace.recs == nullptr;
     if (lora_u_decode_smem_bytes(K, static_cast<int>(T)) <= kLoraUDecodeMaxSmem) {
       LoraUDecodeParams pu;
@@ -686,7 +748,8 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
       pu.A = static_cast<const uint16_t *>(A);
       pu.u = su;
       pu.K = K;
-      pu.ldu = r64;
+      pu.ldu = 2 * r64;
+      pu.plane = r64;
       pu.T = static_cast<int>(T);
       pu.r = r;
       pu.kc = 0;
@@ -695,7 +758,7 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
         TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * r * K, st);
         if (launch_lora_u_decode(pu, st, pdl) != cudaSuccess) return QLORA_ERR_CUDA;
       }
-      return run_gemv(qw, x, T, su, r64, B, r, y, w8, L, st);
+      return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
     }
     SkinnyParams pu = skinny_base(T, K, r, w8, L);
     pu.P = static_cast<const uint16_t *>(x);
@@ -704,40 +767,51 @@ qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *
     pu.ldq = K;
     pu.alpha = s;
     pu.out0 = su;
-    pu.out1 = nullptr;
-    pu.ldo = r64;
+    pu.out1 = su + r64;
+    pu.ldo = 2 * r64;
+    pu.ocols = r64;
     {
       TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * T * K, st);
       if (launch_skinny(pu, false, false, OUT_HILO, st) != cudaSuccess) return QLORA_ERR_CUDA;
     }
-    return run_gemv(qw, x, T, su, r64, B, r, y, w8, L, st);
+    return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
   }
+  // sU on the tensor cores: the row plane for the GEMM / GEMV's rank-r term
+  // and, when the backward will need it, the transposed hi + lo planes
   SkinnyTcArgs au = tc_args(T, K, r, s);
   au.row_hi = su;
-  au.ldo = r64;
+  au.row_lo = su + r64;
+  au.ldo = 2 * r64;
+  au.ocols = r64;
+  if (u_save) {
+    uint8_t *u8 = static_cast<uint8_t *>(u_save);
+    au.t_hi = reinterpret_cast<uint16_t *>(u8);
+    au.t_lo = reinterpret_cast<uint16_t *>(u8 + saved_plane_bytes(T, r));
+    au.ldt = round_up(T, 8);
+  }
   const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, geom_u(T, K, r)};
-  qlora_status rs = run_skinny_tc(tu, au, w8, L, st);
+  TcLaunch lu;
+  qlora_status rs = prepare_single_tc(tu, au, w8, L, lu);
   if (rs != QLORA_OK) return rs;
-  return run_gemm(0, qw, x, su, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), st);
+  if (decode) {
+    rs = launch_tc(lu, st);
+    if (rs != QLORA_OK) return rs;
+    return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
+  }
+  GemmLaunch gl;
+  rs = prepare_gemm(0, qw, x, su, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), gl);
+  if (rs != QLORA_OK) return rs;
+  rs = launch_tc(lu, st);
+  if (rs != QLORA_OK) return rs;
+  return launch_gemm(gl, st);
 }
 
-qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
-                              const void *B, int32_t r, float s, void *dx, void *dA, void *dB, void *ws,
-                              size_t ws_bytes, void *stream) {
-  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
-  if (cs != QLORA_OK) return cs;
-  if ((T > 0 && (!dy || !dx)) || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(dy) || !aligned16(dx) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
+// The backward after validation (T > 0).  u_saved (optional): the planes the
+// forward saved; without them sU is recomputed from X.
+static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
+                                    const void *A, const void *B, int32_t r, float s, const void *u_saved, void *dx,
+                                    void *dA, void *dB, void *ws, cudaStream_t st) {
   const int64_t N = qw->rows, K = qw->cols;
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r))
-    return QLORA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T == 0) {
-    // no tokens: the adapter gradients are empty sums
-    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
-    return QLORA_OK;
-  }
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   const WsLayout L = ws_layout(QLORA_OP_BWD, T, N, K, r);
   const int64_t r64 = round_up(r, 64);
@@ -746,57 +820,144 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
   // TMA reads B in place for dU when its rows are a multiple of 16 bytes
   // (columns past r come back as zeros); otherwise B is first copied to
   // [N, ceil64(r)] rows.
-  const void *bq = B;
-  int64_t ldb = r;
-  if (r % 8 != 0 || !aligned16(B)) {
-    uint16_t *bpad = plane(L.bpad);
-    if (launch_pad_cols(static_cast<const uint16_t *>(B), N, r, bpad, static_cast<int>(r64), st,
-                        num_sms_current()) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    bq = bpad;
-    ldb = r64;
+  const bool pad_b = r % 8 != 0 || !aligned16(B);
+  const void *bq = pad_b ? static_cast<const void *>(plane(L.bpad)) : B;
+  const int64_t ldb = pad_b ? r64 : r;
+  // the sU^T planes: saved by the forward, or computed below
+  const uint16_t *su_hi = plane(L.suT_hi), *su_lo = plane(L.suT_lo);
+  if (u_saved) {
+    const uint8_t *u8 = static_cast<const uint8_t *>(u_saved);
+    su_hi = reinterpret_cast<const uint16_t *>(u8);
+    su_lo = reinterpret_cast<const uint16_t *>(u8 + saved_plane_bytes(T, r));
   }
-  // one grid: sU = s X A^T, transposed, as hi + lo planes [r, ceil8(T)]; and
-  // dU = s dY B as a hi plane [T, ceil64(r)] for the dX GEMM plus transposed hi
-  // + lo planes for dA
-  const PairGeom g1 = geom_u_du(T, N, K, r);
-  SkinnyTcArgs au = tc_args(T, K, r, s);
-  au.t_hi = plane(L.suT_hi);
-  au.t_lo = plane(L.suT_lo);
-  au.ldt = Tp;
+  // dU = s dY B as hi | lo planes [T, 2 ceil64(r)] for the dX GEMM plus
+  // transposed hi + lo planes for dA
   SkinnyTcArgs ad = tc_args(T, N, r, s);
   ad.row_hi = plane(L.du_row);
-  ad.ldo = r64;
+  ad.row_lo = plane(L.du_row) + r64;
+  ad.ldo = 2 * r64;
+  ad.ocols = r64;
   ad.t_hi = plane(L.duT_hi);
   ad.t_lo = plane(L.duT_lo);
   ad.ldt = Tp;
-  const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, g1.g0};
-  const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g1};
-  qlora_status rs = run_skinny_tc_pair(K_LORA_U_DU, tu, au, td, ad, g1, w8, L, st);
-  if (rs != QLORA_OK) return rs;
-  // one grid: dB = dY^T (sU) [N, r] and dA = dU^T X [r, K]; it needs only the
-  // planes above, so it runs on the side stream beside the dX GEMM (which
-  // touches no other workspace than the status word) and joins before return
-  const PairGeom g2 = geom_db_da(T, N, K, r);
+  // dB = dY^T (sU) [N, r] and dA = dU^T X [r, K]
   SkinnyTcArgs ab = tc_args(N, T, r, 1.0f);
   ab.row = static_cast<uint16_t *>(dB);
   SkinnyTcArgs aa = tc_args(K, T, r, 1.0f);
   aa.tr = static_cast<uint16_t *>(dA);
-  const TcProduct tb = {K_LORA_DB, dy, N, true, plane(L.suT_hi), plane(L.suT_lo), Tp, false, g2.g0};
-  const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
-  // (with a trace attached everything stays on the caller's stream, so that each
-  // launch's events time that launch alone)
-  SideStream *side = g_trace.recs == nullptr ? side_stream() : nullptr;
-  if (side && cudaEventRecord(side->fork, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  // dX = dY W' + dU A, first in line for the SMs
-  rs = run_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), st);
+
+  TcLaunch first, second;
+  qlora_status rs;
+  if (!u_saved) {
+    // one grid: sU = s X A^T, transposed, as hi + lo planes, with dU; then
+    // dB with dA in a second grid
+    const PairGeom g1 = geom_u_du(T, N, K, r);
+    SkinnyTcArgs au = tc_args(T, K, r, s);
+    au.t_hi = plane(L.suT_hi);
+    au.t_lo = plane(L.suT_lo);
+    au.ldt = Tp;
+    const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, g1.g0};
+    const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g1};
+    rs = prepare_pair_tc(K_LORA_U_DU, tu, au, td, ad, g1, w8, L, first);
+    if (rs != QLORA_OK) return rs;
+    const PairGeom g2 = geom_db_da(T, N, K, r);
+    const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, g2.g0};
+    const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
+    rs = prepare_pair_tc(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, second);
+  } else {
+    // one grid: dU with dB (both stream dY, sU comes from the forward); then
+    // dA alone
+    const PairGeom g1 = geom_du_db(T, N, r);
+    const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g0};
+    const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, g1.g1};
+    rs = prepare_pair_tc(K_LORA_DU_DB, td, ad, tb, ab, g1, w8, L, first);
+    if (rs != QLORA_OK) return rs;
+    const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, geom_da(T, K, r)};
+    rs = prepare_single_tc(ta, aa, w8, L, second);
+  }
   if (rs != QLORA_OK) return rs;
-  if (!side) return run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, st);
+  // dX = dY W' + dU A
+  GemmLaunch gl;
+  rs = prepare_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), gl);
+  if (rs != QLORA_OK) return rs;
+  // the second grid needs only the first's planes, not dX, so it runs on the
+  // side stream beside the dX GEMM (which touches no other workspace than the
+  // status word) and joins before return; with a trace attached everything
+  // stays on the caller's stream, so that each launch's events time that
+  // launch alone
+  SideStream *side = g_trace.recs == nullptr ? side_stream() : nullptr;
+
+  if (pad_b && launch_pad_cols(static_cast<const uint16_t *>(B), N, r, plane(L.bpad), static_cast<int>(r64), st,
+                               num_sms_current()) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  rs = launch_tc(first, st);
+  if (rs != QLORA_OK) return rs;
+  if (side && cudaEventRecord(side->fork, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  rs = launch_gemm(gl, st);   // first in line for the SMs
+  if (rs != QLORA_OK) return rs;
+  if (!side) return launch_tc(second, st);
   if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
-  rs = run_skinny_tc_pair(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, side->s);
+  rs = launch_tc(second, side->s);
   if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return rs;
+}
+
+static qlora_status linear_bwd_entry(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
+                                     const void *A, const void *B, int32_t r, float s, const void *u_saved,
+                                     bool want_saved, void *dx, void *dA, void *dB, void *ws, size_t ws_bytes,
+                                     void *stream) {
+  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
+  if (cs != QLORA_OK) return cs;
+  if ((T > 0 && (!dy || !dx || (want_saved && !u_saved))) || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(dx) || !aligned16(dA) || !aligned16(dB) || !aligned16(u_saved))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = qw->rows, K = qw->cols;
+  if (!ws_ok(ws, ws_bytes, QLORA_OP_BWD, T, N, K, r)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    // no tokens: the adapter gradients are empty sums
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  return linear_bwd_impl(dy, x, T, qw, A, B, r, s, want_saved ? u_saved : nullptr, dx, dA, dB, ws, st);
+}
+
+qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A, const void *B,
+                              int32_t r, float s, void *y, void *ws, size_t ws_bytes, void *stream) {
+  qlora_status cs = check_fwd(x, T, qw, A, B, r, s, y, nullptr, false);
+  if (cs != QLORA_OK) return cs;
+  if (!ws_ok(ws, ws_bytes, QLORA_OP_FWD, T, qw->rows, qw->cols, r)) return QLORA_ERR_WORKSPACE;
+  if (T == 0) return QLORA_OK;
+  return linear_fwd_impl(x, T, qw, A, B, r, s, y, nullptr, ws, static_cast<cudaStream_t>(stream));
+}
+
+size_t qlora_saved_u_bytes(int64_t T, int32_t r) {
+  if (T < 0 || r < 1 || r > 128) return 0;
+  return 2 * saved_plane_bytes(T, r);
+}
+
+qlora_status qlora_linear_fwd_save(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                                   const void *B, int32_t r, float s, void *y, void *u_save, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  qlora_status cs = check_fwd(x, T, qw, A, B, r, s, y, u_save, true);
+  if (cs != QLORA_OK) return cs;
+  if (!ws_ok(ws, ws_bytes, QLORA_OP_FWD, T, qw->rows, qw->cols, r)) return QLORA_ERR_WORKSPACE;
+  if (T == 0) return QLORA_OK;
+  return linear_fwd_impl(x, T, qw, A, B, r, s, y, u_save, ws, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                              const void *B, int32_t r, float s, void *dx, void *dA, void *dB, void *ws,
+                              size_t ws_bytes, void *stream) {
+  return linear_bwd_entry(dy, x, T, qw, A, B, r, s, nullptr, false, dx, dA, dB, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_saved(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
+                                    const void *A, const void *B, int32_t r, float s, const void *u_saved, void *dx,
+                                    void *dA, void *dB, void *ws, size_t ws_bytes, void *stream) {
+  return linear_bwd_entry(dy, x, T, qw, A, B, r, s, u_saved, true, dx, dA, dB, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -806,33 +967,160 @@ qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const ql
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// A process-unique id of the current context (0 if the driver cannot say):
+// a context created after cudaDeviceReset gets a new id.
+static unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 static void *noalloc_scratch_ptr() {
-  // the symbol's device address, looked up once per device with that device current
+  // the symbol's device address, looked up once per device and context with
+  // that device current (again after the context was reset)
   static void *ptrs[64] = {nullptr};
+  static unsigned long long ctx_ids[64] = {0};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
+  const unsigned long long id = current_ctx_id();
+  if (!ptrs[dev] || id == 0 || id != ctx_ids[dev]) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
     ptrs[dev] = p;
+    ctx_ids[dev] = id;
   }
   return ptrs[dev];
 }
 
 qlora_status qlora_linear_fwd_noalloc(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
                                       const void *B, int32_t r, float s, void *y, void *stream) {
-  qlora_status cs = check_linear(x, T, qw, A, B, r, s);
+  qlora_status cs = check_fwd(x, T, qw, A, B, r, s, y, nullptr, false);
   if (cs != QLORA_OK) return cs;
   const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, T, qw->rows, qw->cols, r);
   if (need == 0 || need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_WORKSPACE;
+  if (T == 0) return QLORA_OK;
   void *ws = noalloc_scratch_ptr();
   if (!ws) return QLORA_ERR_CUDA;
-  // the status word and the split counters must start at zero
+  // the split counters must start at zero (a call stopped by a timeout may have
+  // left some set); the status word keeps what earlier calls recorded until
+  // qlora_noalloc_get_error reads it
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + kWsCounterBytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  return qlora_linear_fwd(x, T, qw, A, B, r, s, y, ws, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+  if (cudaMemsetAsync(static_cast<uint8_t *>(ws) + kWsHeaderBytes, 0, kWsCounterBytes, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return linear_fwd_impl(x, T, qw, A, B, r, s, y, nullptr, ws, st);
+}
+
+qlora_status qlora_noalloc_get_error(void *stream) {
+  void *ws = noalloc_scratch_ptr();
+  if (!ws) return QLORA_ERR_CUDA;
+  return qlora_get_error(ws, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Failure-detection self-test: one thread waits, with the same bounded wait
+// every pipeline of the library uses, on an mbarrier that no thread arrives on.
+// The wait gives up after limit_ns and records DEV_TIMEOUT in the status word.
+// ---------------------------------------------------------------------------
+static __global__ void wait_selftest_kernel(uint32_t *status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // parity 0 of a fresh barrier completes only after one arrival, which never comes
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, status, limit_ns);
+  __syncthreads();
+}
+
+qlora_status qlora_wait_selftest(void *ws, size_t ws_bytes, uint32_t limit_us, void *stream) {
+  if (ws && (ws_bytes < kWsHeaderBytes || (reinterpret_cast<uintptr_t>(ws) & 255u))) return QLORA_ERR_WORKSPACE;
+  if (limit_us == 0 || limit_us > 2000000u) return QLORA_ERR_INVALID_ARG;
+  if (!ws) ws = noalloc_scratch_ptr();   // the allocation-free forward's status word
+  if (!ws) return QLORA_ERR_CUDA;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t *>(ws),
+                                                                        1000ull * limit_us);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// The adapters' optimizer step and its unified-memory ("paged") state
+// ---------------------------------------------------------------------------
+qlora_status qlora_adam_step(float *param, float *m, float *v, const void *grad_bf16, void *param_bf16, int64_t n,
+                             const qlora_adam_hparams *h, void *stream) {
+  if (!h || n < 0) return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (!param || !m || !v || !grad_bf16) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(param) || !aligned16(m) || !aligned16(v) || !aligned16(grad_bf16) || !aligned16(param_bf16))
+    return QLORA_ERR_MISALIGNED;
+  if (h->step < 1 || !isfinite(h->lr) || !isfinite(h->eps) || !isfinite(h->weight_decay) || !(h->eps > 0.f) ||
+      !(h->beta1 >= 0.f && h->beta1 < 1.f) || !(h->beta2 >= 0.f && h->beta2 < 1.f))
+    return QLORA_ERR_INVALID_ARG;
+  AdamArgs a;
+  a.lr = h->lr;
+  a.beta1 = h->beta1;
+  a.beta2 = h->beta2;
+  a.one_minus_beta1 = static_cast<float>(1.0 - static_cast<double>(h->beta1));
+  a.one_minus_beta2 = static_cast<float>(1.0 - static_cast<double>(h->beta2));
+  a.eps = h->eps;
+  a.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * h->weight_decay);
+  a.bc1 = static_cast<float>(1.0 - pow(static_cast<double>(h->beta1), h->step));
+  a.bc2 = static_cast<float>(1.0 - pow(static_cast<double>(h->beta2), h->step));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  TraceScope ts(K_ADAM, 0.0, 28.0 * n - (param_bf16 ? 0.0 : 2.0 * n), st);
+  return launch_adam(param, m, v, static_cast<const uint16_t *>(grad_bf16), static_cast<uint16_t *>(param_bf16), n,
+                     a, st, num_sms_current()) == cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_alloc(size_t bytes, void **ptr) {
+  if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  void *p = nullptr;
+  if (cudaMallocManaged(&p, bytes, cudaMemAttachGlobal) != cudaSuccess) return QLORA_ERR_CUDA;
+  // live on this GPU while there is room; the driver pages out under pressure
+  (void)cudaMemAdvise(p, bytes, cudaMemAdviseSetPreferredLocation, dev);
+  (void)cudaGetLastError();
+  *ptr = p;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_free(void *ptr) {
+  if (!ptr) return QLORA_OK;
+  return cudaFree(ptr) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_prefetch(void *ptr, size_t bytes, int32_t to_host, void *stream) {
+  if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (!to_host && cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  return cudaMemPrefetchAsync(ptr, bytes, to_host ? cudaCpuDeviceId : dev, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
 }
 
 qlora_status qlora_trace_attach(qlora_trace_rec *recs, int32_t capacity, int32_t *count) {

@@ -104,12 +104,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, for at most
-// kWaitLimitNs.  Returns false (and records DEV_TIMEOUT) if it never does.
+// Wait for the phase with the given parity to complete, for at most limit_ns
+// (kWaitLimitNs unless a caller asks for less).  Returns false (and records
+// DEV_TIMEOUT) if it never does.
 // Waiting threads are suspended between probes (try_wait's time hint) and
 // read the global timer only every 64 probes, so that long waits (the
 // epilogue waiting for a whole tile) take few issue slots.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
@@ -118,7 +120,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
       const uint64_t now = globaltimer();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
+      } else if (now - t0 > limit_ns) {
         set_status(status, DEV_TIMEOUT);
         return false;
       }

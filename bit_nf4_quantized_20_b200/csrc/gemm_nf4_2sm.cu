@@ -4,6 +4,10 @@
 //   forward   Y[T, N]  = X[T, K] W'[N, K]^T + (s X A^T)[T, r] B[N, r]^T
 //   backward  dX[T, K] = dY[T, N] W'[N, K] + (s dY B)[T, r] A[r, K]
 //
+// The rank-r operand (s X A^T, or s dY B) arrives as two BF16 planes, hi and
+// lo = bf16(v - hi), each as its own run of 64-wide stages against the same
+// B (or A) rows, so the rank-r term carries about 16 significant bits of it.
+//
 // ("QLoRA: Efficient Fine-Tuning", Step 3 eq. 3 and Step 4; W' is produced in
 // shared memory by dequantization warps, "converted to BF16 on the fly for each
 // matrix multiplication", "What is QLoRA?".)
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(sm.full(s), ph, p.status)) { ok = false; break; }
           tc_fence_after();
           int nk = 4;
-          if (ks >= p.k_main) nk = min(4, (p.r - (ks - p.k_main) * BK + 15) / 16);
+          if (ks >= p.k_main) nk = min(4, (p.r - ((ks - p.k_main) % p.k_lora_plane) * BK + 15) / 16);
           for (int kk = 0; kk < nk; ++kk) {
             const uint64_t adesc = !bwd ? smem_desc_sw128(sm.a(s) + kk * 32, 16, 1024)        // K-major
                                         : smem_desc_sw128(sm.a(s) + kk * 4096, 1024, 2048);   // MN-major
@@ -242,7 +246,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (p.sym) dequant_row<true>(cb, buf, row_addr, phase);
           else dequant_row<false>(cb, buf, row_addr, phase);
         } else {
-          const int l = ks - p.k_main;
+          // rank-r stage: the same B (forward) or A (backward) rows for the hi
+          // and the lo plane of sU / dU
+          const int l = (ks - p.k_main) % p.k_lora_plane;
           if (!bwd) {
             const int64_t n = row0 + tid;
             const int nv = (n < p.N) ? max(0, min(BK, p.r - l * BK)) : 0;

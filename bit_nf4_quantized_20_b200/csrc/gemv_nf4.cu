@@ -2,7 +2,10 @@
 // HBM bandwidth on the 4.127-bit weights ("What is QLoRA?": NF4 converted to
 // BF16 on the fly for each matrix multiplication):
 //
-//   Y[T, N] = X[T, K] W'[N, K]^T + U'[T, r] B[N, r]^T,   U' = BF16(s X A^T)
+//   Y[T, N] = X[T, K] W'[N, K]^T + U'[T, r] B[N, r]^T,   U' = s X A^T
+//
+// (U' as two BF16 planes, hi = bf16(v) and lo = bf16(v - hi), whose products
+// with B are added as two MMA chains: the rank-r term keeps ~16 bits of U'.)
 //
 // Each lane dequantizes whole 64-weight blocks straight into mma.sync A
 // fragments (no shared-memory tiles): the MMA's M is 16 weight rows and its N
@@ -38,6 +41,7 @@
 // in rank 0's shared memory.
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -100,12 +104,14 @@ __device__ __forceinline__ uint32_t ldg_pair_bf16(const uint16_t *p, int64_t i0,
 // tokens, a second MMA for tokens 8-15).  Accumulator: c0/c1 = (row r0, tokens
 // 2t, 2t + 1), c2/c3 = (row r0 + 8, tokens 2t, 2t + 1).
 
-// rank-r term for 16-row tile `tile`: v += B U'^T (k16-steps over r)
+// rank-r term for 16-row tile `tile`: v += B U'^T (k16-steps over r), once
+// with U''s hi plane and once with its lo plane (columns ldu / 2 on)
 template <int TT>
 __device__ __forceinline__ void gemv_lora(const GemvParams &p, int64_t tile, int g, int t, float (&v)[TT / 8][4]) {
   const int64_t r0 = tile * 16 + g, r1 = r0 + 8;
   const bool v0 = r0 < p.N, v1 = r1 < p.N;
   const int rv = p.r;
+  const int64_t lo_off = p.ldu / 2;
   for (int j0 = 0; j0 < rv; j0 += 16) {
     const int ja = j0 + 2 * t, jb = j0 + 2 * t + 8;
     const uint32_t a0 = ldg_pair_bf16(p.B, r0 * rv + ja, r0 * rv + ja + 1, v0 && ja < rv, v0 && ja + 1 < rv);
@@ -115,13 +121,16 @@ __device__ __forceinline__ void gemv_lora(const GemvParams &p, int64_t tile, int
 #pragma unroll
     for (int h = 0; h < TT / 8; ++h) {
       const int tok = 8 * h + g;
-      uint32_t b0 = 0u, b1 = 0u;
+      uint32_t b0 = 0u, b1 = 0u, l0 = 0u, l1 = 0u;
       if (tok < p.T) {
-        const uint16_t *ur = p.u + static_cast<int64_t>(tok) * p.ldu;   // zero-padded to ldu >= ceil16(r)
+        const uint16_t *ur = p.u + static_cast<int64_t>(tok) * p.ldu;   // each plane zero-padded past r
         b0 = *reinterpret_cast<const uint32_t *>(ur + ja);
         b1 = *reinterpret_cast<const uint32_t *>(ur + jb);
+        l0 = *reinterpret_cast<const uint32_t *>(ur + lo_off + ja);
+        l1 = *reinterpret_cast<const uint32_t *>(ur + lo_off + jb);
       }
       mma16816(v[h], a0, a1, a2, a3, b0, b1);
+      mma16816(v[h], a0, a1, a2, a3, l0, l1);
     }
   }
 }
@@ -366,7 +375,7 @@ constexpr int kPGD = 4;                            // units per warp ring (3 in 
 constexpr int kPStage = 2048 + 64 + 64;            // codes [16][128] swizzled, scale words [16], c2 [16]
 constexpr int kPRing = kPWarps * kPGD * kPStage;
 constexpr int kPSlotFloats = 16 * 16;              // one tile's sums: [T <= 16][16 rows]
-constexpr int kPUBytes = 16 * 128 * 2;             // U' [T <= 16][ldu <= 128] BF16
+constexpr int kPUBytes = 16 * 256 * 2;             // U' [T <= 16][ldu <= 256] BF16 (hi and lo planes)
 constexpr int kPSmem = kPRing + kPWarps * 2 * kPSlotFloats * 4 + kPWarps * 2 * 4 + kPUBytes;
 constexpr int kPCtasPerSm = QLORA_PERSIST_CTAS_PER_SM;
 
@@ -657,10 +666,10 @@ __global__ void __launch_bounds__(kPThreads, 2) nf4_gemv_persist_kernel(const Ge
 }
 
 // ---------------------------------------------------------------------------
-// U' = BF16(s X A^T) for T <= 16 tokens.  Grid: 8 x (ldu / 16) CTAs in clusters
-// of 8; cluster c owns columns 16c .. 16c + 15 of U' (A rows past r arrive as
-// zeros, so the padding columns come out zero), rank k owns the k-th slice of
-// the contraction.  Four warps split the slice; each runs mma.sync with
+// U' = s X A^T for T <= 16 tokens, as BF16 hi and lo planes.  Grid:
+// 8 x (plane / 16) CTAs in clusters of 8; cluster c owns columns 16c .. 16c + 15
+// of each plane (A rows past r arrive as zeros, so the padding columns come
+// out zero), rank k owns the k-th slice of the contraction.  Four warps split the slice; each runs mma.sync with
 // A = X [tokens][k] and B = A^T.
 // ---------------------------------------------------------------------------
 constexpr int kUCluster = 8;
@@ -746,14 +755,19 @@ __global__ void __launch_bounds__(kUThreads, 1) lora_u_decode_kernel(const LoraU
                      : "memory");
         v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
       }
-      // fragment: (token g, columns 2t, 2t+1) and (token g + 8, ...)
+      // fragment: (token g, columns 2t, 2t+1) and (token g + 8, ...); the hi
+      // plane, then the lo plane p.plane columns on
       const int64_t col = static_cast<int64_t>(cg) * 16 + nt * 8 + 2 * t;
-      if (g < p.T)
-        *reinterpret_cast<__nv_bfloat162 *>(p.u + static_cast<int64_t>(g) * p.ldu + col) =
-            __floats2bfloat162_rn(p.alpha * v.x, p.alpha * v.y);
-      if (TT == 16 && g + 8 < p.T)
-        *reinterpret_cast<__nv_bfloat162 *>(p.u + static_cast<int64_t>(g + 8) * p.ldu + col) =
-            __floats2bfloat162_rn(p.alpha * v.z, p.alpha * v.w);
+      auto put = [&](int tok, float a, float b) {
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(p.alpha * a, p.alpha * b);
+        const __nv_bfloat162 lo =
+            __floats2bfloat162_rn(p.alpha * a - __low2float(hi), p.alpha * b - __high2float(hi));
+        uint16_t *row = p.u + static_cast<int64_t>(tok) * p.ldu;
+        *reinterpret_cast<__nv_bfloat162 *>(row + col) = hi;
+        *reinterpret_cast<__nv_bfloat162 *>(row + p.plane + col) = lo;
+      };
+      if (g < p.T) put(g, v.x, v.y);
+      if (TT == 16 && g + 8 < p.T) put(g + 8, v.z, v.w);
     }
   }
   cluster_arrive_wait();   // the peers keep their shared memory until rank 0 has read it
@@ -766,22 +780,22 @@ namespace {
 // CTAs of `splits` warps that one SM holds at once (cached per kernel and split count)
 template <int TT, bool SYM>
 int gemv_occupancy(int splits) {
-  static int occ[kGemvMaxWarps + 1] = {0};
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(nf4_gemv_kernel<TT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemv_smem_bytes(kGemvMaxWarps)) != cudaSuccess)
-      return -1;
-    attr_set = true;
-  }
-  if (occ[splits] == 0) {
+  static std::atomic<int> occ[64][kGemvMaxWarps + 1];   // per device; 0 = not yet known
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (ensure_smem_optin(reinterpret_cast<const void *>(nf4_gemv_kernel<TT, SYM>), gemv_smem_bytes(kGemvMaxWarps)) !=
+      cudaSuccess)
+    return -1;
+  int known = occ[dev][splits].load(std::memory_order_relaxed);
+  if (known == 0) {
     int o = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, nf4_gemv_kernel<TT, SYM>, 32 * splits,
                                                       gemv_smem_bytes(splits)) != cudaSuccess)
       return -1;
-    occ[splits] = o > 0 ? o : -1;
+    known = o > 0 ? o : -1;
+    occ[dev][splits].store(known, std::memory_order_relaxed);
   }
-  return occ[splits];
+  return known;
 }
 
 // The most k-splits per 16-row tile whose grid still fits in one wave (all
@@ -836,15 +850,10 @@ int lora_u_decode_smem_bytes(int64_t K, int T) {
 namespace {
 template <int TT>
 cudaError_t launch_u(const LoraUDecodeParams &p, int smem, cudaStream_t st, bool pdl) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(lora_u_decode_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kLoraUDecodeMaxSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(lora_u_decode_kernel<TT>), kLoraUDecodeMaxSmem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(kUCluster * (p.ldu / 16)), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(kUCluster * (p.plane / 16)), 1, 1);
   cfg.blockDim = dim3(kUThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
@@ -863,7 +872,8 @@ cudaError_t launch_u(const LoraUDecodeParams &p, int smem, cudaStream_t st, bool
 
 cudaError_t launch_lora_u_decode(const LoraUDecodeParams &p_in, cudaStream_t st, bool pdl) {
   LoraUDecodeParams p = p_in;
-  if (p.T < 1 || p.T > 16 || p.r < 1 || p.ldu % 16 != 0 || p.ldu < p.r || p.K % 64 != 0)
+  if (p.T < 1 || p.T > 16 || p.r < 1 || p.plane % 16 != 0 || p.plane < p.r || p.ldu < 2 * p.plane ||
+      p.ldu % 8 != 0 || p.K % 64 != 0)
     return cudaErrorInvalidValue;
   p.kc = static_cast<int>(((p.K + kUCluster - 1) / kUCluster + 63) / 64 * 64);
   const int smem = lora_u_decode_smem_bytes(p.K, p.T);
@@ -889,13 +899,8 @@ size_t gemv_persist_partials_bytes(int64_t N, int64_t K, int max_tiles) {
 namespace {
 template <int TT, bool SYM>
 cudaError_t launch_persist(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(nf4_gemv_persist_kernel<TT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(nf4_gemv_persist_kernel<TT, SYM>), kPSmem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.ctas), 1, 1);
   cfg.blockDim = dim3(kPThreads, 1, 1);
@@ -919,7 +924,7 @@ cudaError_t launch_gemv(const GemvParams &p_in, int num_sms, cudaStream_t st, bo
     q.units = static_cast<int>(p.K / 256);
     q.tiles = static_cast<int>((p.N + 15) / 16);
     q.ctas = std::min(p.ctas, num_sms * kPCtasPerSm);
-    if (p.K % 256 != 0 || !q.part || !q.counters || p.ldu > 128 || p.ldu % 8 != 0) return cudaErrorInvalidValue;
+    if (p.K % 256 != 0 || !q.part || !q.counters || p.ldu > 256 || p.ldu % 8 != 0) return cudaErrorInvalidValue;
     if (q.sym) return t16 ? launch_persist<16, true>(q, num_sms, st, pdl) : launch_persist<8, true>(q, num_sms, st, pdl);
     return t16 ? launch_persist<16, false>(q, num_sms, st, pdl) : launch_persist<8, false>(q, num_sms, st, pdl);
   }

@@ -26,13 +26,29 @@ struct SnapTable {
 cudaError_t launch_merge(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t N, int64_t K,
                          const float (&codebook)[16], const uint16_t *A, const uint16_t *B, int r, float s,
                          uint16_t *out, cudaStream_t st, int num_sms);
+// snap_dq: codes snapped against the double-quantized scale s_b instead of c1
 cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
-                            const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms);
+                            const SnapTable &tab, bool snap_dq, uint32_t *status, cudaStream_t st, int num_sms);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scales, const float *c2, int64_t n_weights,
                               const float (&codebook)[16], uint16_t *out, cudaStream_t st, int num_sms);
 
+// Opt `func` in to `bytes` of dynamic shared memory on the current device, once
+// per (function, device); thread-safe (api.cu).
+cudaError_t ensure_smem_optin(const void *func, int bytes);
+
 // ---------------------------------------------------------------------------
-// fused NF4 GEMM (gemm_nf4.cu)
+// the adapters' optimizer step (optim.cu): Adam with decoupled weight decay
+// ---------------------------------------------------------------------------
+struct AdamArgs {
+  float lr, beta1, beta2, one_minus_beta1, one_minus_beta2, eps;
+  float decay;      // 1 - lr * weight_decay
+  float bc1, bc2;   // 1 - beta1^step, 1 - beta2^step
+};
+cudaError_t launch_adam(float *param, float *m, float *v, const uint16_t *grad, uint16_t *out_bf16, int64_t n,
+                        const AdamArgs &a, cudaStream_t st, int num_sms);
+
+// ---------------------------------------------------------------------------
+// fused NF4 GEMM on CTA pairs (gemm_nf4_2sm.cu)
 // ---------------------------------------------------------------------------
 struct GemmParams {
   const uint8_t *codes;
@@ -44,22 +60,19 @@ struct GemmParams {
   int mode;                // 0: forward (M side = N rows), 1: backward dX (M side = K columns)
   const uint16_t *lora;    // forward: B[N, r]; backward: A[r, K]
   int r;
-  int m_tiles, n_tiles;    // weight-side tiles of 128, token tiles of 256
-  int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part
+  int m_tiles, n_tiles;    // weight-side tiles of 256 (one CTA pair), token tiles of 256
+  int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part (hi then lo plane)
+  int k_lora_plane;        // rank-r stages per plane (k_lora = 2 k_lora_plane)
   int sym;                 // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   uint32_t *status;
-  uint16_t *out;           // CTA-pair variant: Y [T, N] or dX [T, K], stored from registers
+  uint16_t *out;           // Y [T, N] or dX [T, K], stored from registers
   int64_t ldo;             // its row stride (N or K)
 };
-int gemm_smem_bytes();
 int gemm_2sm_smem_bytes();
-// CTA-pair variant: m_tiles counts 256-row weight tiles; launched as clusters of 2.
+// launched as clusters of 2 CTAs
 __global__ void nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                     const __grid_constant__ CUtensorMap tmap_lact,
                                     const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
-__global__ void nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_act,
-                                const __grid_constant__ CUtensorMap tmap_lact,
-                                const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
 
 // ---------------------------------------------------------------------------
 // decode-sized forward, T <= 16 (gemv_nf4.cu)
@@ -72,7 +85,7 @@ struct GemvParams {
   int64_t N, K;
   int T;
   const uint16_t *x;     // [T, K]
-  const uint16_t *u;     // U' = BF16(s X A^T), [T, ldu]
+  const uint16_t *u;     // U' = s X A^T as BF16 hi + lo: row t = [hi (ldu/2 cols), lo (ldu/2 cols)]
   int64_t ldu;
   const uint16_t *B;     // [N, r]
   int r;
@@ -102,12 +115,14 @@ size_t gemv_persist_partials_bytes(int64_t N, int64_t K, int max_tiles);
 // launches the persistent kernel when p.ctas > 0, else the per-tile kernel
 cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl);
 
-// U' = BF16(alpha X A^T) [T, ldu] for T <= 16 (gemv_nf4.cu); columns r .. ldu - 1 are written as zero.
+// U' = alpha X A^T for T <= 16 (gemv_nf4.cu) as two BF16 planes in each row of
+// u [T, ldu]: hi = bf16(v) in columns 0 .. plane - 1, lo = bf16(v - hi) in
+// columns plane .. 2 plane - 1; columns r .. plane - 1 of each are written as zero.
 struct LoraUDecodeParams {
   const uint16_t *x;     // [T, K]
   const uint16_t *A;     // [r, K]
-  uint16_t *u;           // [T, ldu], ldu a multiple of 16
-  int64_t K, ldu;
+  uint16_t *u;           // [T, ldu], ldu >= 2 plane
+  int64_t K, ldu, plane; // plane a multiple of 16, >= r
   int T, r;
   int kc;                // contraction per CTA (set by the launcher)
   float alpha;
@@ -141,6 +156,7 @@ struct SkinnyParams {
   uint16_t *out0;      // OUT_HILO: hi plane; else output
   uint16_t *out1;      // OUT_HILO: lo plane
   int64_t ldo;         // OUT_HILO: plane row stride (>= R); unused otherwise
+  int64_t ocols;       // OUT_HILO: columns written per row of each plane (R .. ocols - 1 zero)
   float *partials;     // [splits][M][RP] when splits > 1
   uint32_t *counters;  // one per 64-row tile when splits > 1 (zero on entry, zero on exit)
   uint32_t *status;
@@ -169,8 +185,9 @@ struct SkinnyTcArgs {
   int64_t c_per_split;
   float alpha;
   // outputs (nullptr = not written); v = alpha * C[m, j]
-  uint16_t *row_hi;      // [M, ldo] bf16(v), columns R..ldo-1 zero
-  int64_t ldo;
+  uint16_t *row_hi;      // [M, ldo] bf16(v), columns R..ocols-1 zero
+  uint16_t *row_lo;      // [M, ldo] bf16(v - bf16(v)), columns R..ocols-1 zero (optional)
+  int64_t ldo, ocols;    // row stride; columns written per row (ocols <= ldo)
   uint16_t *t_hi;        // [R, ldt] bf16(v) transposed
   uint16_t *t_lo;        // [R, ldt] bf16(v - bf16(v)) transposed
   int64_t ldt;
@@ -184,9 +201,10 @@ cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, con
                              const CUtensorMap &tm_q1, cudaStream_t st, bool pdl);
 // Two independent products sharing one grid and one tile width (the larger of
 // the two), the CTA slots of one wave shared in proportion to their bytes.  Both
-// have R columns and nq Q planes; each has its own partials and counters.
-void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int64_t M1, int64_t C1, bool q_cj1, int R, int nq,
-                         int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1);
+// have R columns; each has its own Q plane count (nq0, nq1), pipeline depth,
+// partials and counters.
+void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
+                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1);
 // maps: {P, Q0, Q1} for each product
 cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
                                   const CUtensorMap *maps1, cudaStream_t st, bool pdl);

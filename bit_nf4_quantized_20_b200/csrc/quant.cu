@@ -20,6 +20,11 @@
 // has at most 25 significant bits and c1 8, so the product is exact in double.
 // Each block turns its 15 thresholds into the smallest BF16 weights that reach
 // them, B_j, and code = #{ j : w >= B_j } by the same 4-step search.
+//
+// Variant (snap_dq): the block is normalised by the scale it is dequantized
+// with, s_b = RN32(fp8(f_b) * c2_g), instead of c1_b (w_hat = 0 where s_b = 0).
+// s_b has at most 24 significant bits, so mid_j * s_b (<= 49 bits) is still
+// exact in double and the same boundary construction applies.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -61,7 +66,7 @@ __device__ __forceinline__ float snap_boundary(float c1, double mid, bool incl) 
 __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ w, int64_t n_blocks,
                                                       uint32_t *__restrict__ codes, uint8_t *__restrict__ scales,
                                                       float *__restrict__ c2, const SnapTable tab,
-                                                      uint32_t *status) {
+                                                      int snap_dq, uint32_t *status) {
   __shared__ float s_bnd[256 * 16];   // per block of the group: B_0 .. B_14
   __shared__ float s_wmax[QT / 32];
 
@@ -110,9 +115,18 @@ __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ 
 
   const float c2v = __fdiv_rn(gmax, 448.0f);
   if (tid == 0) c2[g] = c2v;
+  // each block's scale byte, and the divisor its codes are snapped against
+  uint32_t fb[8];
+  float dv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    fb[i] = c2v > 0.f ? float_to_e4m3(__fdiv_rn(c1[i], c2v)) : 0u;
+    dv[i] = snap_dq ? __fmul_rn(e4m3_to_float(fb[i]), c2v) : c1[i];
+  }
 
   // the block's boundaries: lane `sub` of its 8 lanes forms B_sub and B_{sub + 8}
-  // (an all-zero block gets boundaries that give every weight the code of 0)
+  // (a block whose divisor is zero gets boundaries that give every weight the
+  // code of 0)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int bl = i * 32 + bw;
@@ -121,7 +135,7 @@ __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ 
       const int j = sub + 8 * h;
       if (j < 15) {
         float bj;
-        if (c1[i] > 0.f) bj = snap_boundary(c1[i], tab.mid[j], ((tab.incl >> j) & 1u) != 0u);
+        if (dv[i] > 0.f) bj = snap_boundary(dv[i], tab.mid[j], ((tab.incl >> j) & 1u) != 0u);
         else bj = j < static_cast<int>(tab.snap0) ? -INFINITY : INFINITY;
         s_bnd[bl * 16 + j] = bj;
       }
@@ -133,7 +147,7 @@ __global__ void __launch_bounds__(QT) quantize_kernel(const uint4 *__restrict__ 
   for (int i = 0; i < 8; ++i) {
     const int bl = i * 32 + bw;
     if (bl < nb) {
-      if (sub == 0) scales[b0 + bl] = static_cast<uint8_t>(c2v > 0.f ? float_to_e4m3(__fdiv_rn(c1[i], c2v)) : 0u);
+      if (sub == 0) scales[b0 + bl] = static_cast<uint8_t>(fb[i]);
       const uint32_t hw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       const float *bnd = s_bnd + bl * 16;
       const float b3 = bnd[3], b7 = bnd[7], b11 = bnd[11];
@@ -246,13 +260,13 @@ cudaError_t launch_merge(const uint8_t *codes, const uint8_t *scales, const floa
 }
 
 cudaError_t launch_quantize(const uint16_t *w, int64_t n_blocks, uint8_t *codes, uint8_t *scales, float *c2,
-                            const SnapTable &tab, uint32_t *status, cudaStream_t st, int num_sms) {
+                            const SnapTable &tab, bool snap_dq, uint32_t *status, cudaStream_t st, int num_sms) {
   (void)num_sms;
   const int64_t groups = (n_blocks + 255) / 256;
   if (groups <= 0) return cudaSuccess;
   quantize_kernel<<<static_cast<unsigned>(groups), QT, 0, st>>>(reinterpret_cast<const uint4 *>(w), n_blocks,
                                                                  reinterpret_cast<uint32_t *>(codes), scales, c2,
-                                                                 tab, status);
+                                                                 tab, snap_dq ? 1 : 0, status);
   return cudaGetLastError();
 }
 

@@ -246,9 +246,9 @@ __global__ void __launch_bounds__(ST) skinny_kernel(const SkinnyParams p, int ou
 
   // write-out
   if (out_mode == OUT_HILO) {
-    const int ldo = static_cast<int>(p.ldo);
-    for (int idx = tid; idx < rows * ldo; idx += ST) {
-      const int row = idx / ldo, col = idx % ldo;
+    const int ocols = static_cast<int>(p.ocols);
+    for (int idx = tid; idx < rows * ocols; idx += ST) {
+      const int row = idx / ocols, col = idx % ocols;
       const float v = (col < p.R && col < RP) ? p.alpha * acc_s[row * L::ACC_PITCH + col] : 0.f;
       const __nv_bfloat16 hi = __float2bfloat16_rn(v);
       const int64_t o = (m0 + row) * p.ldo + col;
@@ -277,12 +277,8 @@ template <bool PCOL, bool QCJ, bool TWOQ, int RP>
 cudaError_t launch_t(const SkinnyParams &p, int out_mode, int q_ncols, int q_vec, cudaStream_t st) {
   using L = Layout<PCOL, QCJ, TWOQ, RP>;
   auto kern = skinny_kernel<PCOL, QCJ, TWOQ, RP>;
-  static bool attr_set = false;   // once per instantiation (keeps calls capturable in CUDA graphs)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(kern), L::SMEM);
+  if (e != cudaSuccess) return e;
   const int64_t m_tiles = (p.M + SBM - 1) / SBM;
   dim3 grid(static_cast<unsigned>(m_tiles), static_cast<unsigned>(p.splits));
   kern<<<grid, ST, L::SMEM, st>>>(p, out_mode, q_ncols, q_vec);

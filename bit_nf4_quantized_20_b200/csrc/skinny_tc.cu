@@ -51,17 +51,21 @@ template <int CW>
 __device__ __forceinline__ void emit_chunk(const SkinnyTcArgs &a, int64_t m, int c0, const float (&v)[CW]) {
   if (a.row_hi) {
     uint16_t *h = a.row_hi + m * a.ldo + c0;
+    uint16_t *l = a.row_lo ? a.row_lo + m * a.ldo + c0 : nullptr;
 #pragma unroll
     for (int g = 0; g < CW; g += 8) {
-      uint32_t w[4];
+      uint32_t w[4], wl[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
         const float x0 = (c0 + g + e < a.R) ? a.alpha * v[g + e] : 0.f;
         const float x1 = (c0 + g + e + 1 < a.R) ? a.alpha * v[g + e + 1] : 0.f;
         const __nv_bfloat162 hh = __floats2bfloat162_rn(x0, x1);
         w[e / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(x0 - __low2float(hh), x1 - __high2float(hh));
+        wl[e / 2] = *reinterpret_cast<const uint32_t *>(&ll);
       }
       *reinterpret_cast<uint4 *>(h + g) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (l) *reinterpret_cast<uint4 *>(l + g) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
     }
   }
 #pragma unroll
@@ -288,10 +292,12 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
         if (m < a.M) emit_chunk<CW>(a, m, c0, v);
       }
     }
-    // the rest of a padded row of the hi plane (columns NB .. ldo - 1) is zero
+    // the rest of a padded row of the hi / lo planes (columns NB .. ocols - 1) is zero
     if (a.row_hi && m < a.M && (a.splits == 1 || s_last)) {
-      for (int64_t c = NB; c < a.ldo; c += 8)
+      for (int64_t c = NB; c < a.ocols; c += 8) {
         *reinterpret_cast<uint4 *>(a.row_hi + m * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
+        if (a.row_lo) *reinterpret_cast<uint4 *>(a.row_lo + m * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
 
@@ -399,11 +405,13 @@ SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int 
   return g;
 }
 
-void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int64_t M1, int64_t C1, bool q_cj1, int R, int nq,
-                         int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1) {
+void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
+                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1) {
   const int nb = tc_nb(R, q_cj0) > tc_nb(R, q_cj1) ? tc_nb(R, q_cj0) : tc_nb(R, q_cj1);
-  const int per_sm = tc_stages(nb, nq, g0);
-  tc_stages(nb, nq, g1);
+  const int per0 = tc_stages(nb, nq0, g0);
+  const int per1 = tc_stages(nb, nq1, g1);
+  // the grid is launched with the larger of the two shared-memory footprints
+  const int per_sm = per0 < per1 ? per0 : per1;
   if (num_sms <= 0) return;
   // one wave for both, the slots shared in proportion to the bytes each streams
   const int64_t slots = static_cast<int64_t>(per_sm) * num_sms;
@@ -424,13 +432,8 @@ namespace {
 template <int NB>
 cudaError_t launch_nb(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
                       const CUtensorMap &tm_q1, cudaStream_t st, bool pdl) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(skinny_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kOnePerSmBudget);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(skinny_tc_kernel<NB>), kOnePerSmBudget);
+  if (e != cudaSuccess) return e;
   const int stage = P_BYTES + a.nq * NB * TBK * 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((a.M + TBM - 1) / TBM), static_cast<unsigned>(a.splits), 1);
@@ -465,19 +468,15 @@ namespace {
 template <int NB>
 cudaError_t launch_pair_nb(const SkinnyTcArgs &a0, const CUtensorMap *m0, const SkinnyTcArgs &a1,
                            const CUtensorMap *m1, cudaStream_t st, bool pdl) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(skinny_tc_pair_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kOnePerSmBudget);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int stage = P_BYTES + a0.nq * NB * TBK * 2;
+  cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(skinny_tc_pair_kernel<NB>), kOnePerSmBudget);
+  if (e != cudaSuccess) return e;
+  const int smem0 = a0.stages * (P_BYTES + a0.nq * NB * TBK * 2) + kFixedSmem;
+  const int smem1 = a1.stages * (P_BYTES + a1.nq * NB * TBK * 2) + kFixedSmem;
   const int64_t n0 = (a0.M + TBM - 1) / TBM * a0.splits, n1 = (a1.M + TBM - 1) / TBM * a1.splits;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n0 + n1), 1, 1);
   cfg.blockDim = dim3(TNUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(a0.stages * stage + kFixedSmem);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem0 > smem1 ? smem0 : smem1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -491,9 +490,10 @@ cudaError_t launch_pair_nb(const SkinnyTcArgs &a0, const CUtensorMap *m0, const 
 cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
                                   const CUtensorMap *maps1, cudaStream_t st, bool pdl) {
   if (a0.M <= 0 || a0.C <= 0 || a1.M <= 0 || a1.C <= 0 || a0.R <= 0) return cudaErrorInvalidValue;
-  if (a0.nb != a1.nb || a0.nq != a1.nq || a0.stages != a1.stages) return cudaErrorInvalidValue;
-  if (a0.stages < 1 || a0.stages > TMAX_STAGES || a0.splits < 1 || a1.splits < 1 || (a0.nq != 1 && a0.nq != 2))
-    return cudaErrorInvalidValue;
+  if (a0.nb != a1.nb) return cudaErrorInvalidValue;
+  for (const SkinnyTcArgs *a : {&a0, &a1})
+    if (a->stages < 1 || a->stages > TMAX_STAGES || a->splits < 1 || (a->nq != 1 && a->nq != 2))
+      return cudaErrorInvalidValue;
   if ((a0.q_cj || a1.q_cj) && a0.nb < 64) return cudaErrorInvalidValue;
   switch (a0.nb) {
     case 16: return launch_pair_nb<16>(a0, maps0, a1, maps1, st, pdl);

@@ -20,14 +20,21 @@
  *     dequantization on the fly in every forward and backward pass.
  *
  * Conventions shared by every entry point:
- *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
- *     never allocates or frees device memory; its only device state is the
- *     fixed scratch array of qlora_linear_fwd_noalloc (a static symbol).
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller (device or
+ *     unified memory).  The library allocates and frees device memory only in
+ *     qlora_paged_alloc / qlora_paged_free, which a caller calls explicitly for
+ *     optimizer state; its only other device state is the fixed scratch array
+ *     of qlora_linear_fwd_noalloc (a static symbol).  Its host state is one
+ *     side stream per host thread and device (backward).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).  Work
  *     is enqueued on it and the call returns after validating the arguments;
  *     results are ready when the stream reaches that point.
  *   - Row-major layouts.  BF16 tensors are arrays of uint16 bit patterns.
- *   - A call that returns anything but QLORA_OK has enqueued nothing.
+ *   - Every check (arguments, alignment, workspace, TMA descriptor encoding)
+ *     runs before the first enqueue: a call that returns INVALID_ARG,
+ *     UNSUPPORTED, MISALIGNED or WORKSPACE has enqueued nothing.  CUDA means a
+ *     runtime call or a kernel launch failed; launches of the same call that
+ *     came before the failing one stay enqueued.
  *   - Device-side failures (a bounded wait that ran out, a non-finite weight)
  *     are recorded in the workspace's status word and read by qlora_get_error.
  *   - Not thread-safe with respect to the trace hook; otherwise re-entrant.
@@ -151,6 +158,22 @@ QLORA_API qlora_status qlora_quantize_nf4(const void *w_bf16, int64_t rows, int6
                                 void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * qlora_quantize_nf4 with options (flags, OR-ed; 0 is qlora_quantize_nf4):
+ *   QLORA_QUANT_SNAP_DQ_SCALE -- snap each block's codes against the scale it
+ *     is dequantized with, s_b = RN32(fp8(f_b) * c2), instead of the exact c1:
+ *     w_hat = RN32(w / s_b) (0 where s_b = 0), code = nearest level as above.
+ *     The pages do not say whether the codes come from c1 or from the
+ *     double-quantized scale ("QLoRA & 4-bit Fine-Tuning", Innovation 2 gives
+ *     quantization, then double quantization); snapping against s_b lowers
+ *     each weight's reconstruction error.  Scale bytes and c2 are unchanged.
+ * Errors: as qlora_quantize_nf4; INVALID_ARG for an unknown flag.
+ */
+#define QLORA_QUANT_SNAP_DQ_SCALE 1u
+QLORA_API qlora_status qlora_quantize_nf4_ex(const void *w_bf16, int64_t rows, int64_t cols, int32_t blocksize,
+                                             int32_t dq_block, const float codebook[16], uint32_t flags,
+                                             qlora_nf4_weight *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Dequantize to BF16: w_out[rows, cols] = W' as defined above ("What is
  * QLoRA?": NF4 converted to BF16 on the fly; prepfeed: W ~ c1 * W_NF4).
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
@@ -201,6 +224,41 @@ QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T
                               void *dB, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The LoRA activation saved for the backward ("QLoRA: Efficient Fine-Tuning",
+ * Step 4 eq. 5 takes x "cached from the forward pass"; here the cached value
+ * is its rank-r image U = s x A^T, which is all that dB needs of x).
+ * Layout, caller-owned device memory of qlora_saved_u_bytes(T, r) bytes,
+ * 16-byte aligned: two BF16 planes of sU^T [r, ceil8(T)] (row stride
+ * ceil8(T)), hi = bf16(v) at offset 0 and lo = bf16(v - hi) at offset
+ * qlora_saved_u_bytes(T, r) / 2, so that hi + lo carries about 16 significant
+ * bits of v = s (x A^T)[t, j].  Returns 0 on invalid arguments.
+ */
+QLORA_API size_t qlora_saved_u_bytes(int64_t T, int32_t r);
+
+/*
+ * qlora_linear_fwd that also writes U to u_save (layout above).  Same
+ * arguments, requirements and errors, plus u_save (INVALID_ARG if null when
+ * T > 0, MISALIGNED if not 16-byte aligned).  At T <= 16 the rank-r product
+ * then runs on the tensor-core kernel instead of the decode cluster kernel.
+ */
+QLORA_API qlora_status qlora_linear_fwd_save(const void *x, int64_t T, const qlora_nf4_weight *qw, const void *A,
+                                             const void *B, int32_t r, float s, void *y, void *u_save, void *ws,
+                                             size_t ws_bytes, void *stream);
+
+/*
+ * qlora_linear_bwd that takes U from a preceding qlora_linear_fwd_save of the
+ * same x, A, s and T instead of recomputing it from x: dU and dB then share one
+ * grid (both stream dY), and x is read once (for dA).  Results equal
+ * qlora_linear_bwd's within the rounding of the FP32 sums.  u_saved is read,
+ * never written.  Errors: as qlora_linear_bwd; INVALID_ARG if u_saved is null
+ * when T > 0, MISALIGNED if it is not 16-byte aligned.
+ */
+QLORA_API qlora_status qlora_linear_bwd_saved(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
+                                              const void *A, const void *B, int32_t r, float s, const void *u_saved,
+                                              void *dx, void *dA, void *dB, void *ws, size_t ws_bytes,
+                                              void *stream);
+
+/*
  * Forward without a caller-supplied workspace (no counterpart on the pages: a
  * deployment aid).  For callers that cannot allocate device memory: code that
  * runs under a host framework which owns every device allocation (a serving
@@ -216,19 +274,83 @@ QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T
  * 14336 x 4096 weight, but not at r = 64).
  *
  * The first call on a device looks up the array's device address on that
- * device (make it before any stream capture).  Every call zeroes the array's
- * status word and counters on `stream`, then reuses it; all calls share the
- * one array, so calls that may overlap on the GPU (different streams, or
+ * device (make it before any stream capture); the lookup is repeated after
+ * the device's context was replaced (cudaDeviceReset).  Every call zeroes the
+ * array's split counters on `stream`, then reuses the array; all calls share
+ * the one array, so calls that may overlap on the GPU (different streams, or
  * concurrent host threads) race and must be serialized by the caller.
- * A device-side failure (a bounded wait that ran out) is recorded in the
- * array's status word, which the next call clears; this entry point has no
- * separate status query.
+ * All arguments are checked before anything is enqueued (T == 0 enqueues
+ * nothing).  A device-side failure (a bounded wait that ran out) is recorded
+ * in the array's status word and kept there until qlora_noalloc_get_error
+ * reads and clears it.
  * Errors: as qlora_linear_fwd; QLORA_ERR_WORKSPACE for sizes beyond the array.
  */
 #define QLORA_NOALLOC_SCRATCH_BYTES (4u << 20)
 QLORA_API qlora_status qlora_linear_fwd_noalloc(const void *x, int64_t T, const qlora_nf4_weight *qw,
                                                 const void *A, const void *B, int32_t r, float s, void *y,
                                                 void *stream);
+
+/*
+ * The status query of qlora_linear_fwd_noalloc on the current device:
+ * synchronize `stream`, read and clear the fixed array's status word.
+ * Returns QLORA_OK, QLORA_ERR_TIMEOUT or QLORA_ERR_CUDA (as qlora_get_error).
+ */
+QLORA_API qlora_status qlora_noalloc_get_error(void *stream);
+
+/*
+ * Failure-detection self-test (a diagnostic; the pages have no counterpart).
+ * Launches one kernel whose thread waits, with the bounded mbarrier wait that
+ * every pipeline of the library uses, on a barrier that nothing arrives on;
+ * after limit_us microseconds the wait gives up, records the timeout in the
+ * workspace's status word and the kernel returns.  qlora_get_error(ws, stream)
+ * then returns QLORA_ERR_TIMEOUT.  The kernels' own waits keep their 2 s
+ * limit.  limit_us in [1, 2000000]; ws: at least 256 bytes, 256-byte aligned,
+ * or NULL for the fixed array of qlora_linear_fwd_noalloc on the current device
+ * (then read with qlora_noalloc_get_error).
+ * Errors: WORKSPACE, INVALID_ARG, CUDA.
+ */
+QLORA_API qlora_status qlora_wait_selftest(void *ws, size_t ws_bytes, uint32_t limit_us, void *stream);
+
+/*
+ * The adapters' optimizer step ("What is QLoRA?", "The three pieces": paged
+ * optimizers; "Worked example: Llama 3.1 8B": adapters in fp32 with gradients
+ * and Adam moments).  Adam (Kingma & Ba, 2015) with decoupled weight decay
+ * (Loshchilov & Hutter, 2019), elementwise over n parameters:
+ *   p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *   p <- p - lr (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps)
+ * in FP32 (IEEE division and square root).  param, m, v: float[n], updated in
+ * place (device or unified memory, e.g. from qlora_paged_alloc); grad_bf16:
+ * BF16[n] (dA or dB of qlora_linear_bwd); param_bf16: BF16[n] output, the
+ * rounded new parameters for the next forward, or NULL.  All 16-byte aligned.
+ * step >= 1 counts the optimizer steps taken, this one included.
+ * Errors: INVALID_ARG (null buffer, step < 1, beta outside [0, 1), eps <= 0,
+ * non-finite lr or wd), MISALIGNED, CUDA.
+ */
+typedef struct {
+  float lr;
+  float beta1;          /* e.g. 0.9 */
+  float beta2;          /* e.g. 0.999 */
+  float eps;            /* e.g. 1e-8 */
+  float weight_decay;   /* decoupled; 0 for plain Adam */
+  int32_t step;
+} qlora_adam_hparams;
+QLORA_API qlora_status qlora_adam_step(float *param, float *m, float *v, const void *grad_bf16, void *param_bf16,
+                                       int64_t n, const qlora_adam_hparams *h, void *stream);
+
+/*
+ * Unified ("paged") memory for optimizer state ("QLoRA & 4-bit Fine-Tuning",
+ * Innovation 3: the state is paged out to host memory when the GPU runs short
+ * and back when it is needed).  qlora_paged_alloc: cudaMallocManaged of
+ * `bytes` with the current device as preferred location; *ptr is usable by
+ * every kernel of this library and by the host.  qlora_paged_free releases it
+ * (NULL is a no-op).  qlora_paged_prefetch moves `bytes` at ptr to the
+ * current device (to_host = 0) or to host memory (to_host != 0), ordered on
+ * `stream`; without it pages move on first touch.
+ * Errors: INVALID_ARG (null, zero bytes), CUDA.
+ */
+QLORA_API qlora_status qlora_paged_alloc(size_t bytes, void **ptr);
+QLORA_API qlora_status qlora_paged_free(void *ptr);
+QLORA_API qlora_status qlora_paged_prefetch(void *ptr, size_t bytes, int32_t to_host, void *stream);
 
 /*
  * Launch trace (profiling hook).  While attached, every kernel the library

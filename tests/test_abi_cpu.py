@@ -213,3 +213,78 @@ def test_product_fails_loudly_without_cuda():
     import bit_nf4_quantized_20_b200 as q
     with pytest.raises(ValueError):
         q.quantize_nf4(torch.zeros(64, 64, dtype=torch.bfloat16))
+
+
+def test_saved_u_validation(L):
+    """The saved-U forward and backward check their extra buffer before
+    touching the GPU; its size query follows the documented layout."""
+    w = _weight()
+    P = C.c_void_p(FAKE)
+    ws, big = C.c_void_p(FAKE), 1 << 30
+    # two planes of r x ceil8(T) BF16, each rounded up to 256 bytes
+    assert L.qlora_saved_u_bytes(4096, 16) == 2 * 16 * 4096 * 2
+    assert L.qlora_saved_u_bytes(5, 3) == 2 * 256
+    assert L.qlora_saved_u_bytes(0, 16) == 0
+    assert L.qlora_saved_u_bytes(16, 0) == 0 and L.qlora_saved_u_bytes(16, 129) == 0
+    fs = L.qlora_linear_fwd_save
+    assert fs(P, 16, C.byref(w), P, P, 8, 2.0, P, None, ws, big, None) == 1                   # no u_save
+    assert fs(P, 16, C.byref(w), P, P, 8, 2.0, P, C.c_void_p(FAKE + 8), ws, big, None) == 3   # misaligned
+    assert fs(P, 16, C.byref(w), P, P, 8, 2.0, P, P, ws, 64, None) == 4                       # workspace
+    assert fs(None, 0, C.byref(w), P, P, 8, 2.0, None, None, ws, big, None) == 0              # T == 0: no-op
+    bs = L.qlora_linear_bwd_saved
+    assert bs(P, P, 16, C.byref(w), P, P, 8, 2.0, None, P, P, P, ws, big, None) == 1
+    assert bs(P, P, 16, C.byref(w), P, P, 8, 2.0, C.c_void_p(FAKE + 2), P, P, P, ws, big, None) == 3
+    assert bs(P, P, 16, C.byref(w), P, P, 8, 2.0, P, P, P, P, ws, 64, None) == 4
+
+
+def test_noalloc_validation_before_any_enqueue(L):
+    """Bad outputs and oversized problems are refused by the allocation-free
+    forward before it looks up its scratch array or enqueues anything (so these
+    calls need no GPU)."""
+    w = _weight()
+    P = C.c_void_p(FAKE)
+    na = L.qlora_linear_fwd_noalloc
+    assert na(P, 16, C.byref(w), P, P, 8, 2.0, None, None) == 1                  # no output
+    assert na(P, 16, C.byref(w), P, P, 8, 2.0, C.c_void_p(FAKE + 4), None) == 3  # misaligned output
+    assert na(P, 16, C.byref(_weight(rows=100)), P, P, 8, 2.0, P, None) == 2      # N % 8
+    big = _weight(rows=14336, cols=4096)
+    assert na(P, 4096, C.byref(big), P, P, 64, 1.0, P, None) == 4                  # beyond the 4 MiB array
+    assert na(None, 0, C.byref(w), P, P, 8, 2.0, None, None) == 0                 # T == 0: no-op
+
+
+def test_wait_selftest_validation(L):
+    P = C.c_void_p(FAKE)
+    assert L.qlora_wait_selftest(C.c_void_p(FAKE + 16), 4096, 100, None) == 4   # not 256-byte aligned
+    assert L.qlora_wait_selftest(P, 64, 100, None) == 4
+    assert L.qlora_wait_selftest(P, 4096, 0, None) == 1
+    assert L.qlora_wait_selftest(P, 4096, 2000001, None) == 1
+    assert L.qlora_wait_selftest(None, 0, 0, None) == 1          # checked before the array's lookup
+
+
+def test_quantize_ex_flags_validation(L):
+    cb = (C.c_float * 16)(*[float(v) for v in O.nf4_codebook()])
+    out = _weight()
+    ws, wsb = C.c_void_p(FAKE), 1 << 20
+    qx = L.qlora_quantize_nf4_ex
+    assert qx(C.c_void_p(FAKE), 128, 128, 64, 256, cb, 2, C.byref(out), ws, wsb, None) == 1   # unknown flag
+    assert qx(C.c_void_p(FAKE), 128, 100, 64, 256, cb, 1, C.byref(out), ws, wsb, None) == 2   # cols % 64
+    assert qx(C.c_void_p(FAKE), 128, 128, 64, 256, cb, 1, C.byref(out), None, wsb, None) == 4
+
+
+def test_adam_and_paged_validation(L):
+    from bit_nf4_quantized_20_b200._lib import AdamHParams
+    P = C.c_void_p(FAKE)
+    h = AdamHParams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    a = L.qlora_adam_step
+    assert a(P, P, P, P, None, 0, C.byref(h), None) == 0              # nothing to do
+    assert a(P, P, P, P, None, 10, None, None) == 1                   # no hyper-parameters
+    assert a(None, P, P, P, None, 10, C.byref(h), None) == 1
+    assert a(P, P, P, C.c_void_p(FAKE + 2), None, 10, C.byref(h), None) == 3
+    assert a(P, P, P, P, C.c_void_p(FAKE + 8), 10, C.byref(h), None) == 3
+    for bad in (AdamHParams(1e-3, 0.9, 0.999, 1e-8, 0.0, 0), AdamHParams(1e-3, 1.0, 0.999, 1e-8, 0.0, 1),
+                AdamHParams(1e-3, 0.9, 0.999, 0.0, 0.0, 1), AdamHParams(float("nan"), 0.9, 0.999, 1e-8, 0.0, 1)):
+        assert a(P, P, P, P, None, 10, C.byref(bad), None) == 1
+    assert L.qlora_paged_alloc(0, C.byref(C.c_void_p())) == 1
+    assert L.qlora_paged_alloc(16, None) == 1
+    assert L.qlora_paged_free(None) == 0
+    assert L.qlora_paged_prefetch(None, 16, 0, None) == 1

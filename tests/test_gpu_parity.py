@@ -400,3 +400,290 @@ def test_layer_asymmetric_codebook(T, N, K, r, s):
     assert_close("dX", dx, rdx)
     assert_close("dA", dA, rdA)
     assert_close("dB", dB, rdB)
+
+
+# --------------------------------------------------------------------------
+# the forward that saves U and the backward that reuses it
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T,N,K,r,s", [
+    (16, 512, 512, 8, 2.0),       # the tiny layer; decode-sized forward with U saved
+    (1, 64, 64, 1, 1.0),          # one token, rank 1
+    (5, 1032, 768, 64, 1.0),      # decode-sized, ragged last row tile
+    (300, 384, 320, 24, 0.5),     # two token tiles (one ragged), ragged rank
+    (33, 256, 128, 128, 0.25),    # maximum rank
+    (257, 128, 256, 65, 1.0),     # rank just over one 64-wide stage
+    (7, 136, 192, 16, 2.0),       # N not a multiple of the weight tile
+])
+def test_layer_saved_u(T, N, K, r, s):
+    q = Q()
+    W, X, A, B, dY = inputs.layer_inputs(92, 0, 0, T, N, K, r, device="cuda")
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    y, u = q.linear_fwd_save(X, qw, A, B, s)
+    assert u.numel() == q.saved_u_bytes(T, r)
+    dx, dA, dB = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    assert_close("Y", y, O.linear_fwd(xb, wd, ab, bb, s))
+    rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    assert_close("dX", dx, rdx)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
+    # the saved planes hold sU = s X A^T as hi + lo: about 16 significant bits
+    Tp = (T + 7) // 8 * 8
+    plane = u.numel() // 2
+    hi = u[:r * Tp * 2].view(torch.bfloat16).float().reshape(r, Tp)
+    lo = u[plane:plane + r * Tp * 2].view(torch.bfloat16).float().reshape(r, Tp)
+    got = (hi + lo).double().cpu().numpy()[:, :T]
+    ref = float(s) * (O.bf16_bits_to_f32(xb).astype(np.float64) @ O.bf16_bits_to_f32(ab).astype(np.float64).T).T
+    assert np.all(np.abs(got - ref) <= 1e-3 + 2.0 ** -14 * np.abs(ref))
+
+
+def test_backward_saved_graph_capture_matches_eager():
+    """The saved-U backward also forks its second grid onto the side stream;
+    captured in a CUDA graph it gives the eager results bit for bit."""
+    q = Q()
+    T, N, K, r, s = 512, 1024, 768, 16, 2.0
+    W, X, A, B, dY = inputs.layer_inputs(94, 0, 0, T, N, K, r, device="cuda")
+    qw = q.quantize_nf4(W)
+    _, u = q.linear_fwd_save(X, qw, A, B, s)
+    ref = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
+    torch.cuda.synchronize()
+    outs = tuple(torch.empty_like(t) for t in ref)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        q.linear_bwd_saved(dY, X, qw, A, B, s, u, outs=outs)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for t in outs:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        q.linear_bwd_saved(dY, X, qw, A, B, s, u, outs=outs)
+    g.replay()
+    q.get_error()
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dX", "dA", "dB"), outs, ref):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), name
+    del g
+
+
+# --------------------------------------------------------------------------
+# failure detection and argument checks on a GPU
+# --------------------------------------------------------------------------
+def test_bounded_wait_runs_out_and_is_reported():
+    """A wait on a barrier that nothing arrives on gives up after its limit
+    (here 2 ms), the status word reports QLORA_ERR_TIMEOUT once, and the
+    context stays usable: a forward right after it is correct."""
+    import time
+    q = Q()
+    q.get_error()                              # start clean
+    t0 = time.perf_counter()
+    q.wait_selftest(2000)
+    with pytest.raises(q.QLoraError) as e:
+        q.get_error()
+    assert e.value.status == 7                 # QLORA_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    q.get_error()                              # the word was cleared
+    check_layer(16, 512, 512, 8, 2.0, config=0)
+
+
+def test_wrong_output_buffers_are_refused_before_launch():
+    q = Q()
+    T, N, K, r = 32, 256, 128, 8
+    W, X, A, B, dY = inputs.layer_inputs(96, 0, 0, T, N, K, r, device="cuda")
+    qw = q.quantize_nf4(W)
+    bad = [torch.empty(T, N + 8, dtype=torch.bfloat16, device="cuda"),   # too wide
+           torch.empty(T - 1, N, dtype=torch.bfloat16, device="cuda"),   # too short
+           torch.empty(T, N, dtype=torch.float32, device="cuda")]        # wrong dtype
+    for out in bad:
+        with pytest.raises(ValueError):
+            q.linear_fwd(X, qw, A, B, 1.0, out=out)
+        with pytest.raises(ValueError):
+            q.linear_fwd_noalloc(X, qw, A, B, 1.0, out)
+    with pytest.raises(ValueError):
+        q.linear_bwd(dY, X, qw, A, B, 1.0, outs=(torch.empty(T, K + 8, dtype=torch.bfloat16, device="cuda"),
+                                                torch.empty(r, K, dtype=torch.bfloat16, device="cuda"),
+                                                torch.empty(N, r, dtype=torch.bfloat16, device="cuda")))
+
+
+# --------------------------------------------------------------------------
+# codebook variants ("QLoRA & 4-bit Fine-Tuning", Innovations 1 and 2)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("table", ["eq2", "eq2_zero", "int4"])
+@pytest.mark.parametrize("rows,cols", [(512, 512), (17, 1024), (64, 64 * 257)])
+def test_quantize_snapped_to_dq_scale_bitexact(table, rows, cols):
+    """Codes snapped against the double-quantized block scale: codes, scale
+    bytes and c2 bit for bit against the oracle, special blocks included, and
+    the dequantization of those codes too."""
+    q = Q()
+    cb = {"eq2": O.nf4_codebook(), "eq2_zero": O.nf4_codebook_with_zero(),
+          "int4": np.array(INT4_LEVELS, np.float32)}[table]
+    w = _special_weight(rows, cols, 7 * rows + cols)
+    qw = q.quantize_nf4(w, codebook=[float(v) for v in cb], snap_to_dq_scale=True)
+    torch.cuda.synchronize()
+    codes, scales, c2 = O.quantize_nf4(bits(w), cb, snap_to_dq_scale=True)
+    assert np.array_equal(qw.c2.cpu().numpy().view(np.uint32), c2.view(np.uint32))
+    assert np.array_equal(qw.scales.cpu().numpy(), scales)
+    got = qw.codes.cpu().numpy()
+    assert np.array_equal(got, codes), f"{np.count_nonzero(got != codes)} code bytes differ"
+    wd = q.dequantize(qw)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(wd), O.dequantize_nf4(codes, scales, c2, rows, cols, cb))
+
+
+@pytest.mark.parametrize("T,N,K,r,s", [(300, 384, 320, 24, 0.5), (4, 1024, 4096, 64, 1.0), (16, 512, 512, 8, 2.0),
+                                       (2, 1032, 768, 16, 1.0)])
+def test_layer_codebook_with_zero_level(T, N, K, r, s):
+    """eq. 2 with an exact zero level through every kernel: quantize and
+    dequantize bit for bit, the tensor-core forward/backward (T > 16) or the
+    decode forward (T <= 16), the saved-U pair, and the adapter merge."""
+    q = Q()
+    cb = O.nf4_codebook_with_zero()
+    W, X, A, B, dY = inputs.layer_inputs(97, 0, 0, T, N, K, r, device="cuda")
+    qw = q.quantize_nf4(W, codebook=[float(v) for v in cb])
+    torch.cuda.synchronize()
+    codes, scales, c2 = O.quantize_nf4(bits(W), cb)
+    assert np.array_equal(qw.codes.cpu().numpy(), codes)
+    assert np.array_equal(qw.scales.cpu().numpy(), scales)
+    wd = O.dequantize_nf4(codes, scales, c2, N, K, cb)
+    assert np.array_equal(bits(q.dequantize(qw)), wd)
+    y = q.linear_fwd(X, qw, A, B, s)
+    y2, u = q.linear_fwd_save(X, qw, A, B, s)
+    dx, dA, dB = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
+    m = q.merge_adapter(qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    ref = O.linear_fwd(xb, wd, ab, bb, s)
+    assert_close("Y", y, ref)
+    assert_close("Y saved", y2, ref)
+    rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    assert_close("dX", dx, rdx)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
+    o = O.merge_adapter(wd, ab, bb, s)
+    af, bf, wf = (O.bf16_bits_to_f32(v).astype(np.float64) for v in (ab, bb, wd))
+    bound = 2.0 ** -7 * np.abs(o) + 2.0 ** -24 * (r + 2) * (np.abs(wf) + abs(s) * (np.abs(bf) @ np.abs(af)))
+    got = O.bf16_bits_to_f32(bits(m)).astype(np.float64)
+    assert np.all(np.abs(got - o) <= bound)
+
+
+@pytest.mark.parametrize("T,N,K", [(1, 4096, 4096), (4, 1024, 4096), (16, 4096, 14336), (300, 384, 320),
+                                   (4096, 1024, 4096)])
+def test_large_adapter_activation(T, N, K):
+    """Token rows aligned with rows of A (x = 64 A_j K^{1/2} in distribution),
+    so that U = s x A^T reaches ~64 in a few columns while B ~ N(0, 0.01^2):
+    the rank-r term is then as large as the base term and partly cancels it,
+    and rounding U to one BF16 value would put outputs near zero outside the
+    tolerance.  Upstream gradients aligned with columns of B likewise make dU
+    large for the backward."""
+    q = Q()
+    r, s = 64, 1.0
+    W, X, A, B, dY = inputs.layer_inputs(98, 0, 0, T, N, K, r, device="cuda")
+    Xf, dYf = X.float(), dY.float()
+    for t in range(min(T, 8)):
+        Xf[t] = A[t % r].float() * (K ** 0.5) * 1.5
+        dYf[t] = B[:, t % r].float() * 300.0
+    X, dY = Xf.to(torch.bfloat16), dYf.to(torch.bfloat16)
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    y = q.linear_fwd(X, qw, A, B, s)
+    y2, u = q.linear_fwd_save(X, qw, A, B, s)
+    dx, dA, dB = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
+    dx2, _, _ = q.linear_bwd(dY, X, qw, A, B, s)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    rows = np.unique(np.concatenate([np.arange(min(T, 8)), [T - 1, T // 2]]))
+    idx = torch.from_numpy(rows).cuda()
+    ref = O.linear_fwd(xb[rows], wd, ab, bb, s)
+    U = O.bf16_bits_to_f32(xb[rows]).astype(np.float64) @ O.bf16_bits_to_f32(ab).astype(np.float64).T
+    assert np.abs(U).max() > 1.4 * K ** 0.5        # the stress really is there (U ~ N(0, 1) otherwise)
+    assert_close("Y", y[idx], ref)
+    assert_close("Y saved", y2[idx], ref)
+    rdx, _, _ = O.linear_bwd(dyb[rows], xb[rows], wd, ab, bb, s)
+    assert_close("dX", dx[idx], rdx)
+    assert_close("dX plain", dx2[idx], rdx)
+    rdA, rdB = O.lora_adapter_grads(dyb, xb, ab, bb, s)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
+
+
+# --------------------------------------------------------------------------
+# the adapters' optimizer step, with device and unified ("paged") state
+# --------------------------------------------------------------------------
+def _adam_inputs(n, seed):
+    g = torch.Generator().manual_seed(seed)
+    p0 = (torch.randn(n, generator=g) * 0.05).float()
+    grads = [inputs.normal_bf16((n,), 0.02, seed + 1 + t) for t in range(4)]
+    return p0, grads
+
+
+def _adam_oracle(p0, grads, hp):
+    p, m, v = p0.double().numpy(), np.zeros(p0.numel()), np.zeros(p0.numel())
+    for t, g in enumerate(grads, start=1):
+        p, m, v = O.adam_step(p, m, v, bits(g), t, **hp)
+    return p, m, v
+
+
+HP = dict(lr=2e-3, beta1=0.9, beta2=0.99, eps=1e-8, weight_decay=0.01)
+
+
+def _check_adam(p, m, v, ref, grads):
+    """FP32 arithmetic against the float64 oracle: each step rounds a few
+    times, so m and v may differ by a few FP32 ulps of the magnitudes summed
+    into them (|m| itself may cancel to near zero), and p by a few ulps of
+    itself and of the updates applied."""
+    rp, rm, rv = ref
+    p, m, v = (np.asarray(a, np.float64) for a in (p, m, v))
+    ulp = 2.0 ** -23
+    mag_m = np.zeros_like(rm)
+    for g in grads:                     # the same recursion on |g|: what m's terms add up to
+        mag_m = HP["beta1"] * mag_m + (1 - HP["beta1"]) * np.abs(O.bf16_bits_to_f32(bits(g)).astype(np.float64))
+    steps = len(grads)
+    assert np.all(np.abs(m - rm) <= 4 * steps * ulp * mag_m + 1e-30)
+    assert np.all(np.abs(v - rv) <= 4 * steps * ulp * rv + 1e-30)
+    assert np.all(np.abs(p - rp) <= 6 * steps * ulp * (np.abs(rp) + HP["lr"]))
+
+
+@pytest.mark.parametrize("n", [1_310_720 + 5, 7, 64 * 4096])
+def test_adam_step_matches_oracle(n):
+    """Four steps on FP32 state in device memory against the float64 oracle;
+    the BF16 parameter copy is the round-to-nearest-even of the FP32 result."""
+    q = Q()
+    p0, grads = _adam_inputs(n, 11 + n % 97)
+    p, m, v = p0.cuda(), torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+    pb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    for t, g in enumerate(grads, start=1):
+        q.adam_step(p, m, v, g.cuda(), pb, step=t, **HP)
+    torch.cuda.synchronize()
+    _check_adam(p.cpu().numpy(), m.cpu().numpy(), v.cpu().numpy(), _adam_oracle(p0, grads, HP), grads)
+    assert torch.equal(pb.view(torch.int16), p.to(torch.bfloat16).view(torch.int16))
+
+
+def test_adam_step_on_paged_state():
+    """The same steps with parameters and moments in unified memory, paged out
+    to the host before every step (the kernel's first touch brings them back):
+    bit-identical to the device-memory run, and readable from the host."""
+    q = Q()
+    n = 1_310_720
+    p0, grads = _adam_inputs(n, 5)
+    pd, md, vd = p0.cuda(), torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+    pp, mp, vp = (q.PagedBuffer(n) for _ in range(3))
+    torch.cuda.synchronize()
+    pp.numpy()[:] = p0.numpy()
+    mp.numpy()[:] = 0.0
+    vp.numpy()[:] = 0.0
+    for t, g in enumerate(grads, start=1):
+        gd = g.cuda()
+        q.adam_step(pd, md, vd, gd, step=t, **HP)
+        for b in (pp, mp, vp):
+            b.prefetch(to_host=True)
+        q.adam_step(pp, mp, vp, gd, step=t, **HP)
+    torch.cuda.synchronize()
+    for dev_t, paged in ((pd, pp), (md, mp), (vd, vp)):
+        assert np.array_equal(dev_t.cpu().numpy().view(np.uint32), paged.numpy().view(np.uint32))
+    _check_adam(pp.numpy(), mp.numpy(), vp.numpy(), _adam_oracle(p0, grads, HP), grads)
