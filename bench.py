@@ -294,7 +294,14 @@ def bench_ours(args, rank, world, local_rank):
                        "share": round(v["ms"] / sum(x["ms"] for x in kern.values()), 4),
                        "tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1) if v["flops"] else None}
                    for k, v in sorted(kern.items(), key=lambda kv: -kv[1]["ms"])}
-        secondary = None if args.no_secondary else bench_secondary(dev, peaks)
+        secondary = None
+        if not args.no_secondary:
+            secondary = bench_secondary(dev, peaks)
+            secondary["stack_8b_32_layers"] = bench_stack_8b(dev, peaks)
+            secondary["codebook_tables"] = bench_tables(dev)
+            secondary["adam_step"] = bench_adam(dev, peaks)
+            if not args.no_65b:
+                secondary["stack_65b_80_layers"] = bench_stack_65b(dev, peaks)
         cpu = None if args.no_cpu else cpu_baseline(args)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -498,6 +505,155 @@ def bench_secondary(dev, peaks):
     return out
 
 
+def _timed(fn, stream=None):
+    """CUDA-event time of fn() on the current stream, in ms."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def bench_stack_8b(dev, peaks):
+    """Every linear weight of a 32-layer Llama-3.1-8B-shaped stack (6.98e9
+    parameters, 14 GB of BF16, generated on the device), quantized to NF4 + DQ
+    and dequantized back, each as one back-to-back pass over the 224 matrices
+    between two CUDA events (the dequantize pass writes over the BF16 input)."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    Ws = [inputs.normal_bf16((N, K), 0.02, inputs.seed_of(3, layer, i, "W"), dev)
+          for layer in range(32) for i, (_, N, K) in enumerate(proj_shapes())]
+    qws = [q.quantize_nf4(W) for W in Ws]        # warm-up, and the buffers the timed pass refills
+    torch.cuda.synchronize()
+    n_w = sum(W.numel() for W in Ws)
+    n_b = sum(qw.nbytes() for qw in qws)
+    tq = _timed(lambda: [q.quantize_nf4_into(W, qw) for W, qw in zip(Ws, qws)])
+    td = _timed(lambda: [q.dequantize(qw, out=W) for W, qw in zip(Ws, qws)])
+    q.get_error(dev)
+    per = 2.0 + 0.5 + 1.0 / 64
+    res = {"weights": n_w, "stored_bytes": n_b, "bits_per_param": n_b * 8 / n_w}
+    for name, ms in (("quantize", tq), ("dequantize", td)):
+        gbs = n_w * per / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    res["timing"] = ("one pass of 224 back-to-back calls between CUDA events, for quantize and for "
+                     "dequantize; the stack is resident in HBM (14 GB BF16 + 3.6 GB NF4), far larger than L2")
+    del Ws, qws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_stack_65b(dev, peaks, clocks_fn=None):
+    """The 65B-shaped stack layer by layer: 80 layers x 7 projections (hidden
+    8192, ffn 22016), NF4 + DQ weights generated and quantized per layer (BF16
+    weights never all resident: 33.4 GB of NF4 are), rank-64 adapters, s =
+    0.25, fwd+bwd of every projection on 4 x 512 tokens (the saved-U path)."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    T, r, s = 2048, 64, 0.25
+    shapes = inputs.LLAMA65B_PROJ
+    per_proj = []
+    for i, (_, N, K) in enumerate(shapes):
+        _, X, _, _, dY = inputs.layer_inputs(4, 0, i, T, N, K, r, device=dev)
+        per_proj.append(dict(X=X, dY=dY, U=torch.empty(q.saved_u_bytes(T, r), dtype=torch.uint8, device=dev),
+                             Y=torch.empty(T, N, dtype=torch.bfloat16, device=dev),
+                             dX=torch.empty(T, K, dtype=torch.bfloat16, device=dev),
+                             dA=torch.empty(r, K, dtype=torch.bfloat16, device=dev),
+                             dB=torch.empty(N, r, dtype=torch.bfloat16, device=dev)))
+    layers = []
+    nf4_bytes = 0
+    t0 = time.perf_counter()
+    for layer in range(80):
+        row = []
+        for i, (_, N, K) in enumerate(shapes):
+            W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(4, layer, i, "W"), dev)
+            qw = q.quantize_nf4(W)
+            del W
+            A = inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(4, layer, i, "A"), dev)
+            B = inputs.normal_bf16((N, r), 0.01, inputs.seed_of(4, layer, i, "B"), dev)
+            nf4_bytes += qw.nbytes()
+            row.append((qw, A, B))
+        layers.append(row)
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t0
+
+    def run(n_layers):
+        for row in layers[:n_layers]:
+            for (qw, A, B), P in zip(row, per_proj):
+                q.linear_fwd_save(P["X"], qw, A, B, s, out=P["Y"], u_save=P["U"])
+                q.linear_bwd_saved(P["dY"], P["X"], qw, A, B, s, P["U"], outs=(P["dX"], P["dA"], P["dB"]))
+
+    run(3)   # warm-up
+    torch.cuda.synchronize()
+    ms = _timed(lambda: run(80))
+    q.get_error(dev)
+    flops = 80 * sum(4.0 * T * N * K + 6.0 * T * r * (N + K) for (_, N, K) in shapes)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"layers": 80, "tokens": T, "lora_rank": r, "lora_scale": s, "flops": flops, "ms": round(ms, 2),
+            "TFLOP/s": round(tf, 1), "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+            "frac_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+            "nf4_bytes_resident": nf4_bytes, "setup_s": round(setup_s, 1),
+            "timing": "CUDA events around one pass of the 80 layers after a 3-layer warm-up; weights "
+                      "generated and quantized layer by layer before it (not timed)"}
+
+
+def bench_tables(dev):
+    """Round-trip error of each 4-bit table through the GPU path: quantize and
+    dequantize a 4096 x 4096 N(0, 0.02^2) weight, RMS of W' - W relative to
+    the weights' RMS, with codes snapped against c1 or against the
+    double-quantized scale."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    cb = q.nf4_codebook()
+    zero = list(cb)
+    zero[7] = 0.0
+    tables = {"nf4_eq2": cb, "nf4_eq2_zero_level": zero, "int4_uniform": [(i - 8) / 8.0 for i in range(16)],
+              "uniform_16": [(2 * i - 15) / 15.0 for i in range(16)]}
+    W = inputs.normal_bf16((4096, 4096), 0.02, 12345, dev)
+    wf = W.float()
+    ref = wf.pow(2).mean().sqrt().item()
+    out = {}
+    for name, table in tables.items():
+        row = {}
+        for snap in (False, True):
+            wd = q.dequantize(q.quantize_nf4(W, codebook=table, snap_to_dq_scale=snap)).float()
+            row["snap_dq_scale" if snap else "snap_c1"] = round((wd - wf).pow(2).mean().sqrt().item() / ref, 5)
+        out[name] = row
+    q.get_error(dev)
+    return {"relative_rms_error": out, "weights": "4096 x 4096 N(0, 0.02^2) BF16, blocks of 64, DQ groups of 256"}
+
+
+def bench_adam(dev, peaks):
+    """The adapters' optimizer step over the 8B stack's 41.9 M rank-16 adapter
+    parameters (32 layers x 1,310,720), FP32 state in device memory and in
+    unified (paged) memory prefetched to the GPU."""
+    import torch
+    import bit_nf4_quantized_20_b200 as q
+    from bit_nf4_quantized_20_b200 import inputs
+    n = 32 * 1_310_720
+    g = inputs.normal_bf16((n,), 0.02, 777, dev)
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    res = {"params": n, "bytes_per_param": 28}
+    dev_state = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(3)]
+    paged = [q.PagedBuffer(n, device=dev) for _ in range(3)]
+    for b in paged:
+        b.prefetch()
+    for name, (p, m, v) in (("device", dev_state), ("paged", paged)):
+        for t in range(1, 4):
+            q.adam_step(p, m, v, g, out, step=t, lr=1e-4)
+        times = [_timed(lambda: q.adam_step(p, m, v, g, out, step=4, lr=1e-4)) for _ in range(5)]
+        ms = statistics.median(times)
+        gbs = 28.0 * n / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    q.get_error(dev)
+    del paged
+    return res
+
+
 # --------------------------------------------------------------------------
 # the CPU oracle (reference arm and cpu_baseline)
 # --------------------------------------------------------------------------
@@ -536,9 +692,44 @@ def cpu_baseline(args, T_sample=256):
     prepared = oracle_sample_step(T_sample)
     sec = oracle_sample_step(T_sample, prepared=prepared)
     v = step_flops(T_sample) / sec / 1e12
-    return {"value": round(v, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"one fwd+bwd pass of all 7 projections at T={T_sample} tokens (of 4096), "
-                      f"including the per-step NF4 dequantization; {sec:.1f} s"}
+    res = {"value": round(v, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"one fwd+bwd pass of all 7 projections at T={T_sample} tokens (of 4096), "
+                     f"including the per-step NF4 dequantization; {sec:.1f} s"}
+    res["other_legs"] = cpu_other_legs()
+    return res
+
+
+def cpu_other_legs():
+    """The oracle on bounded samples of the quantize and decode workloads."""
+    from oracle import oracle as O
+    from bit_nf4_quantized_20_b200 import inputs
+    out = {}
+    # quantize + dequantize of one 4096 x 4096 matrix of the 32-layer stack
+    N, K = 4096, 4096
+    wb = inputs.bf16_bits(inputs.normal_bf16((N, K), 0.02, inputs.seed_of(3, 0, 0, "W")))
+    t0 = time.perf_counter()
+    codes, scales, c2 = O.quantize_nf4(wb)
+    tq = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.dequantize_nf4(codes, scales, c2, N, K)
+    td = time.perf_counter() - t0
+    per = 2.0 + 0.5 + 1.0 / 64
+    out["quantize"] = {"GB/s": round(N * K * per / tq / 1e9, 3), "s": round(tq, 2),
+                       "sample": "one 4096 x 4096 matrix of the 32-layer 8B stack"}
+    out["dequantize"] = {"GB/s": round(N * K * per / td / 1e9, 3), "s": round(td, 2), "sample": "same matrix"}
+    # decode forward of the q projection at T = 1, rank 64 (dequantization included)
+    r = 64
+    W, X, A, B, _ = inputs.layer_inputs(2, 0, 0, 1, N, K, r)
+    codes, scales, c2 = O.quantize_nf4(inputs.bf16_bits(W))
+    xb, ab, bb = inputs.bf16_bits(X), inputs.bf16_bits(A), inputs.bf16_bits(B)
+    t0 = time.perf_counter()
+    O.linear_fwd(xb, O.dequantize_nf4(codes, scales, c2, N, K), ab, bb, 1.0)
+    tf = time.perf_counter() - t0
+    nbytes = N * K * (0.5 + 1 / 64) + 4 * ((N * K // 64 + 255) // 256) + 2 * r * (N + K) + 2 * (N + K)
+    out["decode_T1"] = {"GB/s": round(nbytes / tf / 1e9, 3), "s": round(tf, 2),
+                        "sample": "the q projection (4096 x 4096) at T = 1, rank 64"}
+    out["cores"] = oracle_threads()
+    return out
 
 
 def bench_reference(args, rank, world):
@@ -624,6 +815,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-secondary", action="store_true", help="skip the decode and quantize figures")
+    ap.add_argument("--no-65b", action="store_true", help="skip the 80-layer 65B-shaped stack")
     ap.add_argument("--path", default="saved", choices=["saved", "plain"],
                     help="saved: the forward saves U for the backward (default); plain: U recomputed")
     ap.add_argument("--profile-case", action="store_true",

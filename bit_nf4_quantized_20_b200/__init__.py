@@ -22,7 +22,7 @@ from ._lib import OP_BWD, OP_FWD, OP_QUANTIZE, NF4Weight, QLoraError, check, lib
 __all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "merge_adapter",
            "linear_fwd", "linear_bwd", "linear_fwd_save", "linear_bwd_saved", "saved_u_bytes",
            "linear_fwd_noalloc", "noalloc_get_error", "wait_selftest", "workspace", "workspace_bytes",
-           "get_error", "adam_step", "PagedBuffer", "QLoraError", "lib"]
+           "get_error", "adam_step", "PagedBuffer", "quantize_nf4_into", "QLoraError", "lib"]
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -139,6 +139,22 @@ def quantize_nf4(w: torch.Tensor, codebook=None, blocksize: int = 64, dq_block: 
     return QuantizedNF4(codes, scales, c2, rows, cols, cb, blocksize, dq_block)
 
 
+def quantize_nf4_into(w: torch.Tensor, qw: QuantizedNF4, snap_to_dq_scale: bool = False) -> QuantizedNF4:
+    """Quantize w again into the buffers of an existing QuantizedNF4 of the
+    same shape and codebook (no allocation)."""
+    _need_cuda("w", w)
+    if tuple(w.shape) != (qw.rows, qw.cols) or w.device != qw.device:
+        raise ValueError(f"w must be [{qw.rows}, {qw.cols}] on {qw.device}")
+    out = qw.struct()
+    cbuf = (C.c_float * 16)(*qw.codebook)
+    ws = workspace(qw.device, workspace_bytes(OP_QUANTIZE, 0, 0, 0, 1))
+    flags = _lib.QUANT_SNAP_DQ_SCALE if snap_to_dq_scale else 0
+    check("qlora_quantize_nf4_ex", lib().qlora_quantize_nf4_ex(
+        C.c_void_p(w.data_ptr()), qw.rows, qw.cols, qw.blocksize, qw.dq_block, cbuf, flags, C.byref(out),
+        C.c_void_p(ws.data_ptr()), ws.numel(), _stream(qw.device)))
+    return qw
+
+
 def merge_adapter(qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float) -> torch.Tensor:
     """BF16(W' + s B A) [rows, cols]: the adapter folded into the dequantized
     weight for export (quantize_nf4 of the result gives an NF4 merged model)."""
@@ -157,8 +173,12 @@ def merge_adapter(qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float) 
     return out
 
 
-def dequantize(qw: QuantizedNF4) -> torch.Tensor:
-    out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.device)
+def dequantize(qw: QuantizedNF4, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W' = BF16(RN32(codebook[code] * RN32(fp8 * c2))) as a [rows, cols] tensor."""
+    if out is None:
+        out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.device)
+    else:
+        _check_out("out", out, (qw.rows, qw.cols), qw.device)
     s = qw.struct()
     check("qlora_dequantize", lib().qlora_dequantize(C.byref(s), C.c_void_p(out.data_ptr()), _stream(qw.device)))
     return out

@@ -247,31 +247,46 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
             if (c0 + 4 * g < pw) dst[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
         }
       }
-      __threadfence();
+      // the epilogue's partial writes, ordered before one thread's GPU-scope
+      // release by the CTA barrier (the release is cumulative)
       named_bar_sync(1, 128);
       if (threadIdx.x == 64) {
-        const uint32_t old = atomicAdd(a.counters + m_tile, 1u);
+        uint32_t old;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + m_tile) : "memory");
         s_last = (old == static_cast<uint32_t>(a.splits - 1)) ? 1 : 0;
       }
       named_bar_sync(1, 128);
       if (s_last) {
-        __threadfence();
+        // (the acquiring atomic above, then the CTA barrier, order the other
+        // splits' partials before these reads)
         if (m < a.M) {
 #pragma unroll 1
           for (int c0 = 0; c0 < NB; c0 += CW) {
 #pragma unroll
             for (int j = 0; j < CW; ++j) v[j] = 0.f;
-            for (int sp = 0; sp < a.splits; ++sp) {
-              const float4 *src =
-                  reinterpret_cast<const float4 *>(a.partials + (static_cast<int64_t>(sp) * a.M + m) * pw + c0);
+            // the splits' partials in groups (64 floats of loads in flight per
+            // thread), each group's loads issued together, summed in split order
+            constexpr int G = 64 / CW;
+            constexpr int NV = CW / 4;
+            for (int sp0 = 0; sp0 < a.splits; sp0 += G) {
+              float4 t4[G][NV];
 #pragma unroll
-              for (int g = 0; g < CW / 4; ++g) {
-                if (c0 + 4 * g < pw) {
-                  const float4 t4 = __ldcg(src + g);
-                  v[4 * g] += t4.x;
-                  v[4 * g + 1] += t4.y;
-                  v[4 * g + 2] += t4.z;
-                  v[4 * g + 3] += t4.w;
+              for (int gi = 0; gi < G; ++gi) {
+                const int sp = sp0 + gi;
+                const float4 *src =
+                    reinterpret_cast<const float4 *>(a.partials + (static_cast<int64_t>(sp) * a.M + m) * pw + c0);
+#pragma unroll
+                for (int g = 0; g < NV; ++g)
+                  t4[gi][g] = (sp < a.splits && c0 + 4 * g < pw) ? __ldcg(src + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi) {
+#pragma unroll
+                for (int g = 0; g < NV; ++g) {
+                  v[4 * g] += t4[gi][g].x;
+                  v[4 * g + 1] += t4[gi][g].y;
+                  v[4 * g + 2] += t4[gi][g].z;
+                  v[4 * g + 3] += t4[gi][g].w;
                 }
               }
             }

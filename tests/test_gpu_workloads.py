@@ -105,14 +105,21 @@ def test_8b_block_projection_full_size(proj):
 # --------------------------------------------------------------------------
 # 65B-shaped stack, layer by layer: T = 4 x 512, rank 64, s = 0.25
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("proj", [0, 4, 6], ids=["q", "gate", "down"])
-def test_65b_projection_full_size(proj):
+@pytest.mark.parametrize("layer,proj", [(0, 0), (0, 4), (0, 6), (40, 0), (40, 4), (40, 6), (79, 0), (79, 4), (79, 6)],
+                         ids=lambda v: str(v))
+def test_65b_projection_full_size(layer, proj):
     """The three distinct shapes of a 65B-shaped layer (8192 <- 8192 for q, k,
-    v, o; 22016 <- 8192 for gate, up; 8192 <- 22016 for down)."""
+    v, o; 22016 <- 8192 for gate, up; 8192 <- 22016 for down) on layers 0, 40
+    and 79 of the 80-layer stack, seeded as the bench's layer-by-layer pass
+    seeds them (weights and adapters per layer, tokens and gradients from
+    layer 0)."""
     q = Q()
     name, N, K = inputs.LLAMA65B_PROJ[proj]
     T, r, s = 2048, 64, 0.25
-    W, X, A, B, dY = inputs.layer_inputs(4, 0, proj, T, N, K, r, device="cuda")
+    _, X, _, _, dY = inputs.layer_inputs(4, 0, proj, T, N, K, r, device="cuda")
+    W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(4, layer, proj, "W"), "cuda")
+    A = inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(4, layer, proj, "A"), "cuda")
+    B = inputs.normal_bf16((N, r), 0.01, inputs.seed_of(4, layer, proj, "B"), "cuda")
     qw, wd = quantize_checked(W)
     del W
     y, u = q.linear_fwd_save(X, qw, A, B, s)
