@@ -22,7 +22,8 @@ from ._lib import OP_BWD, OP_FWD, OP_QUANTIZE, NF4Weight, QLoraError, check, lib
 __all__ = ["QuantizedNF4", "nf4_codebook", "storage_bytes", "quantize_nf4", "dequantize", "merge_adapter",
            "linear_fwd", "linear_bwd", "linear_fwd_save", "linear_bwd_saved", "saved_u_bytes",
            "linear_fwd_noalloc", "noalloc_get_error", "wait_selftest", "workspace", "workspace_bytes",
-           "get_error", "adam_step", "PagedBuffer", "quantize_nf4_into", "QLoraError", "lib"]
+           "get_error", "adam_step", "PagedBuffer", "quantize_nf4_into", "linear_fwd_decode_batch",
+           "QLoraError", "lib"]
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -251,6 +252,45 @@ def linear_fwd_save(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch
         float(s), C.c_void_p(y.data_ptr()), C.c_void_p(u_save.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel(),
         _stream(dev)))
     return y, u_save
+
+
+class DecodeBatch:
+    """A prepared grouped decode-sized forward (qlora_linear_fwd_decode_batch):
+    the argument structs are built once, so that repeated calls (or a CUDA
+    graph capture) only cross the boundary.  problems: (x, qw, A, B, s, out)."""
+
+    def __init__(self, problems):
+        if not 1 <= len(problems) <= 8:
+            raise ValueError("1 to 8 problems")
+        T = None
+        self._keep = []
+        self.arr = (_lib.FwdProblem * len(problems))()
+        for i, (x, qw, A, B, s, out) in enumerate(problems):
+            Ti, r = _check_linear(x, qw, A, B)
+            _check_out("out", out, (Ti, qw.rows), x.device)
+            if T is None:
+                T, self.device = Ti, x.device
+            elif Ti != T or x.device != self.device:
+                raise ValueError("every problem must have the same token count and device")
+            st = qw.struct()
+            self._keep.append((st, x, qw, A, B, out))
+            self.arr[i] = _lib.FwdProblem(x.data_ptr(), C.pointer(st), A.data_ptr(), B.data_ptr(), r, float(s),
+                                          out.data_ptr())
+        self.n, self.T = len(problems), T
+        need = int(lib().qlora_decode_batch_workspace_bytes(self.n, self.arr, T))
+        if need == 0:
+            raise ValueError("problems not supported by the grouped decode forward (T <= 16)")
+        self.ws = workspace(self.device, need)
+
+    def __call__(self):
+        check("qlora_linear_fwd_decode_batch", lib().qlora_linear_fwd_decode_batch(
+            self.n, self.arr, self.T, C.c_void_p(self.ws.data_ptr()), self.ws.numel(), _stream(self.device)))
+
+
+def linear_fwd_decode_batch(problems) -> None:
+    """Decode-sized forward (T <= 16) of several projections in one grouped
+    call; problems: list of (x, qw, A, B, s, out), outputs written in place."""
+    DecodeBatch(problems)()
 
 
 def linear_fwd_noalloc(x: torch.Tensor, qw: QuantizedNF4, A: torch.Tensor, B: torch.Tensor, s: float,

@@ -35,6 +35,12 @@ class AdamHParams(C.Structure):
                 ("weight_decay", C.c_float), ("step", C.c_int32)]
 
 
+class FwdProblem(C.Structure):
+    """Mirror of qlora_fwd_problem."""
+    _fields_ = [("x", C.c_void_p), ("qw", C.POINTER(NF4Weight)), ("A", C.c_void_p), ("B", C.c_void_p),
+                ("r", C.c_int32), ("s", C.c_float), ("y", C.c_void_p)]
+
+
 class TraceRec(C.Structure):
     """Mirror of qlora_trace_rec."""
     _fields_ = [("kernel", C.c_int32), ("pad_", C.c_int32), ("start", C.c_void_p), ("stop", C.c_void_p),
@@ -68,6 +74,9 @@ SIGNATURES = {
     "qlora_linear_fwd_noalloc": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
                                            C.c_int32, C.c_float, C.c_void_p, C.c_void_p]),
     "qlora_noalloc_get_error": (C.c_int, [C.c_void_p]),
+    "qlora_decode_batch_workspace_bytes": (C.c_size_t, [C.c_int32, C.POINTER(FwdProblem), C.c_int64]),
+    "qlora_linear_fwd_decode_batch": (C.c_int, [C.c_int32, C.POINTER(FwdProblem), C.c_int64, C.c_void_p,
+                                                C.c_size_t, C.c_void_p]),
     "qlora_saved_u_bytes": (C.c_size_t, [C.c_int64, C.c_int32]),
     "qlora_linear_fwd_save": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(NF4Weight), C.c_void_p, C.c_void_p,
                                         C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,

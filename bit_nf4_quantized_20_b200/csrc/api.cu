@@ -246,8 +246,8 @@ bool codebook_symmetric(const float *cb) {
 // Up to this many tokens the forward runs the decode GEMV, and U = s X A^T
 // runs on the mma.sync kernel (a handful of rows: latency, not bandwidth).
 constexpr int64_t kGemvMaxTokens = 16;
-// the split counters of the decode GEMV are the workspace's tile counters
-constexpr int kGemvMaxCounterTiles = static_cast<int>(kWsCounterBytes / sizeof(uint32_t));
+// the decode GEMV keeps one split counter per 32-row tile in the workspace's counters
+static_assert(kDecodeMaxTiles * sizeof(uint32_t) <= kWsCounterBytes, "decode tile counters");
 
 bool decode_path(int64_t T, int64_t N) {
   (void)N;
@@ -305,12 +305,10 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   if (op == QLORA_OP_FWD) {
     L.su_row = off; off += row_plane;
     // the tensor-core U product (every token count when U is saved for the
-    // backward); at decode sizes also the U' fallback's partials and, after
-    // it has finished, the GEMV's split partials
+    // backward, and at decode sizes when the cluster U kernel's slice does not
+    // fit); at decode sizes, after it, the GEMV's split partials
     part = skinny_tc_partials_bytes(geom_u(T, K, r), T, r);
-    if (decode_path(T, N))
-      part = std::max(part, std::max(skinny_partials_bytes(T, K, r, kSplitSms),
-                                     gemv_persist_partials_bytes(N, K, kGemvMaxCounterTiles)));
+    if (decode_path(T, N)) part = std::max(part, decode_gemv_partials_bytes());
   } else {
     L.suT_hi = off; off += t_plane;
     L.suT_lo = off; off += t_plane;
@@ -326,22 +324,6 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
   off += static_cast<size_t>(round_up(static_cast<int64_t>(part), 256));
   L.total = off;
   return L;
-}
-
-// Parameters of the mma.sync rank-r kernel (decode-sized U only).
-SkinnyParams skinny_base(int64_t M, int64_t C, int R, uint8_t *ws, const WsLayout &L) {
-  SkinnyParams p;
-  memset(&p, 0, sizeof(p));
-  p.M = M;
-  p.C = C;
-  p.R = R;
-  p.splits = skinny_splits(M, C, kSplitSms);
-  int64_t per = (C + p.splits - 1) / p.splits;
-  p.c_per_split = round_up(per, 64);
-  p.partials = reinterpret_cast<float *>(ws + L.partials);
-  p.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
-  p.status = reinterpret_cast<uint32_t *>(ws);
-  return p;
 }
 
 // The fused GEMM's launch, prepared (tensor maps encoded, parameters filled)
@@ -416,35 +398,84 @@ qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
 }
 
 
-// The decode forward; u holds U' = s X A^T as hi | lo BF16 planes per row [T, ldu].
-qlora_status run_gemv(const qlora_nf4_weight *qw, const void *x, int64_t T, const uint16_t *u, int64_t ldu,
-                      const void *B, int r, void *y, uint8_t *ws, const WsLayout &L, cudaStream_t st) {
-  GemvParams p;
+// 2-D byte matrix [rows, cols] (row stride ld bytes), box [box_rows, box_cols],
+// with the 128-byte swizzle when box_cols == 128.
+bool make_map_u8(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows,
+                 int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// One problem of a decode-sized launch: problem i of `a` (and of `ua`, for the
+// U' kernel) from the caller's buffers; U' lives at u [T, 2 ceil64(r)].
+bool fill_decode_problem(DecodeArgs &a, DecodeUArgs &ua, int i, const void *x, const qlora_nf4_weight *qw,
+                         const void *A, const void *B, int r, float s, void *y, uint16_t *u, int64_t T) {
+  const int64_t r64 = round_up(r, 64);
+  if (!make_map_u8(&a.codes_map[i], qw->codes, qw->rows, qw->cols / 2, qw->cols / 2, 32, 128)) return false;
+  DecodeProblem &p = a.prob[i];
   memset(&p, 0, sizeof(p));
-  p.codes = qw->codes;
   p.scales = qw->scales;
   p.c2 = qw->c2;
-  for (int i = 0; i < 16; ++i) p.codebook[i] = qw->codebook[i];
+  for (int j = 0; j < 16; ++j) p.codebook[j] = qw->codebook[j];
   p.N = qw->rows;
   p.K = qw->cols;
-  p.T = static_cast<int>(T);
   p.x = static_cast<const uint16_t *>(x);
   p.u = u;
-  p.ldu = ldu;
+  p.ldu = 2 * r64;
   p.B = static_cast<const uint16_t *>(B);
   p.r = r;
   p.y = static_cast<uint16_t *>(y);
   p.sym = codebook_symmetric(qw->codebook) ? 1 : 0;
-  p.ctas = gemv_persist_ctas(p.N, p.K, num_sms_current(), kGemvMaxCounterTiles);
-  p.part = reinterpret_cast<float *>(ws + L.partials);
-  p.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
-  const double n = static_cast<double>(p.N) * p.K;
-  const double bytes = n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * T * (p.N + p.K) +
-                       2.0 * static_cast<double>(p.N) * r;
-  TraceScope ts(K_GEMV_FWD, 0.0, bytes, st);
+  DecodeUProblem &q = ua.prob[i];
+  memset(&q, 0, sizeof(q));
+  q.x = static_cast<const uint16_t *>(x);
+  q.A = static_cast<const uint16_t *>(A);
+  q.u = u;
+  q.K = qw->cols;
+  q.ldu = 2 * r64;
+  q.plane = r64;
+  q.r = r;
+  q.alpha = s;
+  (void)T;
+  return true;
+}
+
+double decode_bytes(const DecodeArgs &a) {
+  double bytes = 0.0;
+  for (int i = 0; i < a.n; ++i) {
+    const DecodeProblem &p = a.prob[i];
+    const double n = static_cast<double>(p.N) * p.K;
+    bytes += n * (0.5 + 1.0 / 64) + 4.0 * ((n / 64 + 255) / 256) + 2.0 * a.T * (p.N + p.K) +
+             2.0 * static_cast<double>(p.N) * p.r;
+  }
+  return bytes;
+}
+
+qlora_status run_decode_gemv(DecodeArgs &a, cudaStream_t st) {
+  TraceScope ts(K_GEMV_FWD, 0.0, decode_bytes(a), st);
   // programmatic dependent launch only when no trace events sit between the kernels
   const bool pdl = g_trace.recs == nullptr;
-  return launch_gemv(p, num_sms_current(), st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return launch_decode_gemv(a, num_sms_current(), st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status run_decode_u(const DecodeUArgs &ua, cudaStream_t st) {
+  double flops = 0.0, bytes = 0.0;
+  for (int i = 0; i < ua.n; ++i) {
+    flops += 2.0 * ua.T * ua.prob[i].K * ua.prob[i].r;
+    bytes += 2.0 * ua.prob[i].r * ua.prob[i].K + 2.0 * ua.T * ua.prob[i].K;
+  }
+  TraceScope ts(K_LORA_U, flops, bytes, st);
+  const bool pdl = g_trace.recs == nullptr;
+  return launch_decode_u(ua, st, pdl) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 // One tensor-core rank-r product.  P: p_col ? [C rows, M cols] : [M rows, C cols]
@@ -703,6 +734,8 @@ static qlora_status check_linear(const void *x, int64_t T, const qlora_nf4_weigh
   if (T < 0 || r < 1 || r > 128 || !isfinite(s)) return QLORA_ERR_INVALID_ARG;
   if (qw->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
   if (T > 0x7fffffff || qw->rows > 0x7fffffff || qw->cols > 0x7fffffff) return QLORA_ERR_UNSUPPORTED;
+  // decode-sized token counts keep one counter per 32 weight rows
+  if (T >= 1 && decode_path(T, qw->rows) && (qw->rows + 31) / 32 > kDecodeMaxTiles) return QLORA_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_MISALIGNED;
   return QLORA_OK;
 }
@@ -737,44 +770,25 @@ static qlora_status linear_fwd_impl(const void *x, int64_t T, const qlora_nf4_we
   const int64_t r64 = round_up(r, 64);
   uint16_t *su = reinterpret_cast<uint16_t *>(w8 + L.su_row);
   const bool decode = decode_path(T, N);
-  if (decode && !u_save) {
-    // sU = s X A^T [T, ceil64(r)], a handful of rows: a latency-bound product,
-    // on a cluster kernel (one wave, partial sums in distributed shared
-    // memory) where its slice fits
-    const bool pdl = g_trace.recs == nullptr;
-    if (lora_u_decode_smem_bytes(K, static_cast<int>(T)) <= kLoraUDecodeMaxSmem) {
-      LoraUDecodeParams pu;
-      pu.x = static_cast<const uint16_t *>(x);
-      pu.A = static_cast<const uint16_t *>(A);
-      pu.u = su;
-      pu.K = K;
-      pu.ldu = 2 * r64;
-      pu.plane = r64;
-      pu.T = static_cast<int>(T);
-      pu.r = r;
-      pu.kc = 0;
-      pu.alpha = s;
-      {
-        TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * r * K, st);
-        if (launch_lora_u_decode(pu, st, pdl) != cudaSuccess) return QLORA_ERR_CUDA;
-      }
-      return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
+  DecodeArgs da;
+  DecodeUArgs ua;
+  if (decode) {
+    memset(&da, 0, sizeof(da));
+    memset(&ua, 0, sizeof(ua));
+    da.n = ua.n = 1;
+    da.T = ua.T = static_cast<int>(T);
+    da.part = reinterpret_cast<float *>(w8 + L.partials);
+    da.counters = reinterpret_cast<uint32_t *>(w8 + L.counters);
+    da.status = reinterpret_cast<uint32_t *>(ws);
+    if (!fill_decode_problem(da, ua, 0, x, qw, A, B, r, s, y, su, T)) return QLORA_ERR_CUDA;
+    if (!u_save && decode_u_smem_bytes(K, static_cast<int>(T)) <= kDecodeUMaxSmem) {
+      // sU = s X A^T [T, hi | lo], a handful of rows: a latency-bound product on a
+      // cluster kernel (one wave, partial sums in distributed shared memory)
+      qlora_status rs = run_decode_u(ua, st);
+      if (rs != QLORA_OK) return rs;
+      da.early_start = g_trace.recs == nullptr ? 1 : 0;   // programmatic launch only without a trace
+      return run_decode_gemv(da, st);
     }
-    SkinnyParams pu = skinny_base(T, K, r, w8, L);
-    pu.P = static_cast<const uint16_t *>(x);
-    pu.ldp = K;
-    pu.Q0 = static_cast<const uint16_t *>(A);
-    pu.ldq = K;
-    pu.alpha = s;
-    pu.out0 = su;
-    pu.out1 = su + r64;
-    pu.ldo = 2 * r64;
-    pu.ocols = r64;
-    {
-      TraceScope ts(K_LORA_U, 2.0 * T * K * r, 2.0 * T * K, st);
-      if (launch_skinny(pu, false, false, OUT_HILO, st) != cudaSuccess) return QLORA_ERR_CUDA;
-    }
-    return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
   }
   // sU on the tensor cores: the row plane for the GEMM / GEMV's rank-r term
   // and, when the backward will need it, the transposed hi + lo planes
@@ -796,7 +810,7 @@ static qlora_status linear_fwd_impl(const void *x, int64_t T, const qlora_nf4_we
   if (decode) {
     rs = launch_tc(lu, st);
     if (rs != QLORA_OK) return rs;
-    return run_gemv(qw, x, T, su, 2 * r64, B, r, y, w8, L, st);
+    return run_decode_gemv(da, st);
   }
   GemmLaunch gl;
   rs = prepare_gemm(0, qw, x, su, r64, B, r, y, T, reinterpret_cast<uint32_t *>(ws), gl);
@@ -958,6 +972,105 @@ qlora_status qlora_linear_bwd_saved(const void *dy, const void *x, int64_t T, co
                                     const void *A, const void *B, int32_t r, float s, const void *u_saved, void *dx,
                                     void *dA, void *dB, void *ws, size_t ws_bytes, void *stream) {
   return linear_bwd_entry(dy, x, T, qw, A, B, r, s, u_saved, true, dx, dA, dB, ws, ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Decode-sized forward of several projections in one pair of launches
+// ---------------------------------------------------------------------------
+static size_t decode_batch_layout(int32_t n, const qlora_fwd_problem *probs, int64_t T, size_t *u_off,
+                                  size_t *part_off) {
+  size_t off = kWsHeaderBytes + kWsCounterBytes;
+  for (int i = 0; i < n; ++i) {
+    u_off[i] = off;
+    off += static_cast<size_t>(round_up(T * 2 * round_up(probs[i].r, 64) * 2, 256));
+  }
+  size_t part = decode_gemv_partials_bytes();
+  for (int i = 0; i < n; ++i)   // the tensor-core U fallback (a K too long for the cluster kernel)
+    part = std::max(part, skinny_tc_partials_bytes(geom_u(T, probs[i].qw->cols, probs[i].r), T, probs[i].r));
+  *part_off = off;
+  return off + static_cast<size_t>(round_up(static_cast<int64_t>(part), 256));
+}
+
+static qlora_status check_decode_batch(int32_t n, const qlora_fwd_problem *probs, int64_t T) {
+  if (n < 1 || n > kDecodeMaxProblems || !probs) return QLORA_ERR_INVALID_ARG;
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (T > kGemvMaxTokens) return QLORA_ERR_UNSUPPORTED;
+  int64_t tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    const qlora_fwd_problem &p = probs[i];
+    qlora_status cs = check_fwd(p.x, T, p.qw, p.A, p.B, p.r, p.s, p.y, nullptr, false);
+    if (cs != QLORA_OK) return cs;
+    tiles += (p.qw->rows + 31) / 32;
+  }
+  if (tiles > kDecodeMaxTiles) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+size_t qlora_decode_batch_workspace_bytes(int32_t n, const qlora_fwd_problem *probs, int64_t T) {
+  if (check_decode_batch(n, probs, T) != QLORA_OK) return 0;
+  size_t u_off[kDecodeMaxProblems], part_off;
+  return decode_batch_layout(n, probs, T, u_off, &part_off);
+}
+
+qlora_status qlora_linear_fwd_decode_batch(int32_t n, const qlora_fwd_problem *probs, int64_t T, void *ws,
+                                           size_t ws_bytes, void *stream) {
+  qlora_status cs = check_decode_batch(n, probs, T);
+  if (cs != QLORA_OK) return cs;
+  size_t u_off[kDecodeMaxProblems], part_off;
+  const size_t need = decode_batch_layout(n, probs, T, u_off, &part_off);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (T == 0) return QLORA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  DecodeArgs da;
+  DecodeUArgs ua;
+  memset(&da, 0, sizeof(da));
+  memset(&ua, 0, sizeof(ua));
+  da.n = n;
+  da.T = ua.T = static_cast<int>(T);
+  da.part = reinterpret_cast<float *>(w8 + part_off);
+  da.counters = reinterpret_cast<uint32_t *>(w8 + kWsHeaderBytes);
+  da.status = reinterpret_cast<uint32_t *>(ws);
+  // U' of every problem: the cluster kernel for those whose K slice fits, the
+  // tensor-core product for the others (prepared before anything is enqueued)
+  DecodeUArgs all;
+  memset(&all, 0, sizeof(all));
+  TcLaunch tc[kDecodeMaxProblems];
+  bool use_tc[kDecodeMaxProblems];
+  for (int i = 0; i < n; ++i) {
+    const qlora_fwd_problem &p = probs[i];
+    uint16_t *u = reinterpret_cast<uint16_t *>(w8 + u_off[i]);
+    if (!fill_decode_problem(da, all, i, p.x, p.qw, p.A, p.B, p.r, p.s, p.y, u, T)) return QLORA_ERR_CUDA;
+    use_tc[i] = decode_u_smem_bytes(p.qw->cols, static_cast<int>(T)) > kDecodeUMaxSmem;
+    if (use_tc[i]) {
+      const int64_t r64 = round_up(p.r, 64);
+      SkinnyTcArgs au = tc_args(T, p.qw->cols, p.r, p.s);
+      au.row_hi = u;
+      au.row_lo = u + r64;
+      au.ldo = 2 * r64;
+      au.ocols = r64;
+      const TcProduct tu = {K_LORA_U, p.x, p.qw->cols, false, p.A, nullptr, p.qw->cols, false,
+                            geom_u(T, p.qw->cols, p.r)};
+      WsLayout L;
+      L.counters = kWsHeaderBytes;
+      L.partials = part_off;
+      qlora_status rs = prepare_single_tc(tu, au, w8, L, tc[i]);
+      if (rs != QLORA_OK) return rs;
+    } else {
+      ua.prob[ua.n++] = all.prob[i];
+    }
+  }
+  for (int i = 0; i < n; ++i) {
+    if (!use_tc[i]) continue;
+    qlora_status rs = launch_tc(tc[i], st);
+    if (rs != QLORA_OK) return rs;
+  }
+  if (ua.n > 0) {
+    qlora_status rs = run_decode_u(ua, st);
+    if (rs != QLORA_OK) return rs;
+    da.early_start = g_trace.recs == nullptr ? 1 : 0;   // programmatic launch only without a trace
+  }
+  return run_decode_gemv(da, st);
 }
 
 // ---------------------------------------------------------------------------

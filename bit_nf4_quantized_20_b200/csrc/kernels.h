@@ -75,95 +75,69 @@ __global__ void nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act
                                     const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
 
 // ---------------------------------------------------------------------------
-// decode-sized forward, T <= 16 (gemv_nf4.cu)
+// decode-sized forward of one or several projections (decode.cu)
 // ---------------------------------------------------------------------------
-struct GemvParams {
-  const uint8_t *codes;
+constexpr int kDecodeMaxProblems = 8;
+constexpr int kDecodeWarps = 6;
+constexpr int kDecodeMaxCtas = 512;
+constexpr int64_t kDecodeMaxTiles = 16384;       // 32-row tiles over all problems (workspace counters)
+constexpr int kDecodeUMaxSmem = 200 * 1024;
+
+struct DecodeProblem {
   const uint8_t *scales;
   const float *c2;
   float codebook[16];
   int64_t N, K;
-  int T;
+  int64_t kb;            // K / 64 blocks per row                        (filled by the launcher)
+  int kus;               // 256-code units per row                        (filled by the launcher)
+  int64_t tiles;         // 32-row tiles                                  (filled by the launcher)
+  int64_t unit0, tile0;  // first global unit and tile of this problem    (filled by the launcher)
   const uint16_t *x;     // [T, K]
-  const uint16_t *u;     // U' = s X A^T as BF16 hi + lo: row t = [hi (ldu/2 cols), lo (ldu/2 cols)]
+  const uint16_t *u;     // U' = s X A^T as hi | lo BF16 planes per row [T, ldu]
   int64_t ldu;
   const uint16_t *B;     // [N, r]
   int r;
   uint16_t *y;           // [T, N]
   int sym;               // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
-  int units, upw, splits;  // filled from the plan
-  // persistent kernel (K % 256 == 0): `ctas` CTAs (0 = per-tile kernel), the
-  // sums of the tiles that straddle two CTAs [kPersistMaxCtas][2][16][16] fp32, and
-  // one counter per 16-row tile (zero between calls)
-  int tiles, ctas;
-  float *part;
-  uint32_t *counters;
 };
-struct GemvPlan {
-  int units;       // 256-wide k-units per row
-  int upw;         // units per warp
-  int splits;      // warps per CTA (k-splits of one 16-row tile, <= 8)
-  int tiles;       // 16-row tiles = CTAs
-};
-int gemv_smem_bytes(int splits);
-// CTAs of the persistent GEMV for an N x K weight on `num_sms` SMs (0 when it
-// does not apply: K % 256 != 0 or more 16-row tiles than `max_tiles` counters),
-// and the workspace its straddling tiles need (independent of the device)
-constexpr int64_t kPersistMaxCtas = 1024;
-int gemv_persist_ctas(int64_t N, int64_t K, int num_sms, int max_tiles);
-size_t gemv_persist_partials_bytes(int64_t N, int64_t K, int max_tiles);
-// launches the persistent kernel when p.ctas > 0, else the per-tile kernel
-cudaError_t launch_gemv(const GemvParams &p, int num_sms, cudaStream_t st, bool pdl);
-
-// U' = alpha X A^T for T <= 16 (gemv_nf4.cu) as two BF16 planes in each row of
-// u [T, ldu]: hi = bf16(v) in columns 0 .. plane - 1, lo = bf16(v - hi) in
-// columns plane .. 2 plane - 1; columns r .. plane - 1 of each are written as zero.
-struct LoraUDecodeParams {
-  const uint16_t *x;     // [T, K]
-  const uint16_t *A;     // [r, K]
-  uint16_t *u;           // [T, ldu], ldu >= 2 plane
-  int64_t K, ldu, plane; // plane a multiple of 16, >= r
-  int T, r;
-  int kc;                // contraction per CTA (set by the launcher)
-  float alpha;
-};
-constexpr int kLoraUDecodeMaxSmem = 200 * 1024;
-// Dynamic shared memory the kernel needs for (K, T); it runs when <= kLoraUDecodeMaxSmem.
-int lora_u_decode_smem_bytes(int64_t K, int T);
-cudaError_t launch_lora_u_decode(const LoraUDecodeParams &p, cudaStream_t st, bool pdl);
-
-// ---------------------------------------------------------------------------
-// rank-r LoRA GEMMs on the legacy tensor path (skinny.cu)
-//   C[M, R] = alpha * sum_c P(m, c) * Q(c, j),  Q = Q0 (+ Q1)
-// ---------------------------------------------------------------------------
-enum SkinnyOut : int {
-  OUT_HILO = 0,      // two BF16 planes [M, ldo]: hi = bf16(v), lo = bf16(v - hi); cols R..ldo zero
-  OUT_ROW = 1,       // BF16 [M, R] row-major
-  OUT_T = 2,         // BF16 [R, M] (transposed) row-major
-};
-
-struct SkinnyParams {
-  const uint16_t *P;   // BF16
-  int64_t ldp;
-  const uint16_t *Q0;  // BF16
-  const uint16_t *Q1;  // optional second plane (nullptr if none)
-  int64_t ldq;
-  int64_t M, C;        // rows, contraction length
-  int R;               // output columns (<= 128)
-  int splits;          // contraction splits
-  int64_t c_per_split; // multiple of 64
-  float alpha;
-  uint16_t *out0;      // OUT_HILO: hi plane; else output
-  uint16_t *out1;      // OUT_HILO: lo plane
-  int64_t ldo;         // OUT_HILO: plane row stride (>= R); unused otherwise
-  int64_t ocols;       // OUT_HILO: columns written per row of each plane (R .. ocols - 1 zero)
-  float *partials;     // [splits][M][RP] when splits > 1
-  uint32_t *counters;  // one per 64-row tile when splits > 1 (zero on entry, zero on exit)
+struct __align__(64) DecodeArgs {
+  CUtensorMap codes_map[kDecodeMaxProblems];   // codes as bytes [N][K / 2], box [32 rows][128 B], 128-byte swizzle
+  DecodeProblem prob[kDecodeMaxProblems];
+  int n, T;
+  int early_start;       // the preceding kernel is decode_u_kernel: stream before the dependency wait
+  int64_t units;         // (filled by the launcher)
+  float *part;           // [kDecodeMaxCtas][2][16][32] fp32: sums of tiles that straddle CTAs
+  uint32_t *counters;    // one per tile over all problems (zero between calls)
   uint32_t *status;
 };
+size_t decode_gemv_partials_bytes();
+cudaError_t launch_decode_gemv(DecodeArgs &a, int num_sms, cudaStream_t st, bool pdl);
 
-// The same products on tcgen05 (skinny_tc.cu): P and Q arrive by TMA, the
-// accumulator (128 rows x NB columns, FP32) lives in tensor memory.
+struct DecodeUProblem {
+  const uint16_t *x;     // [T, K]
+  const uint16_t *A;     // [r, K]
+  uint16_t *u;           // [T, ldu]: hi plane in columns 0 .. plane - 1, lo plane from column plane
+  int64_t K, ldu, plane; // plane a multiple of 16, >= r
+  int r;
+  float alpha;
+  int kc, cluster0;      // (filled by the launcher)
+};
+struct DecodeUArgs {
+  DecodeUProblem prob[kDecodeMaxProblems];
+  int n, T;
+  int red_off;           // (filled by the launcher)
+};
+// Dynamic shared memory of decode_u_kernel for the longest K of a launch; the
+// kernel runs when it is <= kDecodeUMaxSmem.
+int decode_u_smem_bytes(int64_t K_max, int T);
+cudaError_t launch_decode_u(const DecodeUArgs &a, cudaStream_t st, bool pdl);
+
+// ---------------------------------------------------------------------------
+// the rank-r LoRA products (skinny_tc.cu):
+//   C[M, R] = alpha * sum_c P(m, c) * Q(c, j),  Q = Q0 (+ Q1)
+// P and Q arrive by TMA, the accumulator (128 rows x NB columns, FP32) lives in
+// tensor memory.
+// ---------------------------------------------------------------------------
 struct SkinnyTcGeom {
   int nb;               // MMA N: R rounded up to 16, 32, 64 or 128 (64 or 128 for MN-major Q)
   int stages;           // TMA pipeline depth
@@ -210,11 +184,5 @@ cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *map
                                   const CUtensorMap *maps1, cudaStream_t st, bool pdl);
 cudaError_t launch_pad_cols(const uint16_t *src, int64_t rows, int cols, uint16_t *dst, int ldd, cudaStream_t st,
                             int num_sms);
-
-// p_col: P stored as [c][m] (else [m][c]); q_cj: Q stored as [c][j] (else [j][c]).
-cudaError_t launch_skinny(const SkinnyParams &p, bool p_col, bool q_cj, int out_mode, cudaStream_t st);
-// Split count and partial-buffer bytes the launcher will use for (M, C).
-int skinny_splits(int64_t M, int64_t C, int num_sms);
-size_t skinny_partials_bytes(int64_t M, int64_t C, int R, int num_sms);
 
 }  // namespace qlora

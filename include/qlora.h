@@ -259,6 +259,33 @@ QLORA_API qlora_status qlora_linear_bwd_saved(const void *dy, const void *x, int
                                               void *stream);
 
 /*
+ * The forward of several projections at decode-sized token counts in one pair
+ * of launches (a grouped call; the pages have no counterpart: in a decoder the
+ * q, k, v projections share their input, and so do gate and up).  Problem i
+ * computes y_i = x_i W'_i^T + s_i (x_i A_i^T) B_i^T exactly as qlora_linear_fwd
+ * would, with the arguments and requirements of that call; all share T.
+ * 1 <= n <= 8; 0 <= T <= 16 (UNSUPPORTED above); at most 16384 weight-row
+ * tiles of 32 over all problems (UNSUPPORTED).  ws: at least
+ * qlora_decode_batch_workspace_bytes(n, probs, T) bytes, 256-byte aligned,
+ * zeroed once before first use like any workspace.  The problems' outputs must
+ * not overlap their inputs or each other.
+ * Errors: as qlora_linear_fwd for any problem; INVALID_ARG for n or probs.
+ */
+typedef struct {
+  const void *x;                 /* [T, K] BF16 */
+  const qlora_nf4_weight *qw;    /* N x K */
+  const void *A;                 /* [r, K] BF16 */
+  const void *B;                 /* [N, r] BF16 */
+  int32_t r;
+  float s;
+  void *y;                       /* [T, N] BF16, written */
+} qlora_fwd_problem;
+QLORA_API size_t qlora_decode_batch_workspace_bytes(int32_t n, const qlora_fwd_problem *probs, int64_t T);
+QLORA_API qlora_status qlora_linear_fwd_decode_batch(int32_t n, const qlora_fwd_problem *probs, int64_t T, void *ws,
+                                                     size_t ws_bytes, void *stream);
+
+/*
+ * Forward without a caller-supplied workspace/*
  * Forward without a caller-supplied workspace (no counterpart on the pages: a
  * deployment aid).  For callers that cannot allocate device memory: code that
  * runs under a host framework which owns every device allocation (a serving

@@ -288,3 +288,28 @@ def test_adam_and_paged_validation(L):
     assert L.qlora_paged_alloc(16, None) == 1
     assert L.qlora_paged_free(None) == 0
     assert L.qlora_paged_prefetch(None, 16, 0, None) == 1
+
+
+def test_decode_batch_validation(L):
+    from bit_nf4_quantized_20_b200._lib import FwdProblem
+    w = _weight()
+    P = FAKE
+    arr = (FwdProblem * 9)()
+    for i in range(9):
+        arr[i] = FwdProblem(P, C.pointer(w), P, P, 8, 2.0, P)
+    ws = C.c_void_p(FAKE)
+    assert L.qlora_decode_batch_workspace_bytes(2, arr, 4) > 0
+    assert L.qlora_decode_batch_workspace_bytes(9, arr, 4) == 0          # at most 8 problems
+    assert L.qlora_decode_batch_workspace_bytes(2, arr, 17) == 0         # decode-sized token counts only
+    b = L.qlora_linear_fwd_decode_batch
+    assert b(0, arr, 4, ws, 1 << 30, None) == 1
+    assert b(9, arr, 4, ws, 1 << 30, None) == 1
+    assert b(2, None, 4, ws, 1 << 30, None) == 1
+    assert b(2, arr, 17, ws, 1 << 30, None) == 2
+    assert b(2, arr, 4, ws, 64, None) == 4                               # workspace too small
+    assert b(2, arr, 0, ws, 1 << 30, None) == 0                          # no tokens: nothing to do
+    arr[1] = FwdProblem(P, C.pointer(w), P, P, 8, 2.0, None)             # a problem without output
+    assert b(2, arr, 4, ws, 1 << 30, None) == 1
+    odd = _weight(rows=100)
+    arr[1] = FwdProblem(P, C.pointer(odd), P, P, 8, 2.0, P)              # N % 8 != 0
+    assert b(2, arr, 4, ws, 1 << 30, None) == 2

@@ -687,3 +687,29 @@ def test_adam_step_on_paged_state():
     for dev_t, paged in ((pd, pp), (md, mp), (vd, vp)):
         assert np.array_equal(dev_t.cpu().numpy().view(np.uint32), paged.numpy().view(np.uint32))
     _check_adam(pp.numpy(), mp.numpy(), vp.numpy(), _adam_oracle(p0, grads, HP), grads)
+
+
+@pytest.mark.parametrize("T", [1, 7, 16])
+def test_decode_grouped_mixed_shapes_and_codebooks(T):
+    """The grouped decode forward over problems of different shapes (ragged
+    rows and k-units), ranks, scales and codebooks (sign-symmetric eq. 2 and the
+    asymmetric INT4 table in one call), each against the oracle."""
+    q = Q()
+    specs = [(40, 320, 8, 0.5, None), (1032, 768, 64, 1.0, INT4_LEVELS), (4096, 4096, 16, 2.0, None),
+             (136, 192, 100, 0.25, None), (2048, 14336, 128, 1.0, INT4_LEVELS)]
+    probs, refs = [], []
+    for i, (N, K, r, s, cb) in enumerate(specs):
+        W, X, A, B, _ = inputs.layer_inputs(99, i, 0, T, N, K, r, device="cuda")
+        table = np.array(cb if cb is not None else O.nf4_codebook(), np.float32)
+        qw = q.quantize_nf4(W, codebook=[float(v) for v in table])
+        codes, scales, c2 = O.quantize_nf4(bits(W), table)
+        assert np.array_equal(qw.codes.cpu().numpy(), codes)
+        wd = O.dequantize_nf4(codes, scales, c2, N, K, table)
+        y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        probs.append((X, qw, A, B, s, y))
+        refs.append(O.linear_fwd(bits(X), wd, bits(A), bits(B), s))
+    q.linear_fwd_decode_batch(probs)
+    q.get_error()
+    torch.cuda.synchronize()
+    for i, (p, ref) in enumerate(zip(probs, refs)):
+        assert_close(f"problem {i}", p[5], ref)

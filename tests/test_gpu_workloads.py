@@ -133,30 +133,46 @@ def test_65b_projection_full_size(layer, proj):
 # --------------------------------------------------------------------------
 # decode sweep: the seven 8B shapes at T = 1, 4, 16, rank 64, s = 1
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("proj", range(7), ids=[p[0] for p in inputs.LLAMA8B_PROJ])
-def test_decode_sweep_projection(proj):
-    """All three token counts of one projection of the decode sweep, seeded as
-    the bench seeds it; every output element against the oracle, through the
-    plain forward and the allocation-free one."""
+@pytest.fixture(scope="module")
+def decode_set():
+    """The decode sweep's seven projections, seeded as the bench seeds them:
+    NF4 weights (quantize checked bit for bit), the oracle's W', adapters."""
+    r = 64
+    out = []
+    for proj, (name, N, K) in enumerate(inputs.LLAMA8B_PROJ):
+        W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(2, 0, proj, "W"), "cuda")
+        qw, wd = quantize_checked(W)
+        del W
+        A = inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(2, 0, proj, "A"), "cuda")
+        B = inputs.normal_bf16((N, r), 0.01, inputs.seed_of(2, 0, proj, "B"), "cuda")
+        out.append((name, N, K, qw, wd, A, B))
+    return out
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_decode_sweep(decode_set, T):
+    """All seven projections of the decode sweep at one token count: every
+    output element against the oracle, through the plain forward, the
+    allocation-free one and the grouped call of all seven at once."""
     q = Q()
-    name, N, K = inputs.LLAMA8B_PROJ[proj]
-    r, s = 64, 1.0
-    W = inputs.normal_bf16((N, K), 0.02, inputs.seed_of(2, 0, proj, "W"), "cuda")
-    qw, wd = quantize_checked(W)
-    del W
-    A = inputs.normal_bf16((r, K), (1.0 / K) ** 0.5, inputs.seed_of(2, 0, proj, "A"), "cuda")
-    B = inputs.normal_bf16((N, r), 0.01, inputs.seed_of(2, 0, proj, "B"), "cuda")
-    for T in (1, 4, 16):
+    s = 1.0
+    xs, ys, ynas, ybs = [], [], [], []
+    for proj, (name, N, K, qw, wd, A, B) in enumerate(decode_set):
         X = inputs.normal_bf16((T, K), 1.0, inputs.seed_of(2, T, proj, "X"), "cuda")
-        y = q.linear_fwd(X, qw, A, B, s)
-        y_na = torch.empty_like(y)
-        q.linear_fwd_noalloc(X, qw, A, B, s, y_na)
-        q.get_error()
-        q.noalloc_get_error()
-        torch.cuda.synchronize()
-        ref = O.linear_fwd(bits(X), wd, bits(A), bits(B), s)
-        assert_close(f"Y T={T}", y, ref)
-        assert_close(f"Y noalloc T={T}", y_na, ref)
+        xs.append(X)
+        ys.append(q.linear_fwd(X, qw, A, B, s))
+        ynas.append(torch.empty_like(ys[-1]))
+        q.linear_fwd_noalloc(X, qw, A, B, s, ynas[-1])
+        ybs.append(torch.full_like(ys[-1], float("nan")))
+    q.linear_fwd_decode_batch([(xs[i], p[3], p[5], p[6], s, ybs[i]) for i, p in enumerate(decode_set)])
+    q.get_error()
+    q.noalloc_get_error()
+    torch.cuda.synchronize()
+    for proj, (name, N, K, qw, wd, A, B) in enumerate(decode_set):
+        ref = O.linear_fwd(bits(xs[proj]), wd, bits(A), bits(B), s)
+        assert_close(f"{name} Y T={T}", ys[proj], ref)
+        assert_close(f"{name} Y noalloc T={T}", ynas[proj], ref)
+        assert_close(f"{name} Y grouped T={T}", ybs[proj], ref)
 
 
 # --------------------------------------------------------------------------
