@@ -344,7 +344,9 @@ qlora_status prepare_gemm(int mode, const qlora_nf4_weight *qw, const void *act,
   // each CTA of a pair loads 128 of the tile's 256 tokens
   if (!make_map_bf16(&g.m_act, act, T, Cext, Cext, 128, 64, true)) return QLORA_ERR_CUDA;
   if (!make_map_bf16(&g.m_lact, lact, T, 2 * r64, 2 * r64, 128, 64, true)) return QLORA_ERR_CUDA;
-  if (!make_map_bf16(&g.m_out, out, T, Mside, Mside, 32, 128, false)) return QLORA_ERR_CUDA;
+  // the forward stores Y by TMA from a swizzled [256 tokens][64 features] tile
+  if (mode == 0 && !make_map_bf16(&g.m_out, out, T, Mside, Mside, 256, 64, true)) return QLORA_ERR_CUDA;
+  if (mode != 0) memset(&g.m_out, 0, sizeof(g.m_out));
   GemmParams &p = g.p;
   memset(&p, 0, sizeof(p));
   p.codes = qw->codes;
@@ -376,13 +378,15 @@ qlora_status prepare_gemm(int mode, const qlora_nf4_weight *qw, const void *act,
 }
 
 qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
-  if (ensure_smem_optin(reinterpret_cast<const void *>(nf4_gemm_2sm_kernel), gemm_2sm_smem_bytes()) !=
-      cudaSuccess)
-    return QLORA_ERR_CUDA;
+  const bool fwd = g.p.mode == 0;
+  const void *func = fwd ? reinterpret_cast<const void *>(nf4_gemm_fwd_2sm_kernel)
+                         : reinterpret_cast<const void *>(nf4_gemm_dx_2sm_kernel);
+  const int smem = fwd ? gemm_fwd_2sm_smem_bytes() : gemm_dx_2sm_smem_bytes();
+  if (ensure_smem_optin(func, smem) != cudaSuccess) return QLORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * g.clusters), 1, 1);
   cfg.blockDim = dim3(576, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(gemm_2sm_smem_bytes());
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -392,9 +396,9 @@ qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   TraceScope ts(g.kid, g.flops, g.bytes, st);
-  return cudaLaunchKernelEx(&cfg, nf4_gemm_2sm_kernel, g.m_act, g.m_lact, g.m_out, g.p) == cudaSuccess
-             ? QLORA_OK
-             : QLORA_ERR_CUDA;
+  const cudaError_t e = fwd ? cudaLaunchKernelEx(&cfg, nf4_gemm_fwd_2sm_kernel, g.m_act, g.m_lact, g.m_out, g.p)
+                            : cudaLaunchKernelEx(&cfg, nf4_gemm_dx_2sm_kernel, g.m_act, g.m_lact, g.p);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 

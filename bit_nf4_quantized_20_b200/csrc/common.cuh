@@ -239,6 +239,14 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                : "memory");
 }
 
+// Ties registers filled by an asynchronous tcgen05.ld to this point of the
+// program: placed after tcgen05.wait::ld, no use of them is moved above it.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 bits, 32 consecutive columns: thread i gets lane (base+i), cols c..c+31.
@@ -263,6 +271,22 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+
+// 32 lanes x 32 bits, 32 consecutive columns: thread i writes lane (base+i), cols c..c+31.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
+      "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]),
+      "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// Wait until every tcgen05.st of this thread has completed.
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Thread block clusters and the 2-SM (cta_group::2) forms
@@ -331,6 +355,19 @@ __device__ __forceinline__ void tc_mma_ss_pair(uint32_t d_tmem, uint64_t a_desc,
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D (+)= A * B^T across a CTA pair with A in tensor memory: each CTA's 128 A
+// rows in its own lanes 0..127 at column a_tmem (K-major, two BF16 per 32-bit
+// column, the lower k in the low half), B from shared memory as above.
+__device__ __forceinline__ void tc_mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -502,5 +539,63 @@ __device__ __forceinline__ void lut8_lookup8(const Lut8 &t, uint32_t w, uint32_t
   o2 = prmt(lo1, hi1, 0x5140u);
   o3 = prmt(lo1, hi1, 0x7362u);
 }
+
+// x >> 16 on the multiply pipe (the high word of x * 2^16)
+__device__ __forceinline__ uint32_t shr16_mul(uint32_t x) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, 65536;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+// Magnitude indices of eight codes (c >= 8 -> c - 8, c < 8 -> 7 - c): the low
+// three bits of each code, flipped where bit 3 is clear; the flip mask
+// (7 in each such nibble) is (~w & 0x88888888) * 7 / 8, a multiply-high.
+__device__ __forceinline__ uint32_t mag_index8_mul(uint32_t w) {
+  uint32_t flip;
+  asm("mul.hi.u32 %0, %1, 0xE0000000;" : "=r"(flip) : "r"(~w & 0x88888888u));
+  return (w ^ flip) & 0x77777777u;
+}
+
+// Eight codes of `w` -> four BF16x2 words (entry(c0), entry(c1)), ..,
+// (entry(c6), entry(c7)) from a sign-symmetric 8-magnitude table (as
+// lut8_lookup8, with the two shifts on the multiply pipe).
+__device__ __forceinline__ void sym_lookup8(const Lut8 &t, uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2,
+                                            uint32_t &o3) {
+  const uint32_t mag = mag_index8_mul(w);
+  const uint32_t magh = shr16_mul(mag);
+  const uint32_t w4 = w * 16u;
+  const uint32_t m_lo = prmt(w4, w, 0xD9C8u);
+  const uint32_t m_hi = prmt(w4, w, 0xFBEAu);
+  const uint32_t lo0 = prmt(t.lo[0], t.lo[1], mag);
+  const uint32_t hi0 = prmt(t.hi[0], t.hi[1], mag) | (~m_lo & 0x80808080u);
+  const uint32_t lo1 = prmt(t.lo[0], t.lo[1], magh);
+  const uint32_t hi1 = prmt(t.hi[0], t.hi[1], magh) | (~m_hi & 0x80808080u);
+  o0 = prmt(lo0, hi0, 0x5140u);
+  o1 = prmt(lo0, hi0, 0x7362u);
+  o2 = prmt(lo1, hi1, 0x5140u);
+  o3 = prmt(lo1, hi1, 0x7362u);
+}
+
+// One 64-weight block's lookup table: eight magnitudes and the sign bit for a
+// sign-symmetric codebook, all sixteen entries otherwise.
+template <bool SYM>
+struct BlockLut;
+template <>
+struct BlockLut<true> {
+  Lut8 t;
+  __device__ __forceinline__ void make(const float (&cb)[16], float s) { t = make_lut8(cb, s); }
+  __device__ __forceinline__ void lookup8(uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2, uint32_t &o3) const {
+    sym_lookup8(t, w, o0, o1, o2, o3);
+  }
+};
+template <>
+struct BlockLut<false> {
+  Lut16 t;
+  __device__ __forceinline__ void make(const float (&cb)[16], float s) { t = make_lut16(cb, s); }
+  __device__ __forceinline__ void lookup8(uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2, uint32_t &o3) const {
+    lut16_lookup4(t, w, o0, o1);
+    lut16_lookup4(t, shr16_mul(w), o2, o3);
+  }
+};
 
 }  // namespace qlora

@@ -81,62 +81,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// x >> 16 on the multiply pipe (the high word of x * 2^16)
-__device__ __forceinline__ uint32_t shr16_mul(uint32_t x) {
-  uint32_t r;
-  asm("mul.hi.u32 %0, %1, 65536;" : "=r"(r) : "r"(x));
-  return r;
-}
-
-// Eight codes of `w` -> four BF16x2 B-fragment words (entry(c0), entry(c1)), ..,
-// (entry(c6), entry(c7)) from a sign-symmetric 8-magnitude table (as
-// lut8_lookup8, with the two shifts on the multiply pipe).
-// Magnitude indices of eight codes (c >= 8 -> c - 8, c < 8 -> 7 - c): the low
-// three bits of each code, flipped where bit 3 is clear; the flip mask
-// (7 in each such nibble) is (~w & 0x88888888) * 7 / 8, a multiply-high.
-__device__ __forceinline__ uint32_t mag_index8_mul(uint32_t w) {
-  uint32_t flip;
-  asm("mul.hi.u32 %0, %1, 0xE0000000;" : "=r"(flip) : "r"(~w & 0x88888888u));
-  return (w ^ flip) & 0x77777777u;
-}
-
-__device__ __forceinline__ void sym_lookup8(const Lut8 &t, uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2,
-                                            uint32_t &o3) {
-  const uint32_t mag = mag_index8_mul(w);
-  const uint32_t magh = shr16_mul(mag);
-  const uint32_t w4 = w * 16u;
-  const uint32_t m_lo = prmt(w4, w, 0xD9C8u);
-  const uint32_t m_hi = prmt(w4, w, 0xFBEAu);
-  const uint32_t lo0 = prmt(t.lo[0], t.lo[1], mag);
-  const uint32_t hi0 = prmt(t.hi[0], t.hi[1], mag) | (~m_lo & 0x80808080u);
-  const uint32_t lo1 = prmt(t.lo[0], t.lo[1], magh);
-  const uint32_t hi1 = prmt(t.hi[0], t.hi[1], magh) | (~m_hi & 0x80808080u);
-  o0 = prmt(lo0, hi0, 0x5140u);
-  o1 = prmt(lo0, hi0, 0x7362u);
-  o2 = prmt(lo1, hi1, 0x5140u);
-  o3 = prmt(lo1, hi1, 0x7362u);
-}
-
-template <bool SYM>
-struct BlockLut;
-template <>
-struct BlockLut<true> {
-  Lut8 t;
-  __device__ __forceinline__ void make(const float (&cb)[16], float s) { t = make_lut8(cb, s); }
-  __device__ __forceinline__ void lookup8(uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2, uint32_t &o3) const {
-    sym_lookup8(t, w, o0, o1, o2, o3);
-  }
-};
-template <>
-struct BlockLut<false> {
-  Lut16 t;
-  __device__ __forceinline__ void make(const float (&cb)[16], float s) { t = make_lut16(cb, s); }
-  __device__ __forceinline__ void lookup8(uint32_t w, uint32_t &o0, uint32_t &o1, uint32_t &o2, uint32_t &o3) const {
-    lut16_lookup4(t, w, o0, o1);
-    lut16_lookup4(t, shr16_mul(w), o2, o3);
-  }
-};
-
 // Position of a unit: problem, 32-row tile within it, 256-code k-unit.
 struct UnitPos {
   int p;

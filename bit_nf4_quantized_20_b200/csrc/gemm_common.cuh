@@ -14,10 +14,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -40,14 +36,6 @@ __device__ __forceinline__ bool named_bar_any(int id, int count, bool pred) {
       : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
       : "memory");
   return r != 0;
-}
-
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
 }
 
 // One 64-weight block's inputs for a dequantizing thread, as loaded: the
@@ -82,27 +70,14 @@ __device__ __forceinline__ BlockIn load_block(const GemmParams &p, int64_t blk, 
 template <bool SYM>
 __device__ __forceinline__ void dequant_row(const float (&cb)[16], const BlockIn &in, uint32_t row_addr,
                                             uint32_t phase) {
-  const float scale = __fmul_rn(e4m3_to_float(in.fbyte), in.c2);
+  BlockLut<SYM> lut;
+  lut.make(cb, __fmul_rn(e4m3_to_float(in.fbyte), in.c2));
   const uint32_t w[8] = {in.c0.x, in.c0.y, in.c0.z, in.c0.w, in.c1.x, in.c1.y, in.c1.z, in.c1.w};
-  if (SYM) {
-    const Lut8 lut = make_lut8(cb, scale);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t o0, o1, o2, o3;
-      const uint32_t mag = mag_index8(w[c]);
-      lut8_lookup4(lut, w[c], mag, o0, o1);
-      lut8_lookup4(lut, w[c] >> 16, mag >> 16, o2, o3);
-      st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
-    }
-  } else {
-    const Lut16 lut = make_lut16(cb, scale);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t o0, o1, o2, o3;
-      lut16_lookup4(lut, w[c], o0, o1);
-      lut16_lookup4(lut, w[c] >> 16, o2, o3);
-      st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
-    }
+  for (int c = 0; c < 8; ++c) {
+    uint32_t o0, o1, o2, o3;
+    lut.lookup8(w[c], o0, o1, o2, o3);
+    st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ phase) << 4), o0, o1, o2, o3);
   }
 }
 

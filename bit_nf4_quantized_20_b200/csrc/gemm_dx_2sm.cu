@@ -1,39 +1,39 @@
-// gemm_nf4_2sm.cu -- the fused NF4 dequantization + tcgen05 GEMM on CTA pairs
-// (2-SM UMMA, cta_group::2), forward and backward-dX.
+// gemm_dx_2sm.cu -- the gradient through the frozen weight, fused NF4
+// dequantization + tcgen05 GEMM on CTA pairs (2-SM UMMA, cta_group::2):
 //
-//   forward   Y[T, N]  = X[T, K] W'[N, K]^T + (s X A^T)[T, r] B[N, r]^T
-//   backward  dX[T, K] = dY[T, N] W'[N, K] + (s dY B)[T, r] A[r, K]
+//   dX[T, K] = dY[T, N] W'[N, K] + (s dY B)[T, r] A[r, K]
 //
-// The rank-r operand (s X A^T, or s dY B) arrives as two BF16 planes, hi and
-// lo = bf16(v - hi), each as its own run of 64-wide stages against the same
-// B (or A) rows, so the rank-r term carries about 16 significant bits of it.
+// ("QLoRA: Efficient Fine-Tuning", Step 4: the backward pass needs the
+// gradient with respect to the input through W', which is dequantized on the
+// fly as in the forward, "What is QLoRA?".)  The rank-r operand dU = s dY B
+// arrives as two BF16 planes, hi and lo = bf16(v - hi), each its own run of
+// 64-wide stages against the same A columns.
 //
-// ("QLoRA: Efficient Fine-Tuning", Step 3 eq. 3 and Step 4; W' is produced in
-// shared memory by dequantization warps, "converted to BF16 on the fly for each
-// matrix multiplication", "What is QLoRA?".)
-//
-// A cluster of two CTAs on two SMs owns a 256-weight-row x 256-token tile.
-// Each CTA dequantizes its own 128 weight rows (the MMA's A operand) and
-// TMA-loads its own 128 tokens (half of the B operand); the even CTA issues
-// tcgen05.mma.cta_group::2 (M = 256, N = 256), which reads both CTAs' halves
-// and accumulates each CTA's 128 rows x 256 tokens in that CTA's tensor memory.
-// Compared with one CTA per 128 x 256 tile this halves the token operand each
-// SM streams from L2 per FLOP.
+// A cluster of two CTAs on two SMs owns a 256-column (of W, i.e. of dX) x
+// 256-token tile.  The contraction runs over the N rows of W, so each CTA's A
+// operand is W'^T: its dequantization threads turn 128 64-weight blocks (64
+// rows of W x two 64-column blocks) into an MN-major, 128-byte-swizzled
+// shared-memory tile; TMA loads this CTA's 128 tokens of dY (then of the dU
+// planes) as the B half; the even CTA issues tcgen05.mma.cta_group::2 (M = 256,
+// N = 256) accumulating each CTA's 128 columns x 256 tokens in its own tensor
+// memory, two accumulators of 256 columns so that the epilogue of one tile
+// overlaps the next tile's MMAs.
 //
 // Warp roles (576 threads per CTA, one CTA per SM, persistent over tiles):
-//   warps 0-3   epilogue: tensor memory -> BF16 -> global memory, a pair of features
+//   warps 0-3   epilogue: tensor memory -> BF16 -> global memory, a pair of columns
 //               per 32-bit store (each store instruction writes 64 contiguous bytes
 //               for each of two tokens)
 //   warps 4-15  dequantization in three groups of four warps; group g fills the
 //               pipeline stages it with it % 3 == g
-//   warp 16     TMA loads of this CTA's token half (X / dY, then s*U / dU)
+//   warp 16     TMA loads of this CTA's token half (dY, then the dU planes)
 //   warp 17     paired tensor-memory allocation; on the even CTA, the MMA issue
 // Pipeline barriers: full[s] lives in the even CTA and counts both CTAs' TMA
-// bytes (armed by the even CTA) and both CTAs' dequantization warps; empty[s] and acc_full are signalled in both
-// CTAs by a multicast tcgen05.commit; acc_empty (even CTA) counts both CTAs'
-// epilogue warps.  Every wait is bounded; after a timeout each role stops
-// issuing work, drains what it issued, and both CTAs meet at the final cluster
-// barrier before the tensor memory is freed.
+// bytes (armed by the even CTA) and both CTAs' dequantization warps; empty[s]
+// and acc_full are signalled in both CTAs by a multicast tcgen05.commit;
+// acc_empty (even CTA) counts both CTAs' epilogue warps.  Every wait is
+// bounded; after a timeout each role stops issuing work, drains what it
+// issued, and both CTAs meet at the final cluster barrier before the tensor
+// memory is freed.
 
 #include "common.cuh"
 #include "gemm_common.cuh"
@@ -45,7 +45,7 @@ using namespace gemm;
 
 namespace {
 
-constexpr int PM = 128;                        // weight rows per CTA (256 per pair)
+constexpr int PM = 128;                        // columns of W per CTA (256 per pair)
 constexpr int PN = 256;                        // tokens per tile
 constexpr int HN = 128;                        // tokens loaded by each CTA
 constexpr int BK = 64;
@@ -54,7 +54,7 @@ constexpr int A_BYTES = PM * BK * 2;           // 16 KiB
 constexpr int B_BYTES = HN * BK * 2;           // 16 KiB
 constexpr int EPI_ROWS = 32;
 constexpr int NUM_THREADS = 576;
-constexpr int DQ_GROUPS = 3;          // STAGES is a multiple of it
+constexpr int DQ_GROUPS = 3;
 constexpr int TMEM_COLS = 512;
 
 constexpr int OFF_A = 0;
@@ -85,8 +85,8 @@ struct Smem {
 }  // namespace
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lact,
-                        const __grid_constant__ CUtensorMap tmap_out, const GemmParams p) {
+    nf4_gemm_dx_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lact,
+                           const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem sm;
   sm.base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -94,11 +94,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const bool bwd = p.mode != 0;
   const uint32_t rank = cluster_ctarank();          // 0: leader (issues the MMAs), 1: peer
   const bool leader = rank == 0;
   const int ksteps = p.k_main + p.k_lora;
-  const int m_pairs = p.m_tiles;                     // 256-row weight tiles
+  const int m_pairs = p.m_tiles;                     // 256-column tiles of W
   const int num_tiles = m_pairs * p.n_tiles;
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
@@ -134,30 +133,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 17) {
     // ---------------- MMA issuer (even CTA) ----------------
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, bwd, false);
+      // The issuing thread shares its scheduler with three dequantization
+      // warps, so each stage costs it as few instructions as possible: the
+      // descriptors of stage s, slice kk are the stage-0 ones plus constant
+      // offsets in the address field (A MN-major: a 16-row slice is 4096
+      // bytes on; B K-major: 32 bytes on), which cannot carry out since
+      // shared addresses stay below 256 KiB.
+      const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, true, false);
+      const uint64_t adesc0 = smem_desc_sw128(sm.a(0), 1024, 2048);
+      const uint64_t bdesc0 = smem_desc_sw128(sm.b(0), 16, 1024);
+      // 16-wide K slices of the last rank-r stage of a plane that hold any of
+      // the r rows of A (the slices past them multiply zeros and are skipped)
+      const int nk_tail = min(4, (p.r - (p.k_lora_plane - 1) * BK + 15) / 16);
       int it = 0, tc = 0;
       bool ok = true;
+      auto stage = [&](uint32_t d_tmem, int nk, uint32_t accumulate) -> bool {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(sm.full(s), ph, p.status)) return false;
+        tc_fence_after();
+        const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (B_BYTES >> 4));
+        tc_mma_ss_pair(d_tmem, ad, bd, idesc, accumulate);
+#pragma unroll
+        for (int kk = 1; kk < 4; ++kk)
+          if (kk < nk) tc_mma_ss_pair(d_tmem, ad + kk * (4096 >> 4), bd + kk * (32 >> 4), idesc, 1u);
+        tc_commit_pair_mc(sm.empty(s), 0x3);
+        ++it;
+        return true;
+      };
       for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
         const int acc = tc & 1;
         const uint32_t acc_phase = (tc >> 1) & 1;
         if (!mbar_wait(sm.acc_empty(acc), acc_phase ^ 1, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PN);
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(sm.full(s), ph, p.status)) { ok = false; break; }
-          tc_fence_after();
-          int nk = 4;
-          if (ks >= p.k_main) nk = min(4, (p.r - ((ks - p.k_main) % p.k_lora_plane) * BK + 15) / 16);
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t adesc = !bwd ? smem_desc_sw128(sm.a(s) + kk * 32, 16, 1024)        // K-major
-                                        : smem_desc_sw128(sm.a(s) + kk * 4096, 1024, 2048);   // MN-major
-            const uint64_t bdesc = smem_desc_sw128(sm.b(s) + kk * 32, 16, 1024);
-            tc_mma_ss_pair(d_tmem, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit_pair_mc(sm.empty(s), 0x3);
-        }
+        for (int ks = 0; ks < p.k_main && ok; ++ks) ok = stage(d_tmem, 4, ks > 0 ? 1u : 0u);
+        for (int pl = 0; pl < 2 && ok; ++pl)
+          for (int l = 0; l < p.k_lora_plane && ok; ++l)
+            ok = stage(d_tmem, l == p.k_lora_plane - 1 ? nk_tail : 4, 1u);
         if (!ok) break;
         tc_commit_pair_mc(sm.acc_full(acc), 0x3);
       }
@@ -199,42 +213,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ---------------- dequantization: three groups, rotating stages ----------------
+    // Thread t of a group dequantizes block (row ks * 64 + t % 64 of W, column
+    // block t / 64 of the CTA's two) into row t % 64 of the MN-major tile half
+    // t / 64: 128-byte rows, 8-row swizzle atoms of 1 KiB, the two halves'
+    // atoms interleaved.
     const int grp = (warp - 4) >> 2;                 // group g fills stages it % 3 == g
     const int tid = threadIdx.x - 128 - 128 * grp;   // 0..127
+    const int rho = tid & 63, h = tid >> 6;
     float cb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) cb[i] = p.codebook[i];
     const int64_t kblocks = p.K / 64;
-    uint32_t row_off, phase;
-    if (!bwd) {
-      row_off = (tid >> 3) * 1024 + (tid & 7) * 128;
-      phase = tid & 7;
-    } else {
-      const int rho = tid & 63, h = tid >> 6;
-      row_off = ((rho >> 3) * 2 + h) * 1024 + (rho & 7) * 128;
-      phase = rho & 7;
-    }
+    const uint32_t row_off = static_cast<uint32_t>(((rho >> 3) * 2 + h) * 1024 + (rho & 7) * 128);
+    const uint32_t phase = static_cast<uint32_t>(rho & 7);
     int it_base = 0;
     bool ok = true;
     for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
       const int m_pair = tile % m_pairs;
-      const int64_t row0 = static_cast<int64_t>(m_pair) * 2 * PM + static_cast<int64_t>(rank) * PM;
-      auto block_of = [&](int ks, int64_t &blk) -> bool {
-        int64_t n, kb;
-        if (!bwd) {
-          n = row0 + tid;
-          kb = ks;
-        } else {
-          n = static_cast<int64_t>(ks) * BK + (tid & 63);
-          kb = row0 / 64 + (tid >> 6);
-        }
-        blk = n * kblocks + kb;
-        return n < p.N && kb < kblocks;
-      };
+      const int64_t col0 = static_cast<int64_t>(m_pair) * 2 * PM + static_cast<int64_t>(rank) * PM;
+      const int64_t kb = col0 / 64 + h;              // this thread's column block of W
+      const bool kb_ok = kb < kblocks;
       auto fetch = [&](int ks) -> BlockIn {
-        int64_t blk = 0;
-        const bool v = ks < p.k_main && block_of(ks, blk);
-        return load_block(p, blk, v);
+        const int64_t n = static_cast<int64_t>(ks) * BK + rho;
+        return load_block(p, n * kblocks + kb, ks < p.k_main && n < p.N && kb_ok);
       };
       auto produce = [&](int ks, BlockIn &buf) -> bool {
         const int it = it_base + ks;
@@ -246,21 +247,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (p.sym) dequant_row<true>(cb, buf, row_addr, phase);
           else dequant_row<false>(cb, buf, row_addr, phase);
         } else {
-          // rank-r stage: the same B (forward) or A (backward) rows for the hi
-          // and the lo plane of sU / dU
-          const int l = (ks - p.k_main) % p.k_lora_plane;
-          if (!bwd) {
-            const int64_t n = row0 + tid;
-            const int nv = (n < p.N) ? max(0, min(BK, p.r - l * BK)) : 0;
-            const uint16_t *src = p.lora + (n < p.N ? n : 0) * p.r + l * BK;
-            copy_row(src, nv, (p.r % 8) == 0, row_addr, phase);
-          } else {
-            const int j = l * BK + (tid & 63);
-            const int64_t k0 = row0 + (tid >> 6) * 64;
-            const int nv = (j < p.r && k0 < p.K) ? 64 : 0;
-            const uint16_t *src = p.lora + static_cast<int64_t>(j < p.r ? j : 0) * p.K + (k0 < p.K ? k0 : 0);
-            copy_row(src, nv, true, row_addr, phase);
-          }
+          // rank-r stage: row j of A (64 columns of the CTA's block) for the hi
+          // and the lo plane of dU alike
+          const int j = ((ks - p.k_main) % p.k_lora_plane) * BK + rho;
+          const int64_t k0 = kb * 64;
+          const int nv = (j < p.r && kb_ok) ? 64 : 0;
+          const uint16_t *src = p.lora + static_cast<int64_t>(j < p.r ? j : 0) * p.K + (kb_ok ? k0 : 0);
+          copy_row(src, nv, true, row_addr, phase);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -282,7 +275,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue (warps 0-3) ----------------
     const int q = warp;
-    const int64_t m_side = bwd ? p.K : p.N;
     int tc = 0;
     bool ok = true;
     for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
@@ -295,15 +287,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * PN);
       const int m_local = q * 32 + static_cast<int>(lane);
-      const int feat0 = m_pair * 2 * PM + static_cast<int>(rank) * PM;
-      // lanes 2i and 2i + 1 hold features f and f + 1 (f even); after one exchange
-      // the even lane stores both features of token j, the odd lane those of j + 1
-      const int64_t col = static_cast<int64_t>(feat0) + (m_local & ~1);
+      const int col_base = m_pair * 2 * PM + static_cast<int>(rank) * PM;
+      // lanes 2i and 2i + 1 hold columns c and c + 1 (c even); after one exchange
+      // the even lane stores both columns of token j, the odd lane those of j + 1
+      const int64_t col = static_cast<int64_t>(col_base) + (m_local & ~1);
       const bool odd = (lane & 1) != 0;
       for (int ch = 0; ch < PN / EPI_ROWS; ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + ch * EPI_ROWS, r);
         tc_wait_ld();
+        reg_fence(r);
         if (ch == PN / EPI_ROWS - 1) {
           tc_fence_before();
           __syncwarp();
@@ -317,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float recv = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
           const int64_t tok = tok0 + j + (odd ? 1 : 0);
           // the row stride is a multiple of 8: an even column below it has its pair too
-          if (tok < p.T && col < m_side) {
+          if (tok < p.T && col < p.K) {
             const __nv_bfloat162 v = __floats2bfloat162_rn(odd ? recv : a, odd ? b : recv);
             *reinterpret_cast<__nv_bfloat162 *>(p.out + tok * p.ldo + col) = v;
           }
@@ -336,6 +329,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-int gemm_2sm_smem_bytes() { return SMEM_ALLOC; }
+int gemm_dx_2sm_smem_bytes() { return SMEM_ALLOC; }
 
 }  // namespace qlora

@@ -48,7 +48,7 @@ cudaError_t launch_adam(float *param, float *m, float *v, const uint16_t *grad, 
                         const AdamArgs &a, cudaStream_t st, int num_sms);
 
 // ---------------------------------------------------------------------------
-// fused NF4 GEMM on CTA pairs (gemm_nf4_2sm.cu)
+// fused NF4 GEMMs on CTA pairs (gemm_fwd_2sm.cu, gemm_dx_2sm.cu)
 // ---------------------------------------------------------------------------
 struct GemmParams {
   const uint8_t *codes;
@@ -65,14 +65,20 @@ struct GemmParams {
   int k_lora_plane;        // rank-r stages per plane (k_lora = 2 k_lora_plane)
   int sym;                 // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
   uint32_t *status;
-  uint16_t *out;           // Y [T, N] or dX [T, K], stored from registers
+  uint16_t *out;           // Y [T, N] (stored by TMA through tmap_out) or dX [T, K] (from registers)
   int64_t ldo;             // its row stride (N or K)
 };
-int gemm_2sm_smem_bytes();
-// launched as clusters of 2 CTAs
-__global__ void nf4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
-                                    const __grid_constant__ CUtensorMap tmap_lact,
-                                    const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
+// Launched as clusters of 2 CTAs, one CTA per SM, persistent over the tiles.
+// The forward (mode 0), A from tensor memory; tmap_out: Y [T, N], box [256
+// tokens][64 features], 128-byte swizzle (gemm_fwd_2sm.cu).
+int gemm_fwd_2sm_smem_bytes();
+__global__ void nf4_gemm_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                                        const __grid_constant__ CUtensorMap tmap_lact,
+                                        const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
+// The backward dX (mode 1), A = W'^T from shared memory (gemm_dx_2sm.cu).
+int gemm_dx_2sm_smem_bytes();
+__global__ void nf4_gemm_dx_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                                       const __grid_constant__ CUtensorMap tmap_lact, const GemmParams p);
 
 // ---------------------------------------------------------------------------
 // decode-sized forward of one or several projections (decode.cu)
