@@ -110,33 +110,6 @@ int num_sms_current() {
   return cache[dev];
 }
 
-// A second stream (and its fork / join events) per host thread and device: the
-// backward runs its adapter-gradient products there, beside the dX GEMM, whose
-// last partial round of tiles leaves SMs idle.  Created on first use, kept
-// until exit; nullptr if the device refuses (the caller then stays on one stream).
-struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-  bool tried = false;
-};
-
-SideStream *side_stream() {
-  thread_local SideStream cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  SideStream &ss = cache[dev];
-  if (!ss.tried) {
-    ss.tried = true;
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
-      ss.s = nullptr;
-      (void)cudaGetLastError();
-    }
-  }
-  return ss.s ? &ss : nullptr;
-}
-
 // Splits of the rank-r GEMMs are sized for a fixed CTA target so that the
 // workspace size does not depend on the device.
 constexpr int kSplitSms = 148;
@@ -388,13 +361,18 @@ qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   cfg.blockDim = dim3(576, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  // a programmatic dependent of the rank-r kernel before it: only the loads of
+  // that kernel's planes wait for it (no trace attached: with one, each launch
+  // runs alone between its events)
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = g_trace.recs == nullptr ? 2 : 1;
   TraceScope ts(g.kid, g.flops, g.bytes, st);
   const cudaError_t e = fwd ? cudaLaunchKernelEx(&cfg, nf4_gemm_fwd_2sm_kernel, g.m_act, g.m_lact, g.m_out, g.p)
                             : cudaLaunchKernelEx(&cfg, nf4_gemm_dx_2sm_kernel, g.m_act, g.m_lact, g.p);
@@ -898,27 +876,21 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
   GemmLaunch gl;
   rs = prepare_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), gl);
   if (rs != QLORA_OK) return rs;
-  // the second grid needs only the first's planes, not dX, so it runs on the
-  // side stream beside the dX GEMM (which touches no other workspace than the
-  // status word) and joins before return; with a trace attached everything
-  // stays on the caller's stream, so that each launch's events time that
-  // launch alone
-  SideStream *side = g_trace.recs == nullptr ? side_stream() : nullptr;
+  // The second grid needs only the first's planes, not dX: it follows the dX
+  // GEMM as a programmatic dependent that waits for the GEMM only before it
+  // exits, so that it runs on the SMs the GEMM's last round of tiles leaves
+  // idle.  (The GEMM lets it start after the first grid has completed.)
+  second.a0.dep_late = 1;
+  second.a1.dep_late = 1;
 
   if (pad_b && launch_pad_cols(static_cast<const uint16_t *>(B), N, r, plane(L.bpad), static_cast<int>(r64), st,
                                num_sms_current()) != cudaSuccess)
     return QLORA_ERR_CUDA;
   rs = launch_tc(first, st);
   if (rs != QLORA_OK) return rs;
-  if (side && cudaEventRecord(side->fork, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  rs = launch_gemm(gl, st);   // first in line for the SMs
+  rs = launch_gemm(gl, st);
   if (rs != QLORA_OK) return rs;
-  if (!side) return launch_tc(second, st);
-  if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
-  rs = launch_tc(second, side->s);
-  if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  return rs;
+  return launch_tc(second, st);
 }
 
 static qlora_status linear_bwd_entry(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,

@@ -155,6 +155,18 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library keeps one rule:
+// it waits for the preceding kernel of its stream (griddepcontrol.wait) before
+// it completes and before it touches anything that kernel writes, and it lets
+// its own dependents launch (griddepcontrol.launch_dependents) only after
+// that wait.  A kernel that starts early can therefore rely on everything
+// before its predecessor having completed; only the predecessor's own outputs
+// need the wait.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Proxy fences
 // ---------------------------------------------------------------------------
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA store,

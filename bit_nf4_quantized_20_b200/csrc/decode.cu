@@ -79,8 +79,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // Position of a unit: problem, 32-row tile within it, 256-code k-unit.
 struct UnitPos {
   int p;
@@ -143,6 +141,7 @@ template <int NB>
 __device__ __forceinline__ void finish_tile(const DecodeArgs &a, const UnitPos &u, int g, int t,
                                             float (&v)[2][NB][4]) {
   grid_dep_wait();   // U' comes from the preceding kernel (returns at once after the first call)
+  grid_dep_launch();
   const DecodeProblem &P = a.prob[u.p];
   const int T = a.T;
   const int64_t row0 = u.tile * DT;
@@ -273,12 +272,14 @@ __global__ void __launch_bounds__(DW * 32, 2) decode_gemv_kernel(const __grid_co
   // the first unit's scales (static too)
   ScalePre sp = load_scales(a.prob[cur.p], cur.tile * DT, static_cast<int64_t>(cur.ku) * 4 + t, g);
   __syncthreads();                          // the shared counters are zero
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // X, Y and the workspace may depend on earlier kernels.  After a decode U'
   // kernel (which lets this grid start only once everything before it has
   // completed) only U' may still be in flight, and it is read after its own
   // wait in finish_tile; otherwise wait here.
-  if (!a.early_start) grid_dep_wait();
+  if (!a.early_start) {
+    grid_dep_wait();
+    grid_dep_launch();
+  }
 
   constexpr int NB = T16 ? 2 : 1;   // token halves (MMA N = 8 each)
   float cb[16];
@@ -461,6 +462,9 @@ __global__ void __launch_bounds__(DW * 32, 2) decode_gemv_kernel(const __grid_co
       mbar_wait(bars + 8 * (i2 % DS), static_cast<uint32_t>((i2 / DS) & 1), a.status);
     }
   }
+  // warps that finished no tile have not waited yet
+  grid_dep_wait();
+  grid_dep_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(kUThreads, 1) decode_u_kernel(const __grid_con
   grid_dep_wait();   // X may be written by the preceding kernel, U' read by it
   // every kernel before this one has now completed: the GEMV that follows may
   // start (and read X, the weights and its workspace) while U' is computed
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dep_launch();
   for (int c = threadIdx.x; c < TT * chunks; c += kUThreads) {
     const int tok = c / chunks, q = c % chunks;
     const bool ok = tok < args.T && 8 * q < klen;

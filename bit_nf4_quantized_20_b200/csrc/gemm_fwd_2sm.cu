@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- TMA producer: this CTA's token half ----------------
     if (lane == 0) {
       int it = 0;
-      bool ok = true;
+      bool ok = true, dep_done = false;
       for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
         const int n_tile = tile / m_pairs;
         const int t0 = n_tile * PN + static_cast<int>(rank) * HN;
@@ -224,9 +224,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // load only completes transactions on it
           const uint32_t fb = lead(sm.full(s));
           if (leader) mbar_arrive_expect_tx(sm.full(s), 2 * B_BYTES);
-          if (ks < p.k_main) tma_load_2d_pair(sm.b(s), &tmap_act, fb, ks * BK, t0);
-          else tma_load_2d_pair(sm.b(s), &tmap_lact, fb, (ks - p.k_main) * BK, t0);
+          if (ks < p.k_main) {
+            tma_load_2d_pair(sm.b(s), &tmap_act, fb, ks * BK, t0);
+          } else {
+            // the rank-r planes are the preceding kernel's output
+            if (!dep_done) {
+              grid_dep_wait();
+              grid_dep_launch();
+              dep_done = true;
+            }
+            tma_load_2d_pair(sm.b(s), &tmap_lact, fb, (ks - p.k_main) * BK, t0);
+          }
         }
+      }
+      if (!dep_done) {
+        grid_dep_wait();
+        grid_dep_launch();
       }
       if (!ok) {
         s_abort = 1;

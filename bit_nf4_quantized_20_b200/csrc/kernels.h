@@ -176,6 +176,9 @@ struct SkinnyTcArgs {
   float *partials;       // [splits][M][(R + 3) & ~3] when splits > 1
   uint32_t *counters;    // one per 128-row tile (zero on entry, zero on exit)
   uint32_t *status;
+  int dep_late;          // every input was complete when the preceding kernel let this one
+                         // start: wait for that kernel only before exiting (same in both
+                         // products of a pair launch)
 };
 cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
                              const CUtensorMap &tm_q1, cudaStream_t st, bool pdl);

@@ -19,7 +19,10 @@
 //
 // Launched as a programmatic dependent: the prologue (barriers, tensor memory,
 // descriptor prefetch) overlaps the previous kernel, and every global access
-// comes after griddepcontrol.wait.
+// comes after griddepcontrol.wait -- except in a launch whose inputs all come
+// from kernels that had completed before its predecessor let it start (the
+// adapter gradients after the dX GEMM: dep_late), which waits only before it
+// exits, so that it can run in the GEMM's last wave.
 //
 // Warps: 0 TMA producer, 1 tensor-memory allocation + MMA issue, 2-5 epilogue.
 
@@ -42,9 +45,6 @@ constexpr int kBarBytes = 8 * (2 * TMAX_STAGES + 1) + 8;   // full[], empty[], a
 constexpr int kFixedSmem = kBarBytes + 1024;               // + alignment slack for the 1 KiB swizzle atoms
 constexpr int kTwoPerSmBudget = 110 * 1024;
 constexpr int kOnePerSmBudget = 220 * 1024;
-
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Columns c0 .. c0 + CW - 1 of row m: v[j] is the un-scaled accumulator.
 template <int CW>
@@ -152,7 +152,10 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ld_shared_u32(tmem_slot);
-  grid_dep_wait();
+  if (!a.dep_late) {
+    grid_dep_wait();
+    grid_dep_launch();
+  }
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -316,6 +319,10 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
     }
   }
 
+  if (a.dep_late) {
+    grid_dep_wait();
+    grid_dep_launch();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -328,7 +335,6 @@ template <int NB>
 __global__ void __launch_bounds__(TNUM_THREADS, 2)
     skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q0,
                      const __grid_constant__ CUtensorMap tm_q1, const SkinnyTcArgs a) {
-  grid_dep_launch();
   skinny_tc_body<NB>(&tm_p, &tm_q0, &tm_q1, a, static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y));
 }
 
@@ -340,7 +346,6 @@ __global__ void __launch_bounds__(TNUM_THREADS, 2)
                           const __grid_constant__ CUtensorMap tm_q10, const __grid_constant__ CUtensorMap tm_p1,
                           const __grid_constant__ CUtensorMap tm_q01, const __grid_constant__ CUtensorMap tm_q11,
                           const SkinnyTcArgs a0, const SkinnyTcArgs a1) {
-  grid_dep_launch();
   const int mt0 = static_cast<int>((a0.M + TBM - 1) / TBM);
   const int n0 = mt0 * a0.splits;
   const int b = static_cast<int>(blockIdx.x);

@@ -24,11 +24,17 @@
  *     unified memory).  The library allocates and frees device memory only in
  *     qlora_paged_alloc / qlora_paged_free, which a caller calls explicitly for
  *     optimizer state; its only other device state is the fixed scratch array
- *     of qlora_linear_fwd_noalloc (a static symbol).  Its host state is one
- *     side stream per host thread and device (backward).
+ *     of qlora_linear_fwd_noalloc (a static symbol).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).  Work
  *     is enqueued on it and the call returns after validating the arguments;
  *     results are ready when the stream reaches that point.
+ *   - Kernels are launched as programmatic dependents (they may start while
+ *     the preceding kernel of the stream finishes).  Each waits for that
+ *     kernel before it completes and before it touches anything that kernel
+ *     writes, and lets its own dependents start only after that wait; a
+ *     caller's kernel that follows a library call on the stream sees all of
+ *     the call's results, as usual.
+ *   - Outputs must not overlap the call's inputs or each other.
  *   - Row-major layouts.  BF16 tensors are arrays of uint16 bit patterns.
  *   - Every check (arguments, alignment, workspace, TMA descriptor encoding)
  *     runs before the first enqueue: a call that returns INVALID_ARG,
@@ -212,11 +218,8 @@ QLORA_API qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf
  * dy[T, N], x[T, K], A[r, K], B[N, r]; outputs dx[T, K], dA[r, K], dB[N, r]
  * (BF16, overwritten, not accumulated).  Same requirements as the forward.
  * ws: at least qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r) bytes.
- * Streams: all work is ordered on `stream`; dB and dA are computed on a
- * library-owned second stream (one per host thread and device, forked from and
- * joined back into `stream` with events, so graph capture of `stream` captures
- * it too) beside the dX GEMM.  With a trace attached everything runs on
- * `stream`.
+ * Streams: all work is ordered on `stream`; the grid computing dB and dA
+ * follows the dX GEMM and runs on the SMs its last round of tiles leaves idle.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.
  */
 QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,

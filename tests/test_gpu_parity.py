@@ -441,8 +441,9 @@ def test_layer_saved_u(T, N, K, r, s):
 
 
 def test_backward_saved_graph_capture_matches_eager():
-    """The saved-U backward also forks its second grid onto the side stream;
-    captured in a CUDA graph it gives the eager results bit for bit."""
+    """The saved-U backward (its adapter-gradient grid a programmatic
+    dependent of the dX GEMM), captured in a CUDA graph on a non-default
+    stream, gives the eager results bit for bit."""
     q = Q()
     T, N, K, r, s = 512, 1024, 768, 16, 2.0
     W, X, A, B, dY = inputs.layer_inputs(94, 0, 0, T, N, K, r, device="cuda")
