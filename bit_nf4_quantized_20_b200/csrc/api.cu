@@ -302,7 +302,7 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
 // The fused GEMM's launch, prepared (tensor maps encoded, parameters filled)
 // before anything of the call is enqueued.
 struct GemmLaunch {
-  CUtensorMap m_act, m_lact, m_out;
+  CUtensorMap m_act, m_lact, m_act_h, m_lact_h, m_out;
   GemmParams p;
   int64_t clusters;
   int32_t kid;
@@ -314,11 +314,13 @@ qlora_status prepare_gemm(int mode, const qlora_nf4_weight *qw, const void *act,
   const int64_t N = qw->rows, K = qw->cols;
   const int64_t Mside = mode == 0 ? N : K;     // weight-side extent
   const int64_t Cext = mode == 0 ? K : N;      // contraction extent
-  // each CTA of a pair loads 128 of the tile's 256 tokens
+  // each CTA of a pair loads 128 of a tile's 256 tokens (64 of a half tile's 128)
   if (!make_map_bf16(&g.m_act, act, T, Cext, Cext, 128, 64, true)) return QLORA_ERR_CUDA;
   if (!make_map_bf16(&g.m_lact, lact, T, 2 * r64, 2 * r64, 128, 64, true)) return QLORA_ERR_CUDA;
-  // the forward stores Y by TMA from a swizzled [256 tokens][64 features] tile
-  if (mode == 0 && !make_map_bf16(&g.m_out, out, T, Mside, Mside, 256, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&g.m_act_h, act, T, Cext, Cext, 64, 64, true)) return QLORA_ERR_CUDA;
+  if (!make_map_bf16(&g.m_lact_h, lact, T, 2 * r64, 2 * r64, 64, 64, true)) return QLORA_ERR_CUDA;
+  // the forward stores Y by TMA from a swizzled staging tile, 128 tokens x 64 features a box
+  if (mode == 0 && !make_map_bf16(&g.m_out, out, T, Mside, Mside, 128, 64, true)) return QLORA_ERR_CUDA;
   if (mode != 0) memset(&g.m_out, 0, sizeof(g.m_out));
   GemmParams &p = g.p;
   memset(&p, 0, sizeof(p));
@@ -346,6 +348,11 @@ qlora_status prepare_gemm(int mode, const qlora_nf4_weight *qw, const void *act,
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   const int sms = num_sms_current();
   g.clusters = tiles < sms / 2 ? tiles : sms / 2;
+  // a last round at most half full runs its tiles as 128-token halves
+  const int64_t rounds = tiles / g.clusters, rem = tiles - rounds * g.clusters;
+  const bool halves = rem > 0 && rounds >= 1 && 2 * rem <= g.clusters;
+  p.units_full = static_cast<int>(halves ? tiles - rem : tiles);
+  p.units = static_cast<int>(halves ? tiles + rem : tiles);
   g.kid = mode == 0 ? K_GEMM_FWD : K_GEMM_BWD;
   return QLORA_OK;
 }
@@ -374,8 +381,9 @@ qlora_status launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = g_trace.recs == nullptr ? 2 : 1;
   TraceScope ts(g.kid, g.flops, g.bytes, st);
-  const cudaError_t e = fwd ? cudaLaunchKernelEx(&cfg, nf4_gemm_fwd_2sm_kernel, g.m_act, g.m_lact, g.m_out, g.p)
-                            : cudaLaunchKernelEx(&cfg, nf4_gemm_dx_2sm_kernel, g.m_act, g.m_lact, g.p);
+  const cudaError_t e =
+      fwd ? cudaLaunchKernelEx(&cfg, nf4_gemm_fwd_2sm_kernel, g.m_act, g.m_lact, g.m_act_h, g.m_lact_h, g.m_out, g.p)
+          : cudaLaunchKernelEx(&cfg, nf4_gemm_dx_2sm_kernel, g.m_act, g.m_lact, g.m_act_h, g.m_lact_h, g.p);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -357,29 +357,36 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
 
-// D (+)= A * B^T across a CTA pair: A rows split 128/128 between the two CTAs'
-// shared memory (same offset), B rows (the N operand) split likewise, D in
-// both CTAs' tensor memory.  Issued by the leader (even rank) only.
-__device__ __forceinline__ void tc_mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                               uint32_t accumulate) {
+// D (+)= A * B^T across a CTA pair, issued by the leader (even rank) only,
+// kind::f16 (BF16 inputs, FP32 accumulate), D in both CTAs' tensor memory:
+// each CTA holds 128 of A's 256 rows and half of B's rows (the N operand).
+//   _ts: A in tensor memory (each CTA's 128 rows in its lanes 0..127 at column
+//        a_tmem, K-major, two BF16 per 32-bit column, the lower k in the low
+//        half), B from shared memory;
+//   _ss: A and B from shared memory.
+// Shared-memory descriptors are passed as 32-bit halves: only the low half,
+// which holds the start address, changes from stage to stage, so a stage
+// costs the issuing thread 32-bit adds.
+__device__ __forceinline__ void tc_mma_ts_pair_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                                  uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// D (+)= A * B^T across a CTA pair with A in tensor memory: each CTA's 128 A
-// rows in its own lanes 0..127 at column a_tmem (K-major, two BF16 per 32-bit
-// column, the lower k in the low half), B from shared memory as above.
-__device__ __forceinline__ void tc_mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                               uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ss_pair_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                                  uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 ad, {%1, %2};\n\t"
+      "mov.b64 bd, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -38,6 +38,29 @@ __device__ __forceinline__ bool named_bar_any(int id, int count, bool pred) {
   return r != 0;
 }
 
+// A work unit of a CTA pair: weight-side tile m_pair (256 rows of the MMA's
+// M side) against tokens tok0 .. tok0 + ntok - 1 (ntok = 256, or 128 for a
+// half tile).
+struct Unit {
+  int m_pair;
+  int tok0;
+  int ntok;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmParams &p, int u) {
+  int tile = u, half = -1;
+  if (u >= p.units_full) {
+    const int h = u - p.units_full;
+    tile = p.units_full + (h >> 1);
+    half = h & 1;
+  }
+  Unit r;
+  r.m_pair = tile % p.m_tiles;
+  r.tok0 = (tile / p.m_tiles) * 256 + (half > 0 ? 128 : 0);
+  r.ntok = half < 0 ? 256 : 128;
+  return r;
+}
+
 // One 64-weight block's inputs for a dequantizing thread, as loaded: the
 // scale s_b = RN32(fp8 * c2) is formed only when the block is dequantized, so
 // that issuing the loads never waits for them.

@@ -17,7 +17,8 @@
 // planes) as the B half; the even CTA issues tcgen05.mma.cta_group::2 (M = 256,
 // N = 256) accumulating each CTA's 128 columns x 256 tokens in its own tensor
 // memory, two accumulators of 256 columns so that the epilogue of one tile
-// overlaps the next tile's MMAs.
+// overlaps the next tile's MMAs.  When the last round of tiles would leave
+// most pairs idle, its tiles run as 128-token halves (N = 128).
 //
 // Warp roles (576 threads per CTA, one CTA per SM, persistent over tiles):
 //   warps 0-3   epilogue: tensor memory -> BF16 -> global memory, a pair of columns
@@ -86,7 +87,8 @@ struct Smem {
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     nf4_gemm_dx_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lact,
-                           const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tmap_act_h,
+                           const __grid_constant__ CUtensorMap tmap_lact_h, const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem sm;
   sm.base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -97,8 +99,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t rank = cluster_ctarank();          // 0: leader (issues the MMAs), 1: peer
   const bool leader = rank == 0;
   const int ksteps = p.k_main + p.k_lora;
-  const int m_pairs = p.m_tiles;                     // 256-column tiles of W
-  const int num_tiles = m_pairs * p.n_tiles;
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
 
@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tmap_act);
     tma_prefetch_desc(&tmap_lact);
+    if (p.units > p.units_full) {
+      tma_prefetch_desc(&tmap_act_h);
+      tma_prefetch_desc(&tmap_lact_h);
+    }
   }
   if (warp == 17) {
     tmem_alloc_pair(sm.tmem_slot(), TMEM_COLS);
@@ -133,45 +137,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 17) {
     // ---------------- MMA issuer (even CTA) ----------------
     if (leader && lane == 0) {
-      // The issuing thread shares its scheduler with three dequantization
-      // warps, so each stage costs it as few instructions as possible: the
-      // descriptors of stage s, slice kk are the stage-0 ones plus constant
-      // offsets in the address field (A MN-major: a 16-row slice is 4096
-      // bytes on; B K-major: 32 bytes on), which cannot carry out since
-      // shared addresses stay below 256 KiB.
-      const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, true, false);
+      // The issuing thread shares its scheduler and ALU pipe with three
+      // dequantization warps, so a stage costs it as few instructions as
+      // possible: the ring position, the phase, the stage's barrier addresses
+      // and the low words of its descriptors are advanced incrementally (the
+      // address fields cannot carry out: shared addresses stay below 256
+      // KiB); slice kk adds 4096 bytes to A (MN-major: 16 rows of the
+      // contraction) and 32 bytes to B (K-major), i.e. 256 and 2 in the fields.
+      const uint32_t idesc_full = idesc_bf16_f32(2 * PM, PN, true, false);
+      const uint32_t idesc_half = idesc_bf16_f32(2 * PM, PN / 2, true, false);
       const uint64_t adesc0 = smem_desc_sw128(sm.a(0), 1024, 2048);
       const uint64_t bdesc0 = smem_desc_sw128(sm.b(0), 16, 1024);
+      const uint32_t a_lo0 = static_cast<uint32_t>(adesc0), a_hi = static_cast<uint32_t>(adesc0 >> 32);
+      const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0), b_hi = static_cast<uint32_t>(bdesc0 >> 32);
       // 16-wide K slices of the last rank-r stage of a plane that hold any of
       // the r rows of A (the slices past them multiply zeros and are skipped)
       const int nk_tail = min(4, (p.r - (p.k_lora_plane - 1) * BK + 15) / 16);
-      int it = 0, tc = 0;
+      int s = 0, tc = 0;
+      uint32_t ph = 0, a_lo = a_lo0, b_lo = b_lo0, fb = sm.full(0), eb = sm.empty(0);
       bool ok = true;
-      auto stage = [&](uint32_t d_tmem, int nk, uint32_t accumulate) -> bool {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(sm.full(s), ph, p.status)) return false;
-        tc_fence_after();
-        const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
-        const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (B_BYTES >> 4));
-        tc_mma_ss_pair(d_tmem, ad, bd, idesc, accumulate);
-#pragma unroll
-        for (int kk = 1; kk < 4; ++kk)
-          if (kk < nk) tc_mma_ss_pair(d_tmem, ad + kk * (4096 >> 4), bd + kk * (32 >> 4), idesc, 1u);
-        tc_commit_pair_mc(sm.empty(s), 0x3);
-        ++it;
-        return true;
+      auto advance = [&]() {
+        a_lo += A_BYTES >> 4;
+        b_lo += B_BYTES >> 4;
+        fb += 8;
+        eb += 8;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+          a_lo = a_lo0;
+          b_lo = b_lo0;
+          fb = sm.full(0);
+          eb = sm.empty(0);
+        }
       };
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
+      for (int u = cluster_id; u < p.units && ok; u += num_clusters, ++tc) {
+        const uint32_t idesc = unit_of(p, u).ntok == PN ? idesc_full : idesc_half;
         const int acc = tc & 1;
         const uint32_t acc_phase = (tc >> 1) & 1;
         if (!mbar_wait(sm.acc_empty(acc), acc_phase ^ 1, p.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PN);
-        for (int ks = 0; ks < p.k_main && ok; ++ks) ok = stage(d_tmem, 4, ks > 0 ? 1u : 0u);
-        for (int pl = 0; pl < 2 && ok; ++pl)
-          for (int l = 0; l < p.k_lora_plane && ok; ++l)
-            ok = stage(d_tmem, l == p.k_lora_plane - 1 ? nk_tail : 4, 1u);
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * PN);
+        for (int ks = 0; ks < p.k_main; ++ks) {
+          if (!mbar_wait(fb, ph, p.status)) { ok = false; break; }
+          tc_fence_after();
+          tc_mma_ss_pair_lo(d, a_lo, a_hi, b_lo, b_hi, idesc, ks > 0 ? 1u : 0u);
+          tc_mma_ss_pair_lo(d, a_lo + 256, a_hi, b_lo + 2, b_hi, idesc, 1u);
+          tc_mma_ss_pair_lo(d, a_lo + 512, a_hi, b_lo + 4, b_hi, idesc, 1u);
+          tc_mma_ss_pair_lo(d, a_lo + 768, a_hi, b_lo + 6, b_hi, idesc, 1u);
+          tc_commit_pair_mc(eb, 0x3);
+          advance();
+        }
+        for (int pl = 0; pl < 2 && ok; ++pl) {
+          for (int l = 0; l < p.k_lora_plane; ++l) {
+            const int nk = l == p.k_lora_plane - 1 ? nk_tail : 4;
+            if (!mbar_wait(fb, ph, p.status)) { ok = false; break; }
+            tc_fence_after();
+            for (int kk = 0; kk < nk; ++kk)
+              tc_mma_ss_pair_lo(d, a_lo + kk * 256, a_hi, b_lo + kk * 2, b_hi, idesc, 1u);
+            tc_commit_pair_mc(eb, 0x3);
+            advance();
+          }
+        }
         if (!ok) break;
         tc_commit_pair_mc(sm.acc_full(acc), 0x3);
       }
@@ -185,9 +211,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool ok = true, dep_done = false;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-        const int n_tile = tile / m_pairs;
-        const int t0 = n_tile * PN + static_cast<int>(rank) * HN;
+      for (int u = cluster_id; u < p.units && ok; u += num_clusters) {
+        const Unit w = unit_of(p, u);
+        const bool half = w.ntok != PN;              // each CTA loads 64 of 128 tokens
+        const int t0 = w.tok0 + static_cast<int>(rank) * (w.ntok / 2);
+        const CUtensorMap *m_act = half ? &tmap_act_h : &tmap_act;
+        const CUtensorMap *m_lact = half ? &tmap_lact_h : &tmap_lact;
+        const uint32_t bytes = 2u * static_cast<uint32_t>(half ? B_BYTES / 2 : B_BYTES);
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -195,9 +225,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the leader arms its full barrier for both CTAs' bytes; the peer's
           // load only completes transactions on it
           const uint32_t fb = lead(sm.full(s));
-          if (leader) mbar_arrive_expect_tx(sm.full(s), 2 * B_BYTES);
+          if (leader) mbar_arrive_expect_tx(sm.full(s), bytes);
           if (ks < p.k_main) {
-            tma_load_2d_pair(sm.b(s), &tmap_act, fb, ks * BK, t0);
+            tma_load_2d_pair(sm.b(s), m_act, fb, ks * BK, t0);
           } else {
             // the rank-r planes are the preceding kernel's output
             if (!dep_done) {
@@ -205,7 +235,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               grid_dep_launch();
               dep_done = true;
             }
-            tma_load_2d_pair(sm.b(s), &tmap_lact, fb, (ks - p.k_main) * BK, t0);
+            tma_load_2d_pair(sm.b(s), m_lact, fb, (ks - p.k_main) * BK, t0);
           }
         }
       }
@@ -241,8 +271,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t phase = static_cast<uint32_t>(rho & 7);
     int it_base = 0;
     bool ok = true;
-    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-      const int m_pair = tile % m_pairs;
+    for (int u = cluster_id; u < p.units && ok; u += num_clusters) {
+      const int m_pair = unit_of(p, u).m_pair;
       const int64_t col0 = static_cast<int64_t>(m_pair) * 2 * PM + static_cast<int64_t>(rank) * PM;
       const int64_t kb = col0 / 64 + h;              // this thread's column block of W
       const bool kb_ok = kb < kblocks;
@@ -290,9 +320,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp;
     int tc = 0;
     bool ok = true;
-    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
-      const int m_pair = tile % m_pairs;
-      const int n_tile = tile / m_pairs;
+    for (int u = cluster_id; u < p.units && ok; u += num_clusters, ++tc) {
+      const Unit w = unit_of(p, u);
       const int acc = tc & 1;
       const uint32_t acc_phase = (tc >> 1) & 1;
       const bool fail = s_abort || !mbar_wait(sm.acc_full(acc), acc_phase, p.status);
@@ -300,22 +329,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * PN);
       const int m_local = q * 32 + static_cast<int>(lane);
-      const int col_base = m_pair * 2 * PM + static_cast<int>(rank) * PM;
+      const int col_base = w.m_pair * 2 * PM + static_cast<int>(rank) * PM;
       // lanes 2i and 2i + 1 hold columns c and c + 1 (c even); after one exchange
       // the even lane stores both columns of token j, the odd lane those of j + 1
       const int64_t col = static_cast<int64_t>(col_base) + (m_local & ~1);
       const bool odd = (lane & 1) != 0;
-      for (int ch = 0; ch < PN / EPI_ROWS; ++ch) {
+      const int nch = w.ntok / EPI_ROWS;             // accumulator chunks (8, or 4 for a half tile)
+      for (int ch = 0; ch < nch; ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + ch * EPI_ROWS, r);
         tc_wait_ld();
         reg_fence(r);
-        if (ch == PN / EPI_ROWS - 1) {
+        if (ch == nch - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(lead(sm.acc_empty(acc)));
         }
-        const int64_t tok0 = static_cast<int64_t>(n_tile) * PN + ch * EPI_ROWS;
+        const int64_t tok0 = static_cast<int64_t>(w.tok0) + ch * EPI_ROWS;
         if (tok0 >= p.T) continue;   // uniform
 #pragma unroll
         for (int j = 0; j < EPI_ROWS; j += 2) {

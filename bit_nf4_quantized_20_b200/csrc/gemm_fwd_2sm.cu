@@ -19,7 +19,8 @@
 // With one accumulator the epilogue drains it (tcgen05.ld -> BF16 -> a
 // swizzled shared-memory tile) before the next tile's first MMA; the MMA pipe
 // restarts with the A and B rings already full, and the tile goes to global
-// memory by TMA store while the next tile runs.
+// memory by TMA store while the next tile runs.  When the last round of tiles
+// would leave most pairs idle, its tiles run as 128-token halves (N = 128).
 //
 // Warp roles (576 threads per CTA, one CTA per SM, persistent over tiles):
 //   warps 0-3   epilogue (warp q reads accumulator lanes 32q..32q+31)
@@ -57,7 +58,7 @@ static_assert(ACC_COLS + STAGES * A_COLS == TMEM_COLS, "tensor memory budget");
 constexpr int NUM_THREADS = 576;
 constexpr int DQ_GROUPS = 3;
 constexpr int EPI_COLS = 32;                   // accumulator columns per tcgen05.ld
-constexpr int OUT_BOX_BYTES = PN * 128;        // 256 tokens x 64 features, BF16
+constexpr int OUT_BOX_BYTES = PN * 128;        // 256 tokens x 64 features, BF16 (stored as two 128-token boxes)
 constexpr int EPI_BAR = 1, EPI_ANY_BAR = 2;    // named barriers of the epilogue warps
 
 constexpr int OFF_B = 0;
@@ -120,7 +121,9 @@ __device__ __forceinline__ void load_row64(const uint16_t *src, int n_valid, boo
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     nf4_gemm_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lact,
-                            const __grid_constant__ CUtensorMap tmap_out, const GemmParams p) {
+                            const __grid_constant__ CUtensorMap tmap_act_h,
+                            const __grid_constant__ CUtensorMap tmap_lact_h, const __grid_constant__ CUtensorMap tmap_out,
+                            const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem sm;
   sm.base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -131,8 +134,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t rank = cluster_ctarank();          // 0: leader (issues the MMAs), 1: peer
   const bool leader = rank == 0;
   const int ksteps = p.k_main + p.k_lora;
-  const int m_pairs = p.m_tiles;                     // 256-row weight tiles
-  const int num_tiles = m_pairs * p.n_tiles;
   const int cluster_id = blockIdx.x >> 1;
   const int num_clusters = gridDim.x >> 1;
 
@@ -150,6 +151,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tmap_act);
     tma_prefetch_desc(&tmap_lact);
+    if (p.units > p.units_full) {
+      tma_prefetch_desc(&tmap_act_h);
+      tma_prefetch_desc(&tmap_lact_h);
+    }
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_out);
   if (warp == 17) {
@@ -167,39 +172,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 17) {
     // ---------------- MMA issuer (even CTA) ----------------
     if (leader && lane == 0) {
-      // The issuing thread shares its scheduler with three dequantization
-      // warps, so each stage costs it as few instructions as possible: the
-      // descriptors of stage s, slice kk are the stage-0 ones plus constant
-      // offsets (B: (s * B_BYTES + kk * 32) >> 4 in the address field, which
-      // cannot carry out since shared addresses stay below 256 KiB).
-      const uint32_t idesc = idesc_bf16_f32(2 * PM, PN, false, false);
+      // The issuing thread shares its scheduler and ALU pipe with three
+      // dequantization warps, so a stage costs it as few instructions as
+      // possible: the ring position, the phase, the stage's barrier and
+      // tensor-memory addresses and the low word of its B descriptor are
+      // advanced incrementally (the descriptor's address field cannot carry
+      // out: shared addresses stay below 256 KiB); slice kk adds kk * 8
+      // columns to A and 32 bytes (2 in the field) to B.
+      const uint32_t idesc_full = idesc_bf16_f32(2 * PM, PN, false, false);
+      const uint32_t idesc_half = idesc_bf16_f32(2 * PM, PN / 2, false, false);
       const uint64_t bdesc0 = smem_desc_sw128(sm.b(0), 16, 1024);
+      const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0), b_hi = static_cast<uint32_t>(bdesc0 >> 32);
       // 16-wide K slices of the last rank-r stage of a plane that hold any of
       // the r columns (the slices past them multiply zeros and are skipped)
       const int nk_tail = min(4, (p.r - (p.k_lora_plane - 1) * BK + 15) / 16);
-      int it = 0, tc = 0;
+      int s = 0, tc = 0;
+      uint32_t ph = 0, ad = tmem_a, b_lo = b_lo0, fb = sm.full(0), eb = sm.empty(0);
       bool ok = true;
-      auto stage = [&](int nk, uint32_t accumulate) -> bool {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(sm.full(s), ph, p.status)) return false;
-        tc_fence_after();
-        const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (B_BYTES >> 4));
-        const uint32_t ad = tmem_a + static_cast<uint32_t>(s * A_COLS);
-        tc_mma_ts_pair(tmem_base, ad, bd, idesc, accumulate);
-#pragma unroll
-        for (int kk = 1; kk < 4; ++kk)
-          if (kk < nk) tc_mma_ts_pair(tmem_base, ad + kk * 8, bd + kk * 2, idesc, 1u);
-        tc_commit_pair_mc(sm.empty(s), 0x3);
-        ++it;
-        return true;
+      auto advance = [&]() {
+        ad += A_COLS;
+        b_lo += B_BYTES >> 4;
+        fb += 8;
+        eb += 8;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+          ad = tmem_a;
+          b_lo = b_lo0;
+          fb = sm.full(0);
+          eb = sm.empty(0);
+        }
       };
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
+      for (int u = cluster_id; u < p.units && ok; u += num_clusters, ++tc) {
+        const uint32_t idesc = unit_of(p, u).ntok == PN ? idesc_full : idesc_half;
         if (!mbar_wait(sm.acc_empty(), (tc & 1) ^ 1, p.status)) { ok = false; break; }
         tc_fence_after();
-        for (int ks = 0; ks < p.k_main && ok; ++ks) ok = stage(4, ks > 0 ? 1u : 0u);
-        for (int pl = 0; pl < 2 && ok; ++pl)
-          for (int l = 0; l < p.k_lora_plane && ok; ++l) ok = stage(l == p.k_lora_plane - 1 ? nk_tail : 4, 1u);
+        for (int ks = 0; ks < p.k_main; ++ks) {
+          if (!mbar_wait(fb, ph, p.status)) { ok = false; break; }
+          tc_fence_after();
+          tc_mma_ts_pair_lo(tmem_base, ad, b_lo, b_hi, idesc, ks > 0 ? 1u : 0u);
+          tc_mma_ts_pair_lo(tmem_base, ad + 8, b_lo + 2, b_hi, idesc, 1u);
+          tc_mma_ts_pair_lo(tmem_base, ad + 16, b_lo + 4, b_hi, idesc, 1u);
+          tc_mma_ts_pair_lo(tmem_base, ad + 24, b_lo + 6, b_hi, idesc, 1u);
+          tc_commit_pair_mc(eb, 0x3);
+          advance();
+        }
+        for (int pl = 0; pl < 2 && ok; ++pl) {
+          for (int l = 0; l < p.k_lora_plane; ++l) {
+            const int nk = l == p.k_lora_plane - 1 ? nk_tail : 4;
+            if (!mbar_wait(fb, ph, p.status)) { ok = false; break; }
+            tc_fence_after();
+            for (int kk = 0; kk < nk; ++kk)
+              tc_mma_ts_pair_lo(tmem_base, ad + kk * 8, b_lo + kk * 2, b_hi, idesc, 1u);
+            tc_commit_pair_mc(eb, 0x3);
+            advance();
+          }
+        }
         if (!ok) break;
         tc_commit_pair_mc(sm.acc_full(), 0x3);
       }
@@ -213,9 +241,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool ok = true, dep_done = false;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-        const int n_tile = tile / m_pairs;
-        const int t0 = n_tile * PN + static_cast<int>(rank) * HN;
+      for (int u = cluster_id; u < p.units && ok; u += num_clusters) {
+        const Unit w = unit_of(p, u);
+        const bool half = w.ntok != PN;              // each CTA loads 64 of 128 tokens
+        const int t0 = w.tok0 + static_cast<int>(rank) * (w.ntok / 2);
+        const CUtensorMap *m_act = half ? &tmap_act_h : &tmap_act;
+        const CUtensorMap *m_lact = half ? &tmap_lact_h : &tmap_lact;
+        const uint32_t bytes = 2u * static_cast<uint32_t>(half ? B_BYTES / 2 : B_BYTES);
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -223,9 +255,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the leader arms its full barrier for both CTAs' bytes; the peer's
           // load only completes transactions on it
           const uint32_t fb = lead(sm.full(s));
-          if (leader) mbar_arrive_expect_tx(sm.full(s), 2 * B_BYTES);
+          if (leader) mbar_arrive_expect_tx(sm.full(s), bytes);
           if (ks < p.k_main) {
-            tma_load_2d_pair(sm.b(s), &tmap_act, fb, ks * BK, t0);
+            tma_load_2d_pair(sm.b(s), m_act, fb, ks * BK, t0);
           } else {
             // the rank-r planes are the preceding kernel's output
             if (!dep_done) {
@@ -233,7 +265,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               grid_dep_launch();
               dep_done = true;
             }
-            tma_load_2d_pair(sm.b(s), &tmap_lact, fb, (ks - p.k_main) * BK, t0);
+            tma_load_2d_pair(sm.b(s), m_lact, fb, (ks - p.k_main) * BK, t0);
           }
         }
       }
@@ -265,8 +297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool lora_aligned = (p.r % 8) == 0;
     int it_base = 0;
     bool ok = true;
-    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-      const int m_pair = tile % m_pairs;
+    for (int u = cluster_id; u < p.units && ok; u += num_clusters) {
+      const int m_pair = unit_of(p, u).m_pair;
       const int64_t n = static_cast<int64_t>(m_pair) * 2 * PM + static_cast<int64_t>(rank) * PM + tid;
       const bool row_ok = n < p.N;
       auto fetch = [&](int ks) -> BlockIn { return load_block(p, n * kblocks + ks, row_ok && ks < p.k_main); };
@@ -325,9 +357,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int tc = 0;
     bool ok = true;
-    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++tc) {
-      const int m_pair = tile % m_pairs;
-      const int n_tile = tile / m_pairs;
+    for (int u = cluster_id; u < p.units && ok; u += num_clusters, ++tc) {
+      const Unit w = unit_of(p, u);
+      const int nch = w.ntok / EPI_COLS;             // accumulator chunks (8, or 4 for a half tile)
       const bool fail = s_abort || !mbar_wait(sm.acc_full(), tc & 1, p.status);
       // the previous tile's TMA store has finished reading the staging tile
       if (threadIdx.x == 0) tma_store_wait_read<0>();
@@ -354,13 +386,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
 #pragma unroll 1
-      for (int ch = 0; ch < PN / EPI_COLS; ch += 2) {
+      for (int ch = 0; ch < nch; ch += 2) {
         // the load of the next chunk is in flight while this one is stored
         tmem_ld_32x32b_x32(t_row + (ch + 1) * EPI_COLS, rb);
         emit(ra, ch);
         tc_wait_ld();
         reg_fence(rb);
-        if (ch + 2 < PN / EPI_COLS) {
+        if (ch + 2 < nch) {
           tmem_ld_32x32b_x32(t_row + (ch + 2) * EPI_COLS, ra);
         } else {
           // every accumulator column is in registers: release it to the next tile
@@ -369,7 +401,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) mbar_arrive_cluster(lead(sm.acc_empty()));
         }
         emit(rb, ch + 1);
-        if (ch + 2 < PN / EPI_COLS) {
+        if (ch + 2 < nch) {
           tc_wait_ld();
           reg_fence(ra);
         }
@@ -377,10 +409,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_proxy_async_smem();
       named_bar_sync(EPI_BAR, 128);
       if (threadIdx.x == 0) {
-        const int feat0 = m_pair * 2 * PM + static_cast<int>(rank) * PM;
-        const int tok0 = n_tile * PN;
-        tma_store_2d(&tmap_out, sm.out(0), feat0, tok0);
-        tma_store_2d(&tmap_out, sm.out(1), feat0 + 64, tok0);
+        // boxes of 128 tokens x 64 features; a 128-token box of the staging
+        // tile starts 16 KiB on, a whole number of swizzle atoms
+        const int feat0 = w.m_pair * 2 * PM + static_cast<int>(rank) * PM;
+        for (int th = 0; th < w.ntok / 128; ++th)
+          for (int b = 0; b < 2; ++b)
+            tma_store_2d(&tmap_out, sm.out(b) + th * 128 * 128, feat0 + 64 * b, w.tok0 + 128 * th);
         tma_store_commit();
       }
     }

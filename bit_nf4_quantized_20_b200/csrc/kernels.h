@@ -61,6 +61,11 @@ struct GemmParams {
   const uint16_t *lora;    // forward: B[N, r]; backward: A[r, K]
   int r;
   int m_tiles, n_tiles;    // weight-side tiles of 256 (one CTA pair), token tiles of 256
+  // Work units, in order: tiles 0 .. units_full - 1 whole (tile t: weight tile
+  // t % m_tiles, token tile t / m_tiles), then each remaining tile as two
+  // 128-token halves (units - units_full of them), so that a last round that
+  // would leave most CTA pairs idle takes half as long.
+  int units, units_full;
   int k_main, k_lora;      // 64-wide contraction stages: weight part, rank-r part (hi then lo plane)
   int k_lora_plane;        // rank-r stages per plane (k_lora = 2 k_lora_plane)
   int sym;                 // codebook[15 - i] == -codebook[i] exactly (8-entry lookup)
@@ -68,17 +73,25 @@ struct GemmParams {
   uint16_t *out;           // Y [T, N] (stored by TMA through tmap_out) or dX [T, K] (from registers)
   int64_t ldo;             // its row stride (N or K)
 };
-// Launched as clusters of 2 CTAs, one CTA per SM, persistent over the tiles.
-// The forward (mode 0), A from tensor memory; tmap_out: Y [T, N], box [256
+// Launched as clusters of 2 CTAs, one CTA per SM, persistent over the work
+// units.  Token operand maps: act = X or dY [T, C], lact = the rank-r planes
+// [T, 2 ceil64(r)]; boxes of 64 columns by 128 rows (whole tiles: each CTA
+// loads half of 256 tokens) or by 64 rows (the "_h" maps: half tiles),
+// 128-byte swizzle.
+// The forward (mode 0), A from tensor memory; tmap_out: Y [T, N], box [128
 // tokens][64 features], 128-byte swizzle (gemm_fwd_2sm.cu).
 int gemm_fwd_2sm_smem_bytes();
 __global__ void nf4_gemm_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
                                         const __grid_constant__ CUtensorMap tmap_lact,
+                                        const __grid_constant__ CUtensorMap tmap_act_h,
+                                        const __grid_constant__ CUtensorMap tmap_lact_h,
                                         const __grid_constant__ CUtensorMap tmap_out, const GemmParams p);
 // The backward dX (mode 1), A = W'^T from shared memory (gemm_dx_2sm.cu).
 int gemm_dx_2sm_smem_bytes();
 __global__ void nf4_gemm_dx_2sm_kernel(const __grid_constant__ CUtensorMap tmap_act,
-                                       const __grid_constant__ CUtensorMap tmap_lact, const GemmParams p);
+                                       const __grid_constant__ CUtensorMap tmap_lact,
+                                       const __grid_constant__ CUtensorMap tmap_act_h,
+                                       const __grid_constant__ CUtensorMap tmap_lact_h, const GemmParams p);
 
 // ---------------------------------------------------------------------------
 // decode-sized forward of one or several projections (decode.cu)
