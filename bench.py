@@ -64,18 +64,27 @@ def measured_peaks():
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi every 10 ms; summary() keeps the samples taken inside the
+    window mark_start() .. mark_stop() (all samples if none fell inside)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "10",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -93,17 +102,26 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        import datetime
         rows = []
         for line in (self.out or "").splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((float(parts[2]), float(parts[3]), float(parts[4]), parts[5:], ts))
             except ValueError:
                 continue
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if self.t0 <= r[4] <= self.t1]
+            if inside:
+                rows = inside
+            else:
+                window = "whole run (no sample fell inside the timed region)"
         sm = [r[0] for r in rows]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -112,7 +130,7 @@ class ClockSampler:
                 if v.strip().lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows),
+                "reasons": sorted(reasons), "samples": len(rows), "window": window,
                 "power_w_max": max(r[2] for r in rows)}
 
 
@@ -227,17 +245,19 @@ def bench_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
         start.record()
         for _ in range(args.steps):
             run_step(layers, s, args.path == "saved")
         stop.record()
         torch.cuda.synchronize()
+        clk.mark_stop()
     q.get_error(dev)
     ms = start.elapsed_time(stop) / args.steps
     # per-kernel breakdown: the same steps again with an event pair around every
-    # launch (outside the timed region: the events serialise the launches, and
-    # the backward's dB/dA products then run on the caller's stream instead of
-    # beside the dX GEMM, so that every pair of events times one launch alone)
+    # launch (outside the timed region: the events serialise the launches, so
+    # no kernel starts early and the backward's dB/dA grid runs after the dX
+    # GEMM instead of in its last round; every pair of events times one launch)
     with tracer:
         for _ in range(args.steps):
             run_step(layers, s, args.path == "saved")
