@@ -134,6 +134,22 @@ class ClockSampler:
                 "power_w_max": max(r[2] for r in rows)}
 
 
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time per step (every rank gets it); `ms` unchanged
+    on one process.  Works on any backend: the tensor lives on `device`."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_rank_step, ms):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
@@ -263,13 +279,11 @@ def bench_ours(args, rank, world, local_rank):
             run_step(layers, s, args.path == "saved")
     torch.cuda.synchronize()
     q.get_error(dev)
+    ms = max_over_ranks(ms, dist, dev)
     if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     flops = step_flops(T, r)
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops, ms)
     kern = tracer.per_kernel()
     gpu_launches = int(tracer.count.value)
 
@@ -399,12 +413,8 @@ def bench_e2e(args, layers, dev, s, world, dist):
         e2e_step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    v = world * step_flops() / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(a.elapsed_time(b) / steps, dist, dev)
+    v = aggregate_tflops(world, step_flops(), ms)
     return {"value": round(v, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms, 3), "steps": steps}
 
