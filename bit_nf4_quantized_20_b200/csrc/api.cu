@@ -521,6 +521,7 @@ struct TcLaunch {
 qlora_status prepare_single_tc(const TcProduct &t, SkinnyTcArgs a, uint8_t *ws, const WsLayout &L,
                                TcLaunch &l) {
   if (!prepare_tc(t, a, ws, L.partials, L.counters, l.m0)) return QLORA_ERR_CUDA;
+  a.cluster = 1;   // a single product reduces its splits inside a cluster
   l.kid = t.kid;
   l.pair = false;
   l.a0 = a;
@@ -850,7 +851,8 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
   SkinnyTcArgs aa = tc_args(K, T, r, 1.0f);
   aa.tr = static_cast<uint16_t *>(dA);
 
-  TcLaunch first, second;
+  TcLaunch first, mid, second;
+  bool have_mid = false;
   qlora_status rs;
   if (!u_saved) {
     // one grid: sU = s X A^T, transposed, as hi + lo planes, with dU; then
@@ -869,13 +871,20 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
     const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
     rs = prepare_pair_tc(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, second);
   } else {
-    // one grid: dU with dB (both stream dY, sU comes from the forward); then
-    // dA alone
-    const PairGeom g1 = geom_du_db(T, N, r);
-    const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, g1.g0};
-    const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, g1.g1};
-    rs = prepare_pair_tc(K_LORA_DU_DB, td, ad, tb, ab, g1, w8, L, first);
+    // dB (sU comes from the forward) and dU both stream dY, as two launches
+    // sharing one wave: dU is a programmatic dependent of dB that waits for it
+    // only before exiting (its inputs were complete before dB started), so
+    // both run at once, each reducing its splits in clusters; then dA
+    SkinnyTcGeom gb, gd;
+    skinny_tc_share_geom(N, T, false, 2, T, N, true, 1, r, kSplitSms, gb, gd);
+    const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, gb};
+    const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, gd};
+    rs = prepare_single_tc(tb, ab, w8, L, first);
     if (rs != QLORA_OK) return rs;
+    rs = prepare_single_tc(td, ad, w8, L, mid);
+    if (rs != QLORA_OK) return rs;
+    mid.a0.dep_late = 1;
+    have_mid = true;
     const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, geom_da(T, K, r)};
     rs = prepare_single_tc(ta, aa, w8, L, second);
   }
@@ -896,6 +905,10 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
     return QLORA_ERR_CUDA;
   rs = launch_tc(first, st);
   if (rs != QLORA_OK) return rs;
+  if (have_mid) {
+    rs = launch_tc(mid, st);
+    if (rs != QLORA_OK) return rs;
+  }
   rs = launch_gemm(gl, st);
   if (rs != QLORA_OK) return rs;
   return launch_tc(second, st);

@@ -165,7 +165,15 @@ struct SkinnyTcGeom {
   int64_t c_per_split;  // multiple of 64
 };
 // nq: Q planes (1, or 2 for hi + lo); q_cj: Q stored [c][j] (MN-major) else [j][c].
+// At most kSkinnyMaxClusterSplits splits, so that a launch of one product can
+// reduce its splits inside a thread-block cluster.
+constexpr int kSkinnyMaxClusterSplits = 8;
 SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int num_sms);
+// Two products launched one after the other to run side by side in one wave:
+// each with its own tile width and pipeline depth, the CTA slots shared in
+// proportion to their bytes, at most kSkinnyMaxClusterSplits splits each.
+void skinny_tc_share_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
+                          int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1);
 size_t skinny_tc_partials_bytes(const SkinnyTcGeom &g, int64_t M, int R);
 
 struct SkinnyTcArgs {
@@ -189,18 +197,22 @@ struct SkinnyTcArgs {
   float *partials;       // [splits][M][(R + 3) & ~3] when splits > 1
   uint32_t *counters;    // one per 128-row tile (zero on entry, zero on exit)
   uint32_t *status;
+  int cluster;           // single-product launches with splits <= 8: the splits of a row tile are
+                         // one cluster and reduce through distributed shared memory (no partials,
+                         // no counters)
   int dep_late;          // every input was complete when the preceding kernel let this one
                          // start: wait for that kernel only before exiting (same in both
                          // products of a pair launch)
 };
 cudaError_t launch_skinny_tc(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUtensorMap &tm_q0,
                              const CUtensorMap &tm_q1, cudaStream_t st, bool pdl);
-// Two independent products sharing one grid and one tile width (the larger of
-// the two), the CTA slots of one wave shared in proportion to their bytes.  Both
-// have R columns; each has its own Q plane count (nq0, nq1), pipeline depth,
-// partials and counters.
+// Two independent products sharing one wave -- in one grid (the pair launch),
+// or as two launches that run side by side -- with one tile width (the larger
+// of the two), the CTA slots of the wave shared in proportion to their bytes.
+// Both have R columns; each has its own Q plane count (nq0, nq1), pipeline
+// depth, partials and counters.  max_splits > 0 caps each product's splits.
 void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
-                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1);
+                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1, int max_splits = 0);
 // maps: {P, Q0, Q1} for each product
 cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
                                   const CUtensorMap *maps1, cudaStream_t st, bool pdl);

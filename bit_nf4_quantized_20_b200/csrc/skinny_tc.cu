@@ -13,9 +13,14 @@
 // memory.  U and dU are also written transposed as two BF16 planes hi = bf16(v),
 // lo = bf16(v - hi), which dB and dA take as two MMAs into one accumulator.
 // The contraction is split across CTAs so that the grid fills the GPU in one
-// wave (two CTAs per SM); each split writes an FP32 partial tile and the last
-// CTA of a row tile (a workspace counter, reset by that CTA) sums the partials
-// in split order and writes the outputs.
+// wave (two CTAs per SM).  With `cluster` set, the splits of a row tile form
+// one thread-block cluster (at most 8 CTAs, co-scheduled): each CTA leaves its
+// FP32 partial tile in its own shared memory, and after a cluster barrier
+// every CTA sums its share of the tile's rows over the cluster's CTAs, in
+// split order, through distributed shared memory and writes them out.
+// Otherwise each split writes an FP32 partial tile to the workspace and the
+// last CTA of a row tile (a workspace counter, reset by that CTA) sums the
+// partials in split order and writes the outputs.
 //
 // Launched as a programmatic dependent: the prologue (barriers, tensor memory,
 // descriptor prefetch) overlaps the previous kernel, and every global access
@@ -44,6 +49,10 @@ constexpr int TNUM_THREADS = 192;
 constexpr int kBarBytes = 8 * (2 * TMAX_STAGES + 1) + 8;   // full[], empty[], accumulator, tensor-memory slot
 constexpr int kFixedSmem = kBarBytes + 1024;               // + alignment slack for the 1 KiB swizzle atoms
 constexpr int kTwoPerSmBudget = 110 * 1024;
+// row pitch (floats) of a CTA's partial tile in shared memory in cluster mode:
+// 16-byte aligned rows, offset by 4 floats to spread the banks
+template <int NB>
+constexpr int RED_PITCH = NB + 4;
 constexpr int kOnePerSmBudget = 220 * 1024;
 
 // Columns c0 .. c0 + CW - 1 of row m: v[j] is the un-scaled accumulator.
@@ -97,6 +106,19 @@ __device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, float (&v)[CW]) 
   tc_wait_ld();
 #pragma unroll
   for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 }  // namespace
@@ -234,7 +256,23 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int pw = (a.R + 3) & ~3;      // partial row width (the R meaningful columns, float4 granular)
     float v[CW];
-    if (a.splits > 1) {
+    if (a.cluster && a.splits > 1) {
+      // this CTA's partial rows into its own shared memory (the drained stage
+      // ring), read by every CTA of the cluster after the cluster barrier
+      const uint32_t red_row = base + static_cast<uint32_t>(row) * static_cast<uint32_t>(RED_PITCH<NB> * 4);
+#pragma unroll 1
+      for (int c0 = 0; c0 < NB; c0 += CW) {
+        if (have) {
+          tmem_load_chunk<CW>(trow + c0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] = 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < CW; g += 4)
+          st_shared_f4(red_row + static_cast<uint32_t>(c0 + g) * 4u, v[g], v[g + 1], v[g + 2], v[g + 3]);
+      }
+    } else if (a.splits > 1) {
 #pragma unroll 1
       for (int c0 = 0; c0 < NB; c0 += CW) {
         if (have) {
@@ -311,7 +349,7 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
       }
     }
     // the rest of a padded row of the hi / lo planes (columns NB .. ocols - 1) is zero
-    if (a.row_hi && m < a.M && (a.splits == 1 || s_last)) {
+    if (a.row_hi && m < a.M && (a.splits == 1 || (s_last && !a.cluster))) {
       for (int64_t c = NB; c < a.ocols; c += 8) {
         *reinterpret_cast<uint4 *>(a.row_hi + m * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
         if (a.row_lo) *reinterpret_cast<uint4 *>(a.row_lo + m * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
@@ -319,6 +357,44 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
     }
   }
 
+  if (a.cluster && a.splits > 1) {
+    // every CTA of the cluster has its partial rows in shared memory
+    cluster_arrive_wait();
+    // this CTA's rows: [split * rows_per, +rows_per) of the tile, in 8-column
+    // groups (only the groups that hold any of the R columns), consecutive
+    // threads on consecutive rows so that the transposed outputs coalesce
+    const int rows_per = (TBM + a.splits - 1) / a.splits;
+    const int r0 = split * rows_per;
+    const int nrows = min(rows_per, TBM - r0);
+    const int groups = (a.R + 7) / 8;
+    for (int i = static_cast<int>(threadIdx.x); i < nrows * groups; i += TNUM_THREADS) {
+      const int rl = r0 + i % nrows, c0 = (i / nrows) * 8;
+      const int64_t mg = m0 + rl;
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      const uint32_t local = base + static_cast<uint32_t>(rl) * static_cast<uint32_t>(RED_PITCH<NB> * 4) +
+                             static_cast<uint32_t>(c0) * 4u;
+      for (int k = 0; k < a.splits; ++k) {   // split order: the sum does not depend on timing
+        const uint32_t remote = mapa_shared(local, static_cast<uint32_t>(k));
+        const float4 x0 = ld_dsmem_f4(remote), x1 = ld_dsmem_f4(remote + 16u);
+        acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+        acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
+      }
+      if (mg < a.M) {
+        emit_chunk<8>(a, mg, c0, acc);
+        // the rest of a padded row of the hi / lo planes is zero
+        if (a.row_hi && c0 == 8 * (groups - 1)) {
+          for (int64_t c = 8 * groups; c < a.ocols; c += 8) {
+            *reinterpret_cast<uint4 *>(a.row_hi + mg * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
+            if (a.row_lo) *reinterpret_cast<uint4 *>(a.row_lo + mg * a.ldo + c) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      }
+    }
+    // no CTA leaves (and frees its shared memory) while another still reads it
+    cluster_arrive_wait();
+  }
   if (a.dep_late) {
     grid_dep_wait();
     grid_dep_launch();
@@ -403,10 +479,11 @@ int tc_stages(int nb, int nq, SkinnyTcGeom &g) {
   return per_sm;
 }
 // Contraction splits for `slots` CTAs over the 128-row tiles of an M x C product.
-void tc_splits(int64_t M, int64_t C, int64_t slots, SkinnyTcGeom &g) {
+void tc_splits(int64_t M, int64_t C, int64_t slots, SkinnyTcGeom &g, int max_splits = 0) {
   if (M <= 0 || C <= 0) return;
   const int64_t m_tiles = (M + TBM - 1) / TBM;
   int64_t s = slots / m_tiles;
+  if (max_splits > 0 && s > max_splits) s = max_splits;
   const int64_t cap = (C + 2 * TBK - 1) / (2 * TBK);      // at least two stages per split
   if (s > cap) s = cap;
   if (s < 1) s = 1;
@@ -421,12 +498,12 @@ SkinnyTcGeom skinny_tc_geom(int64_t M, int64_t C, int R, int nq, bool q_cj, int 
   SkinnyTcGeom g;
   const int per_sm = tc_stages(tc_nb(R, q_cj), nq, g);
   // one wave: m_tiles x splits <= the CTAs the GPU holds at once
-  if (num_sms > 0) tc_splits(M, C, static_cast<int64_t>(per_sm) * num_sms, g);
+  if (num_sms > 0) tc_splits(M, C, static_cast<int64_t>(per_sm) * num_sms, g, kSkinnyMaxClusterSplits);
   return g;
 }
 
 void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
-                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1) {
+                         int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1, int max_splits) {
   const int nb = tc_nb(R, q_cj0) > tc_nb(R, q_cj1) ? tc_nb(R, q_cj0) : tc_nb(R, q_cj1);
   const int per0 = tc_stages(nb, nq0, g0);
   const int per1 = tc_stages(nb, nq1, g1);
@@ -439,8 +516,22 @@ void skinny_tc_pair_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1
   int64_t s0 = b0 + b1 > 0 ? static_cast<int64_t>(slots * b0 / (b0 + b1) + 0.5) : slots / 2;
   if (s0 < 1) s0 = 1;
   if (s0 > slots - 1) s0 = slots - 1;
-  tc_splits(M0, C0, s0, g0);
-  tc_splits(M1, C1, slots - s0, g1);
+  tc_splits(M0, C0, s0, g0, max_splits);
+  tc_splits(M1, C1, slots - s0, g1, max_splits);
+}
+
+void skinny_tc_share_geom(int64_t M0, int64_t C0, bool q_cj0, int nq0, int64_t M1, int64_t C1, bool q_cj1, int nq1,
+                          int R, int num_sms, SkinnyTcGeom &g0, SkinnyTcGeom &g1) {
+  const int per0 = tc_stages(tc_nb(R, q_cj0), nq0, g0);
+  const int per1 = tc_stages(tc_nb(R, q_cj1), nq1, g1);
+  if (num_sms <= 0) return;
+  const int64_t slots = static_cast<int64_t>(per0 < per1 ? per0 : per1) * num_sms;
+  const double b0 = static_cast<double>(M0) * C0, b1 = static_cast<double>(M1) * C1;
+  int64_t s0 = b0 + b1 > 0 ? static_cast<int64_t>(slots * b0 / (b0 + b1) + 0.5) : slots / 2;
+  if (s0 < 1) s0 = 1;
+  if (s0 > slots - 1) s0 = slots - 1;
+  tc_splits(M0, C0, s0, g0, kSkinnyMaxClusterSplits);
+  tc_splits(M1, C1, slots - s0, g1, kSkinnyMaxClusterSplits);
 }
 
 size_t skinny_tc_partials_bytes(const SkinnyTcGeom &g, int64_t M, int R) {
@@ -455,16 +546,31 @@ cudaError_t launch_nb(const SkinnyTcArgs &a, const CUtensorMap &tm_p, const CUte
   cudaError_t e = ensure_smem_optin(reinterpret_cast<const void *>(skinny_tc_kernel<NB>), kOnePerSmBudget);
   if (e != cudaSuccess) return e;
   const int stage = P_BYTES + a.nq * NB * TBK * 2;
+  const bool cluster = a.cluster && a.splits > 1;
+  // the partial tile of cluster mode lives in the (drained) stage ring
+  if (cluster && (a.splits > kSkinnyMaxClusterSplits || a.stages * stage < TBM * RED_PITCH<NB> * 4))
+    return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((a.M + TBM - 1) / TBM), static_cast<unsigned>(a.splits), 1);
   cfg.blockDim = dim3(TNUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(a.stages * stage + kFixedSmem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (cluster) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = static_cast<unsigned>(a.splits);
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, skinny_tc_kernel<NB>, tm_p, tm_q0, tm_q1, a);
 }
 }  // namespace
@@ -510,6 +616,7 @@ cudaError_t launch_pair_nb(const SkinnyTcArgs &a0, const CUtensorMap *m0, const 
 cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *maps0, const SkinnyTcArgs &a1,
                                   const CUtensorMap *maps1, cudaStream_t st, bool pdl) {
   if (a0.M <= 0 || a0.C <= 0 || a1.M <= 0 || a1.C <= 0 || a0.R <= 0) return cudaErrorInvalidValue;
+  if (a0.cluster || a1.cluster) return cudaErrorInvalidValue;   // one grid of both products: no cluster mode
   if (a0.nb != a1.nb) return cudaErrorInvalidValue;
   for (const SkinnyTcArgs *a : {&a0, &a1})
     if (a->stages < 1 || a->stages > TMAX_STAGES || a->splits < 1 || (a->nq != 1 && a->nq != 2))
