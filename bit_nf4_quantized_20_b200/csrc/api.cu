@@ -66,7 +66,7 @@ enum KernelId : int32_t {
   K_LORA_U_DU = 9,      // U and dU in one grid (backward)
   K_LORA_DB_DA = 10,    // dB and dA in one grid (backward)
   K_MERGE = 11,         // adapter merge for export
-  K_LORA_DU_DB = 12,    // dU and dB in one grid (backward with the forward's saved U)
+  K_LORA_DU_DB = 12,    // dU and dB in one grid (no launch uses it; ids stay stable for trace readers)
   K_ADAM = 13,          // the adapters' optimizer step
   K_COUNT = 14,
 };
