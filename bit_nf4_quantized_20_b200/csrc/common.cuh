@@ -155,13 +155,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// Programmatic dependent launch.  Every kernel of the library keeps one rule:
-// it waits for the preceding kernel of its stream (griddepcontrol.wait) before
-// it completes and before it touches anything that kernel writes, and it lets
-// its own dependents launch (griddepcontrol.launch_dependents) only after
-// that wait.  A kernel that starts early can therefore rely on everything
-// before its predecessor having completed; only the predecessor's own outputs
-// need the wait.
+// Programmatic dependent launch.  Every kernel of the library waits for the
+// preceding kernel of its stream (griddepcontrol.wait) before it completes
+// and before it touches anything that kernel writes, so a kernel completes
+// only after everything before it.  It lets its own dependents launch
+// (griddepcontrol.launch_dependents) only after that wait -- so that a kernel
+// that starts early can rely on everything before its predecessor having
+// completed -- with one exception: a rank-r launch whose inputs were all
+// complete before its predecessor started (it waits only before exiting)
+// lets its dependent start at once; that dependent is the next kernel of the
+// same layer call and reads this launch's outputs only after its own wait.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }

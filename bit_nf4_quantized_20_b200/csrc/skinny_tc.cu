@@ -25,9 +25,12 @@
 // Launched as a programmatic dependent: the prologue (barriers, tensor memory,
 // descriptor prefetch) overlaps the previous kernel, and every global access
 // comes after griddepcontrol.wait -- except in a launch whose inputs all come
-// from kernels that had completed before its predecessor let it start (the
-// adapter gradients after the dX GEMM: dep_late), which waits only before it
-// exits, so that it can run in the GEMM's last wave.
+// from kernels that had completed before its predecessor let it start
+// (dep_late: dU beside dB, the adapter gradients after the dX GEMM), which
+// waits only before it exits, so that it runs beside its predecessor, and
+// lets its own dependent start at once (that dependent is the next kernel of
+// the same layer call, which touches nothing the predecessor writes and reads
+// this launch's outputs only after its own wait).
 //
 // Warps: 0 TMA producer, 1 tensor-memory allocation + MMA issue, 2-5 epilogue.
 
@@ -174,10 +177,8 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ld_shared_u32(tmem_slot);
-  if (!a.dep_late) {
-    grid_dep_wait();
-    grid_dep_launch();
-  }
+  if (!a.dep_late) grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -395,10 +396,7 @@ __device__ __forceinline__ void skinny_tc_body(const CUtensorMap *tm_p, const CU
     // no CTA leaves (and frees its shared memory) while another still reads it
     cluster_arrive_wait();
   }
-  if (a.dep_late) {
-    grid_dep_wait();
-    grid_dep_launch();
-  }
+  if (a.dep_late) grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

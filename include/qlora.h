@@ -31,9 +31,11 @@
  *   - Kernels are launched as programmatic dependents (they may start while
  *     the preceding kernel of the stream finishes).  Each waits for that
  *     kernel before it completes and before it touches anything that kernel
- *     writes, and lets its own dependents start only after that wait; a
- *     caller's kernel that follows a library call on the stream sees all of
- *     the call's results, as usual.
+ *     writes, so it completes only after everything before it on the stream;
+ *     the first kernel of a call also waits before it touches anything at
+ *     all.  A caller's kernel that follows a library call on the stream sees
+ *     all of the call's results, as usual (a caller's own programmatic
+ *     dependent must wait with griddepcontrol.wait before reading them).
  *   - Outputs must not overlap the call's inputs or each other.
  *   - Row-major layouts.  BF16 tensors are arrays of uint16 bit patterns.
  *   - Every check (arguments, alignment, workspace, TMA descriptor encoding)
