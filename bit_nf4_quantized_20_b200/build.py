@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libqlora.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "quant.cu", "gemm_fwd_2sm.cu", "gemm_dx_2sm.cu", "skinny_tc.cu", "optim.cu", "decode.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm_fwd_2sm.cu", "gemm_dx_2sm.cu", "skinny_tc.cu", "dudb.cu", "optim.cu", "decode.cu"]
 HEADERS = ["common.cuh", "gemm_common.cuh", "kernels.h", os.path.join("..", "..", "include", "qlora.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")

@@ -66,15 +66,16 @@ enum KernelId : int32_t {
   K_LORA_U_DU = 9,      // U and dU in one grid (backward)
   K_LORA_DB_DA = 10,    // dB and dA in one grid (backward)
   K_MERGE = 11,         // adapter merge for export
-  K_LORA_DU_DB = 12,    // dU and dB in one grid (no launch uses it; ids stay stable for trace readers)
+  K_LORA_DU_DB = 12,    // dU and dB from one read of dY (block partial sums)
   K_ADAM = 13,          // the adapters' optimizer step
-  K_COUNT = 14,
+  K_LORA_DU_DB_SUM = 14,  // the sums of those partials: dU planes and dB
+  K_COUNT = 15,
 };
 
 const char *kKernelNames[K_COUNT] = {"quantize_nf4_dq", "dequantize_nf4", "lora_u",       "lora_du",
                                      "lora_dB",         "lora_dA",        "nf4_gemm_fwd", "nf4_gemm_bwd_dx",
                                      "nf4_gemv_fwd",    "lora_u+du",      "lora_dB+dA",   "merge_adapter",
-                                     "lora_du+dB",      "adam_step"};
+                                     "lora_du+dB",      "adam_step",      "lora_du+dB_sum"};
 
 struct TraceScope {
   cudaStream_t st;
@@ -289,8 +290,10 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     L.duT_hi = off; off += t_plane;
     L.duT_lo = off; off += t_plane;
     L.bpad = off; off += static_cast<size_t>(round_up(N * r64 * 2, 256));
-    const size_t p[4] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r)),
-                         pair_partials(geom_du_db(T, N, r)), skinny_tc_partials_bytes(geom_da(T, K, r), K, r)};
+    DuDbGeom gdd;
+    const size_t p[5] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r)),
+                         pair_partials(geom_du_db(T, N, r)), skinny_tc_partials_bytes(geom_da(T, K, r), K, r),
+                         dudb_geom(T, N, r, kSplitSms, gdd) ? dudb_partials_bytes(gdd, T, N, r) : 0};
     for (size_t v : p) part = v > part ? v : part;
   }
   L.partials = off;
@@ -853,6 +856,11 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
 
   TcLaunch first, mid, second;
   bool have_mid = false;
+  // saved path, r <= 64: dU and dB from one read of dY, then the sums of the
+  // blocks' partials
+  bool fused = false;
+  DuDbArgs fa;
+  CUtensorMap fm_dy, fm_b, fm_su_hi, fm_su_lo;
   qlora_status rs;
   if (!u_saved) {
     // one grid: sU = s X A^T, transposed, as hi + lo planes, with dU; then
@@ -871,20 +879,55 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
     const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
     rs = prepare_pair_tc(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, second);
   } else {
-    // dB (sU comes from the forward) and dU both stream dY, as two launches
-    // sharing one wave: dU is a programmatic dependent of dB that waits for it
-    // only before exiting (its inputs were complete before dB started), so
-    // both run at once, each reducing its splits in clusters; then dA
-    SkinnyTcGeom gb, gd;
-    skinny_tc_share_geom(N, T, false, 2, T, N, true, 1, r, kSplitSms, gb, gd);
-    const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, gb};
-    const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, gd};
-    rs = prepare_single_tc(tb, ab, w8, L, first);
-    if (rs != QLORA_OK) return rs;
-    rs = prepare_single_tc(td, ad, w8, L, mid);
-    if (rs != QLORA_OK) return rs;
-    mid.a0.dep_late = 1;
-    have_mid = true;
+    DuDbGeom gdd;
+    if (dudb_geom(T, N, r, kSplitSms, gdd)) {
+      // dU and dB from one read of dY: block partial sums in the workspace,
+      // then one launch sums them and writes dU's planes and dB
+      fused = true;
+      memset(&fa, 0, sizeof(fa));
+      fa.T = T;
+      fa.N = N;
+      fa.R = r;
+      fa.tt = gdd.tt;
+      fa.nn = gdd.nn;
+      fa.t_ranges = gdd.t_ranges;
+      fa.n_ranges = gdd.n_ranges;
+      fa.rb = gdd.rb;
+      fa.stages = gdd.stages;
+      fa.tmem_cols = gdd.tmem_cols;
+      fa.s = s;
+      fa.part_u = reinterpret_cast<float *>(w8 + L.partials);
+      fa.part_b = reinterpret_cast<float *>(w8 + L.partials + dudb_part_u_bytes(gdd, T, r));
+      fa.du_hi = ad.row_hi;
+      fa.du_lo = ad.row_lo;
+      fa.ldo = ad.ldo;
+      fa.ocols = ad.ocols;
+      fa.duT_hi = ad.t_hi;
+      fa.duT_lo = ad.t_lo;
+      fa.ldt = ad.ldt;
+      fa.dB = static_cast<uint16_t *>(dB);
+      fa.status = reinterpret_cast<uint32_t *>(ws);
+      if (!make_map_bf16(&fm_dy, dy, T, N, N, 128, 64, true) || !make_map_bf16(&fm_b, bq, N, r, ldb, 64, 64, true) ||
+          !make_map_bf16(&fm_su_hi, su_hi, r, T, Tp, gdd.rb, 64, true) ||
+          !make_map_bf16(&fm_su_lo, su_lo, r, T, Tp, gdd.rb, 64, true))
+        return QLORA_ERR_CUDA;
+    } else {
+      // dB (sU comes from the forward) and dU both stream dY, as two launches
+      // sharing one wave: dU is a programmatic dependent of dB that waits for
+      // it only before exiting (its inputs were complete before dB started),
+      // so both run at once, each reducing its splits in clusters
+      SkinnyTcGeom gb, gd;
+      skinny_tc_share_geom(N, T, false, 2, T, N, true, 1, r, kSplitSms, gb, gd);
+      const TcProduct tb = {K_LORA_DB, dy, N, true, su_hi, su_lo, Tp, false, gb};
+      const TcProduct td = {K_LORA_DU, dy, N, false, bq, nullptr, ldb, true, gd};
+      rs = prepare_single_tc(tb, ab, w8, L, first);
+      if (rs != QLORA_OK) return rs;
+      rs = prepare_single_tc(td, ad, w8, L, mid);
+      if (rs != QLORA_OK) return rs;
+      mid.a0.dep_late = 1;
+      have_mid = true;
+    }
+    // then dA
     const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, geom_da(T, K, r)};
     rs = prepare_single_tc(ta, aa, w8, L, second);
   }
@@ -903,11 +946,24 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
   if (pad_b && launch_pad_cols(static_cast<const uint16_t *>(B), N, r, plane(L.bpad), static_cast<int>(r64), st,
                                num_sms_current()) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  rs = launch_tc(first, st);
-  if (rs != QLORA_OK) return rs;
-  if (have_mid) {
-    rs = launch_tc(mid, st);
+  if (fused) {
+    const bool pdl = g_trace.recs == nullptr;
+    {
+      TraceScope ts(K_LORA_DU_DB, 6.0 * T * N * r, 2.0 * T * N, st);
+      if (launch_dudb(fa, fm_dy, fm_b, fm_su_hi, fm_su_lo, st, pdl) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    {
+      const double part = 4.0 * ((r + 3) & ~3) * (static_cast<double>(fa.n_ranges) * T + static_cast<double>(fa.t_ranges) * N);
+      TraceScope ts(K_LORA_DU_DB_SUM, 0.0, part + 2.0 * (2.0 * T * fa.ocols + 2.0 * r * T + static_cast<double>(N) * r), st);
+      if (launch_dudb_finish(fa, st, pdl, num_sms_current()) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+  } else {
+    rs = launch_tc(first, st);
     if (rs != QLORA_OK) return rs;
+    if (have_mid) {
+      rs = launch_tc(mid, st);
+      if (rs != QLORA_OK) return rs;
+    }
   }
   rs = launch_gemm(gl, st);
   if (rs != QLORA_OK) return rs;

@@ -219,4 +219,49 @@ cudaError_t launch_skinny_tc_pair(const SkinnyTcArgs &a0, const CUtensorMap *map
 cudaError_t launch_pad_cols(const uint16_t *src, int64_t rows, int cols, uint16_t *dst, int ldd, cudaStream_t st,
                             int num_sms);
 
+// ---------------------------------------------------------------------------
+// dU = s dY B and dB = dY^T (sU) from one read of dY (dudb.cu), for r <= 64:
+// each CTA streams a block of dY (tt 128-token tiles x nn 128-feature chunks)
+// once, both accumulators in tensor memory; the blocks' FP32 partial sums go
+// to the workspace and a second launch sums them and writes the outputs.
+// ---------------------------------------------------------------------------
+constexpr int kDudbMaxRank = 64;
+constexpr int kDudbMaxStages = 8;
+constexpr int kDudbMaxChunks = 32;
+struct DuDbGeom {
+  int tt, nn;                  // 128-token tiles, 128-feature chunks per CTA
+  int t_ranges, n_ranges;      // the grid: t_ranges x n_ranges CTAs
+  int rb;                      // dB accumulator columns: r rounded up to 16, 32 or 64
+  int stages;                  // dY tiles in flight (32 KiB each)
+  int smem;                    // dynamic shared memory bytes
+  int tmem_cols;               // tensor-memory columns allocated (a power of two)
+};
+// false: the shape is not covered (r > kDudbMaxRank, or no geometry fits).
+bool dudb_geom(int64_t T, int64_t N, int r, int num_sms, DuDbGeom &g);
+// the two partial-sum buffers: dU [n_ranges][T][(r + 3) & ~3], then (256-aligned)
+// dB [t_ranges][N][(r + 3) & ~3], FP32
+size_t dudb_part_u_bytes(const DuDbGeom &g, int64_t T, int r);
+size_t dudb_partials_bytes(const DuDbGeom &g, int64_t T, int64_t N, int r);
+
+struct DuDbArgs {
+  int64_t T, N;
+  int R;
+  int tt, nn, t_ranges, n_ranges, rb, stages, tmem_cols;
+  float s;                     // dU = s dY B (dB takes sU, already scaled)
+  float *part_u;               // [n_ranges][T][(R + 3) & ~3]
+  float *part_b;               // [t_ranges][N][(R + 3) & ~3]
+  // outputs of the second launch; v = s dU-sum
+  uint16_t *du_hi, *du_lo;     // [T, ldo] bf16(v) and bf16(v - bf16(v)), columns R..ocols-1 zero
+  int64_t ldo, ocols;          // ocols a multiple of 4
+  uint16_t *duT_hi, *duT_lo;   // [R, ldt] the same, transposed
+  int64_t ldt;
+  uint16_t *dB;                // [N, R]
+  uint32_t *status;
+};
+// maps: dY [T rows, N cols] box 128 x 64; B as [N rows, R cols] box 64 x 64
+// (columns past R read as zeros); the sU^T planes [R rows, T cols] box rb x 64.
+cudaError_t launch_dudb(const DuDbArgs &a, const CUtensorMap &tm_dy, const CUtensorMap &tm_b,
+                        const CUtensorMap &tm_su_hi, const CUtensorMap &tm_su_lo, cudaStream_t st, bool pdl);
+cudaError_t launch_dudb_finish(const DuDbArgs &a, cudaStream_t st, bool pdl, int num_sms);
+
 }  // namespace qlora

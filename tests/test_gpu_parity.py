@@ -453,6 +453,56 @@ def test_layer_saved_u(T, N, K, r, s):
     assert np.all(np.abs(got - ref) <= 1e-3 + 2.0 ** -14 * np.abs(ref))
 
 
+def _launched_kernels(fn):
+    """Names of the library kernels that fn() launches (the trace hook, without events)."""
+    import ctypes as C
+    from bit_nf4_quantized_20_b200 import _lib
+    recs = (_lib.TraceRec * 64)()
+    count = C.c_int32(0)
+    lib = _lib.lib()
+    _lib.check("qlora_trace_attach", lib.qlora_trace_attach(recs, 64, C.byref(count)))
+    try:
+        fn()
+    finally:
+        lib.qlora_trace_attach(None, 0, None)
+    return [lib.qlora_kernel_name(recs[i].kernel).decode() for i in range(min(count.value, 64))]
+
+
+@pytest.mark.parametrize("T,N,K,r,s,one_read", [
+    (2500, 3080, 256, 24, 0.5, True),   # blocks of 2 token tiles x 2 feature chunks; ragged T and N
+    (3000, 4104, 128, 13, 2.0, True),   # 2 x 3 blocks, rank 13
+    (2500, 6144, 64, 36, 1.0, True),    # 64-column dB accumulators, three pipeline stages
+    (513, 4104, 192, 1, 1.0, True),     # rank 1; one token in the last tile
+    (1300, 4104, 64, 8, 1.0, True),     # three token tiles a block
+    (300, 384, 320, 24, 0.5, False),    # partial sums would outweigh the second read of dY
+    (257, 1024, 128, 65, 1.0, False),   # rank above 64
+])
+def test_layer_saved_u_one_read_of_dy(T, N, K, r, s, one_read):
+    """The saved-U backward with dU and dB from one read of dY (block partial
+    sums, then a launch that sums them), against the oracle; shapes where the
+    partial sums do not pay off, or the rank is above 64, run dU and dB as two
+    launches instead."""
+    q = Q()
+    W, X, A, B, dY = inputs.layer_inputs(93, 0, 0, T, N, K, r, device="cuda")
+    qw, (codes, scales, c2) = quantize_and_check(W)
+    y, u = q.linear_fwd_save(X, qw, A, B, s)
+    names = _launched_kernels(lambda: q.linear_bwd_saved(dY, X, qw, A, B, s, u))
+    torch.cuda.synchronize()
+    if one_read:
+        assert "lora_du+dB" in names and "lora_du+dB_sum" in names and "lora_dB" not in names, names
+    else:
+        assert "lora_du+dB" not in names and "lora_dB" in names and "lora_du" in names, names
+    dx, dA, dB = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
+    q.get_error()
+    torch.cuda.synchronize()
+    wd = O.dequantize_nf4(codes, scales, c2, N, K)
+    xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
+    rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
+    assert_close("dX", dx, rdx)
+    assert_close("dA", dA, rdA)
+    assert_close("dB", dB, rdB)
+
+
 def test_backward_saved_graph_capture_matches_eager():
     """The saved-U backward (its adapter-gradient grid a programmatic
     dependent of the dX GEMM), captured in a CUDA graph on a non-default
