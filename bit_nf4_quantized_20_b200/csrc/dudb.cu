@@ -12,9 +12,10 @@
 // MN-major (rows n in two 64-feature halves, contraction t) for dB.  All the
 // block's accumulators stay in tensor memory for the whole block: dU for each
 // token tile (64 columns: B's rows arrive as an MN-major [n][j] operand whose
-// columns past r read as zeros), dB for each feature chunk (r rounded up to
-// 16, 32 or 64 columns; the hi and lo planes of sU are two MMAs into one
-// accumulator).  The sU planes of the block's tokens are loaded once, B's rows
+// columns past r read as zeros), dB for each feature chunk (the hi and lo
+// planes of sU, r rounded up to rb = 16, 32 or 64 rows each, stacked into one
+// N = 2 rb operand: one MMA per step, the two halves of the accumulator summed
+// when it is drained).  The sU planes of the block's tokens are loaded once, B's rows
 // of a feature chunk once per chunk (two buffers); the loop runs over feature
 // chunks, and over the block's token tiles inside each chunk.
 //
@@ -52,7 +53,7 @@ constexpr int kBarBytes = 8 * (2 * kDudbMaxStages + 4 + 2 + kDudbMaxChunks) + 8;
 constexpr int kFixed = 2 * BT_BYTES + kBarBytes + 1024;   // + alignment slack for the swizzle atoms
 constexpr int kSmemBudget = 220 * 1024;
 
-int su_bytes(int tt, int rb) { return tt * 4 * rb * 128; }   // tt tiles x {hi, lo} x two boxes [rb j][64 t]
+int su_bytes(int tt, int rb) { return tt * 4 * rb * 128; }   // tt tiles x two 64-token halves x {hi, lo} boxes [rb j][64 t]
 
 __device__ __forceinline__ void st_global_f4(float *p, const float (&v)[4]) {
   *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -91,6 +92,57 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, bool have, bool valid,
   }
 }
 
+// v += sum over k < n of src[k * stride] (float4), in k order, eight loads in
+// flight at a time.
+__device__ __forceinline__ void sum_partials(const float *src, int64_t stride, int n, float (&v)[4]) {
+  int k = 0;
+  for (; k + 8 <= n; k += 8) {
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = __ldcg(reinterpret_cast<const float4 *>(src + (k + u) * stride));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      v[0] += x[u].x;
+      v[1] += x[u].y;
+      v[2] += x[u].z;
+      v[3] += x[u].w;
+    }
+  }
+  for (; k < n; ++k) {
+    const float4 x = __ldcg(reinterpret_cast<const float4 *>(src + k * stride));
+    v[0] += x.x;
+    v[1] += x.y;
+    v[2] += x.z;
+    v[3] += x.w;
+  }
+}
+
+// The same for a dB accumulator: columns c and rb + c (the hi and lo planes'
+// products) summed.
+__device__ __forceinline__ void drain_row_pair(uint32_t taddr, int rb, bool have, bool valid, float *dst, int r4) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < r4; c0 += 16) {
+    float v[16], w[16];
+    if (have) {
+      tmem_load16(taddr + static_cast<uint32_t>(c0), v);
+      tmem_load16(taddr + static_cast<uint32_t>(rb + c0), w);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = w[j] = 0.f;
+    }
+    if (valid) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (c0 + 4 * g < r4) {
+          const float x[4] = {v[4 * g] + w[4 * g], v[4 * g + 1] + w[4 * g + 1], v[4 * g + 2] + w[4 * g + 2],
+                              v[4 * g + 3] + w[4 * g + 3]};
+          st_global_f4(dst + c0 + 4 * g, x);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -105,7 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bt0 = su0 + static_cast<uint32_t>(TT) * 4u * su_box;
   const uint32_t bar0 = bt0 + 2 * BT_BYTES;
   auto stage = [&](int s) { return base + static_cast<uint32_t>(s) * TILE_BYTES; };
-  auto su = [&](int i, int p, int h) { return su0 + static_cast<uint32_t>((i * 2 + p) * 2 + h) * su_box; };
+  // token tile i, 64-token half h: the hi box [RB j][64 t], the lo box right after it
+  auto su = [&](int i, int h) { return su0 + static_cast<uint32_t>(i * 2 + h) * 2u * su_box; };
   auto btile = [&](int b) { return bt0 + static_cast<uint32_t>(b) * BT_BYTES; };
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kDudbMaxStages + s); };
@@ -168,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < tt_n; ++i)
         for (int p = 0; p < 2; ++p)
           for (int h = 0; h < 2; ++h)
-            tma_load_2d(su(i, p, h), p ? &tm_su_lo : &tm_su_hi, su_full,
+            tma_load_2d(su(i, h) + p * su_box, p ? &tm_su_lo : &tm_su_hi, su_full,
                         static_cast<int32_t>(t_base + i * DT + h * 64), 0);                  // [RB j][64 t]
       int issued = 0, b_issued = 0;
       bool ok = true;
@@ -211,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issue ----------------
     if (lane == 0) {
       const uint32_t idesc_u = idesc_bf16_f32(DT, UB, false, true);
-      const uint32_t idesc_b = idesc_bf16_f32(DN, static_cast<uint32_t>(RB), true, false);
+      const uint32_t idesc_b = idesc_bf16_f32(DN, static_cast<uint32_t>(2 * RB), true, false);
       bool ok = mbar_wait(su_full, 0, a.status);
       int c = 0;
       for (; c < nn_n && ok; ++c) {
@@ -220,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t d_b = tmem + static_cast<uint32_t>(TT * UB + c * RB);
+        const uint32_t d_b = tmem + static_cast<uint32_t>(TT * UB + c * 2 * RB);
         for (int i = 0; i < tt_n; ++i) {
           const int st = c * tt_n + i;
           const int s = st % NS;
@@ -241,13 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             // dB: the tile MN-major (features in two 64-wide boxes, 16 tokens a
-            // step), the sU planes K-major
+            // step), the stacked hi | lo sU planes K-major (N = 2 RB)
             const uint64_t ad = smem_desc_sw128(stage(s) + kk * 2048, BOX_BYTES, 1024);
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-              const uint64_t bd = smem_desc_sw128(su(i, p, kk >> 2) + (kk & 3) * 32, 16, 1024);
-              tc_mma_ss(d_b, ad, bd, idesc_b, (i > 0 || kk > 0 || p > 0) ? 1u : 0u);
-            }
+            const uint64_t bd = smem_desc_sw128(su(i, kk >> 2) + (kk & 3) * 32, 16, 1024);
+            tc_mma_ss(d_b, ad, bd, idesc_b, (i > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(empty(s));
         }
@@ -275,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool have = __all_sync(0xffffffffu, okc && !s_abort);   // tcgen05.ld is warp-collective
       tc_fence_after();
       const int64_t n = n_base + static_cast<int64_t>(c) * DN + row;
-      drain_row(trow + static_cast<uint32_t>(TT * UB + c * RB), have, n < a.N,
-                a.part_b + (static_cast<int64_t>(tr) * a.N + n) * r4, r4);
+      drain_row_pair(trow + static_cast<uint32_t>(TT * UB + c * 2 * RB), RB, have, n < a.N,
+                     a.part_b + (static_cast<int64_t>(tr) * a.N + n) * r4, r4);
     }
     const bool oka = mbar_wait(acc_bar, 0, a.status);
     const bool have = __all_sync(0xffffffffu, oka && !s_abort);
@@ -313,15 +363,7 @@ __global__ void __launch_bounds__(256) dudb_finish_kernel(const DuDbArgs a) {
     if (i < nu) {
       const int64_t t = i / gu;
       const int c0 = static_cast<int>(i - t * gu) * 4;
-      if (c0 < r4) {
-        for (int k = 0; k < a.n_ranges; ++k) {
-          const float4 x = __ldcg(reinterpret_cast<const float4 *>(a.part_u + (static_cast<int64_t>(k) * a.T + t) * r4 + c0));
-          v[0] += x.x;
-          v[1] += x.y;
-          v[2] += x.z;
-          v[3] += x.w;
-        }
-      }
+      if (c0 < r4) sum_partials(a.part_u + t * r4 + c0, a.T * r4, a.n_ranges, v);
       uint16_t hi[4], lo[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -343,13 +385,7 @@ __global__ void __launch_bounds__(256) dudb_finish_kernel(const DuDbArgs a) {
       const int64_t j = i - nu;
       const int64_t n = j / gb;
       const int c0 = static_cast<int>(j - n * gb) * 4;
-      for (int k = 0; k < a.t_ranges; ++k) {
-        const float4 x = __ldcg(reinterpret_cast<const float4 *>(a.part_b + (static_cast<int64_t>(k) * a.N + n) * r4 + c0));
-        v[0] += x.x;
-        v[1] += x.y;
-        v[2] += x.z;
-        v[3] += x.w;
-      }
+      sum_partials(a.part_b + n * r4 + c0, a.N * r4, a.t_ranges, v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (c0 + e < a.R) {
@@ -374,7 +410,7 @@ bool dudb_geom(int64_t T, int64_t N, int r, int num_sms, DuDbGeom &g) {
     int stages = (kSmemBudget - kFixed - su_bytes(tt, rb)) / TILE_BYTES;
     if (stages > kDudbMaxStages) stages = kDudbMaxStages;
     if (stages < 2) continue;
-    int64_t nn_max = (512 - tt * UB) / rb;   // tensor-memory columns
+    int64_t nn_max = (512 - tt * UB) / (2 * rb);   // tensor-memory columns
     if (nn_max > kDudbMaxChunks) nn_max = kDudbMaxChunks;
     if (nn_max > n_chunks) nn_max = n_chunks;
     for (int64_t nn0 = 1; nn0 <= nn_max; ++nn0) {
@@ -396,7 +432,7 @@ bool dudb_geom(int64_t T, int64_t N, int r, int num_sms, DuDbGeom &g) {
       g.stages = stages;
       g.smem = stages * TILE_BYTES + su_bytes(tt, rb) + kFixed;
       int cols = 32;
-      while (cols < tt * UB + static_cast<int>(nn) * rb) cols *= 2;
+      while (cols < tt * UB + static_cast<int>(nn) * 2 * rb) cols *= 2;
       g.tmem_cols = cols;
     }
   }
@@ -421,7 +457,7 @@ cudaError_t launch_dudb(const DuDbArgs &a, const CUtensorMap &tm_dy, const CUten
   if (a.rb != (a.R <= 16 ? 16 : a.R <= 32 ? 32 : 64)) return cudaErrorInvalidValue;
   if (a.stages < 2 || a.stages > kDudbMaxStages || a.tt < 1 || a.nn < 1 || a.nn > kDudbMaxChunks)
     return cudaErrorInvalidValue;
-  if (a.tt * UB + a.nn * a.rb > a.tmem_cols || a.tmem_cols > 512) return cudaErrorInvalidValue;
+  if (a.tt * UB + a.nn * 2 * a.rb > a.tmem_cols || a.tmem_cols > 512) return cudaErrorInvalidValue;
   const int64_t t_tiles = (a.T + DT - 1) / DT, n_chunks = (a.N + DN - 1) / DN;
   // every CTA of the grid owns at least one tile and one chunk
   if (a.t_ranges != (t_tiles + a.tt - 1) / a.tt || a.n_ranges != (n_chunks + a.nn - 1) / a.nn)

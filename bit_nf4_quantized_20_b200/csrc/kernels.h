@@ -231,7 +231,8 @@ constexpr int kDudbMaxChunks = 32;
 struct DuDbGeom {
   int tt, nn;                  // 128-token tiles, 128-feature chunks per CTA
   int t_ranges, n_ranges;      // the grid: t_ranges x n_ranges CTAs
-  int rb;                      // dB accumulator columns: r rounded up to 16, 32 or 64
+  int rb;                      // r rounded up to 16, 32 or 64: the hi and lo sU planes stacked
+                               // make a 2 rb-column dB accumulator
   int stages;                  // dY tiles in flight (32 KiB each)
   int smem;                    // dynamic shared memory bytes
   int tmem_cols;               // tensor-memory columns allocated (a power of two)

@@ -252,11 +252,15 @@ QLORA_API qlora_status qlora_linear_fwd_save(const void *x, int64_t T, const qlo
 
 /*
  * qlora_linear_bwd that takes U from a preceding qlora_linear_fwd_save of the
- * same x, A, s and T instead of recomputing it from x: dU and dB then share one
- * grid (both stream dY), and x is read once (for dA).  Results equal
- * qlora_linear_bwd's within the rounding of the FP32 sums.  u_saved is read,
- * never written.  Errors: as qlora_linear_bwd; INVALID_ARG if u_saved is null
- * when T > 0, MISALIGNED if it is not 16-byte aligned.
+ * same x, A, s and T instead of recomputing it from x, so that x is read once
+ * (for dA).  dU and dB both contract dY: for r <= 64, one kernel reads each
+ * tile of dY once for both (block partial sums in the workspace, summed in a
+ * fixed order by the next launch), unless those partial sums would cost more
+ * than the second read of dY that they replace; otherwise dU and dB run as two
+ * launches side by side.  Results equal qlora_linear_bwd's within the rounding
+ * of the FP32 sums and do not depend on timing.  u_saved is read, never
+ * written.  Errors: as qlora_linear_bwd; INVALID_ARG if u_saved is null when
+ * T > 0, MISALIGNED if it is not 16-byte aligned.
  */
 QLORA_API qlora_status qlora_linear_bwd_saved(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,
                                               const void *A, const void *B, int32_t r, float s, const void *u_saved,

@@ -471,7 +471,7 @@ def _launched_kernels(fn):
 @pytest.mark.parametrize("T,N,K,r,s,one_read", [
     (2500, 3080, 256, 24, 0.5, True),   # blocks of 2 token tiles x 2 feature chunks; ragged T and N
     (3000, 4104, 128, 13, 2.0, True),   # 2 x 3 blocks, rank 13
-    (2500, 6144, 64, 36, 1.0, True),    # 64-column dB accumulators, three pipeline stages
+    (2500, 4104, 64, 36, 1.0, True),    # hi and lo planes of 64 rows each (N = 128), three stages
     (513, 4104, 192, 1, 1.0, True),     # rank 1; one token in the last tile
     (1300, 4104, 64, 8, 1.0, True),     # three token tiles a block
     (300, 384, 320, 24, 0.5, False),    # partial sums would outweigh the second read of dY
