@@ -854,15 +854,16 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
   SkinnyTcArgs aa = tc_args(K, T, r, 1.0f);
   aa.tr = static_cast<uint16_t *>(dA);
 
-  TcLaunch first, mid, second;
-  bool have_mid = false;
-  // saved path, r <= 64: dU and dB from one read of dY, then the sums of the
-  // blocks' partials
-  bool fused = false;
+  TcLaunch first, mid, second, ul;
+  bool have_mid = false, have_u = false;
+  // r <= 64: dU and dB from one read of dY, then the sums of the blocks'
+  // partials (without the saved planes, sU is computed first)
+  DuDbGeom gdd;
+  const bool fused = dudb_geom(T, N, r, kSplitSms, gdd);
   DuDbArgs fa;
   CUtensorMap fm_dy, fm_b, fm_su_hi, fm_su_lo;
   qlora_status rs;
-  if (!u_saved) {
+  if (!u_saved && !fused) {
     // one grid: sU = s X A^T, transposed, as hi + lo planes, with dU; then
     // dB with dA in a second grid
     const PairGeom g1 = geom_u_du(T, N, K, r);
@@ -879,11 +880,20 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
     const TcProduct ta = {K_LORA_DA, x, K, true, plane(L.duT_hi), plane(L.duT_lo), Tp, false, g2.g1};
     rs = prepare_pair_tc(K_LORA_DB_DA, tb, ab, ta, aa, g2, w8, L, second);
   } else {
-    DuDbGeom gdd;
-    if (dudb_geom(T, N, r, kSplitSms, gdd)) {
+    if (!u_saved) {
+      // sU = s X A^T as transposed hi + lo planes in the workspace, for dB
+      SkinnyTcArgs au = tc_args(T, K, r, s);
+      au.t_hi = plane(L.suT_hi);
+      au.t_lo = plane(L.suT_lo);
+      au.ldt = Tp;
+      const TcProduct tu = {K_LORA_U, x, K, false, A, nullptr, K, false, geom_u(T, K, r)};
+      rs = prepare_single_tc(tu, au, w8, L, ul);
+      if (rs != QLORA_OK) return rs;
+      have_u = true;
+    }
+    if (fused) {
       // dU and dB from one read of dY: block partial sums in the workspace,
       // then one launch sums them and writes dU's planes and dB
-      fused = true;
       memset(&fa, 0, sizeof(fa));
       fa.T = T;
       fa.N = N;
@@ -948,6 +958,10 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
     return QLORA_ERR_CUDA;
   if (fused) {
     const bool pdl = g_trace.recs == nullptr;
+    if (have_u) {
+      rs = launch_tc(ul, st);
+      if (rs != QLORA_OK) return rs;
+    }
     {
       TraceScope ts(K_LORA_DU_DB, 6.0 * T * N * r, 2.0 * T * N, st);
       if (launch_dudb(fa, fm_dy, fm_b, fm_su_hi, fm_su_lo, st, pdl) != cudaSuccess) return QLORA_ERR_CUDA;

@@ -220,8 +220,10 @@ QLORA_API qlora_status qlora_linear_fwd(const void *x, int64_t T, const qlora_nf
  * dy[T, N], x[T, K], A[r, K], B[N, r]; outputs dx[T, K], dA[r, K], dB[N, r]
  * (BF16, overwritten, not accumulated).  Same requirements as the forward.
  * ws: at least qlora_workspace_bytes(QLORA_OP_BWD, T, N, K, r) bytes.
- * Streams: all work is ordered on `stream`; the grid computing dB and dA
- * follows the dX GEMM and runs on the SMs its last round of tiles leaves idle.
+ * Streams: all work is ordered on `stream`.  For r <= 64, where it pays, U is
+ * computed first and dU and dB then share one read of dY (as in
+ * qlora_linear_bwd_saved); the launch computing dA (with dB otherwise) follows
+ * the dX GEMM and runs on the SMs its last round of tiles leaves idle.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.
  */
 QLORA_API qlora_status qlora_linear_bwd(const void *dy, const void *x, int64_t T, const qlora_nf4_weight *qw,

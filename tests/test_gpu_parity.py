@@ -478,29 +478,34 @@ def _launched_kernels(fn):
     (257, 1024, 128, 65, 1.0, False),   # rank above 64
 ])
 def test_layer_saved_u_one_read_of_dy(T, N, K, r, s, one_read):
-    """The saved-U backward with dU and dB from one read of dY (block partial
-    sums, then a launch that sums them), against the oracle; shapes where the
-    partial sums do not pay off, or the rank is above 64, run dU and dB as two
-    launches instead."""
+    """Both backwards with dU and dB from one read of dY (block partial sums,
+    then a launch that sums them), against the oracle: the saved-U one, and
+    the plain one, which first computes sU.  Shapes where the partial sums do
+    not pay off, or the rank is above 64, run dU and dB as two launches (saved)
+    or in the two paired grids (plain) instead."""
     q = Q()
     W, X, A, B, dY = inputs.layer_inputs(93, 0, 0, T, N, K, r, device="cuda")
     qw, (codes, scales, c2) = quantize_and_check(W)
     y, u = q.linear_fwd_save(X, qw, A, B, s)
     names = _launched_kernels(lambda: q.linear_bwd_saved(dY, X, qw, A, B, s, u))
+    plain = _launched_kernels(lambda: q.linear_bwd(dY, X, qw, A, B, s))
     torch.cuda.synchronize()
     if one_read:
         assert "lora_du+dB" in names and "lora_du+dB_sum" in names and "lora_dB" not in names, names
+        assert plain[:3] == ["lora_u", "lora_du+dB", "lora_du+dB_sum"] and "lora_u+du" not in plain, plain
     else:
         assert "lora_du+dB" not in names and "lora_dB" in names and "lora_du" in names, names
-    dx, dA, dB = q.linear_bwd_saved(dY, X, qw, A, B, s, u)
-    q.get_error()
-    torch.cuda.synchronize()
+        assert "lora_u+du" in plain and "lora_du+dB" not in plain, plain
     wd = O.dequantize_nf4(codes, scales, c2, N, K)
     xb, ab, bb, dyb = bits(X), bits(A), bits(B), bits(dY)
     rdx, rdA, rdB = O.linear_bwd(dyb, xb, wd, ab, bb, s)
-    assert_close("dX", dx, rdx)
-    assert_close("dA", dA, rdA)
-    assert_close("dB", dB, rdB)
+    for bwd in (lambda: q.linear_bwd_saved(dY, X, qw, A, B, s, u), lambda: q.linear_bwd(dY, X, qw, A, B, s)):
+        dx, dA, dB = bwd()
+        q.get_error()
+        torch.cuda.synchronize()
+        assert_close("dX", dx, rdx)
+        assert_close("dA", dA, rdA)
+        assert_close("dB", dB, rdB)
 
 
 def test_backward_saved_graph_capture_matches_eager():
