@@ -92,6 +92,15 @@ def test_workspace_bytes(L):
     assert L.qlora_workspace_bytes(2, 0, 4096, 4096, 16) > 0
     # grows with the token count
     assert L.qlora_workspace_bytes(2, 8192, 4096, 4096, 16) > b
+    # the backward of the 8B gate shape: status header (256) and tile
+    # counters (64 KiB), sU^T and dU^T (two planes each, 16 x 4096 BF16), dU's
+    # hi | lo row planes (4096 x 128 BF16), B padded to 64 columns (14336 x 64
+    # BF16), and the largest partial-sum buffer, here the fused dU/dB kernel's:
+    # 3 x 9-tile blocks give 13 feature ranges and 11 token ranges of FP32 rows
+    # of 16, 13 * 4096 * 64 + 11 * 14336 * 64 bytes
+    parts = 13 * 4096 * 64 + 11 * 14336 * 64
+    fixed = 256 + 65536 + 4 * 16 * 4096 * 2 + 4096 * 128 * 2 + 14336 * 64 * 2
+    assert L.qlora_workspace_bytes(2, 4096, 14336, 4096, 16) == fixed + parts
 
 
 def test_decode_workspace_fits_the_noalloc_scratch(L):
