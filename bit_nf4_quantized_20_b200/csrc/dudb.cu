@@ -15,9 +15,9 @@
 // columns past r read as zeros), dB for each feature chunk (the hi and lo
 // planes of sU, r rounded up to rb = 16, 32 or 64 rows each, stacked into one
 // N = 2 rb operand: one MMA per step, the two halves of the accumulator summed
-// when it is drained).  The sU planes of the block's tokens are loaded once, B's rows
-// of a feature chunk once per chunk (two buffers); the loop runs over feature
-// chunks, and over the block's token tiles inside each chunk.
+// when it is drained).  The sU planes of the block's tokens are loaded once,
+// B's rows of a feature chunk once per chunk (two buffers); the loop runs over
+// feature chunks, and over the block's token tiles inside each chunk.
 //
 // The block's dU rows are partial sums over its features and its dB rows over
 // its tokens: both go to the workspace in FP32 -- each chunk's dB rows as soon
