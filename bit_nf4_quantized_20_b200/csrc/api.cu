@@ -946,10 +946,11 @@ static qlora_status linear_bwd_impl(const void *dy, const void *x, int64_t T, co
   GemmLaunch gl;
   rs = prepare_gemm(1, qw, dy, plane(L.du_row), r64, A, r, dx, T, reinterpret_cast<uint32_t *>(ws), gl);
   if (rs != QLORA_OK) return rs;
-  // The second grid needs only the first's planes, not dX: it follows the dX
-  // GEMM as a programmatic dependent that waits for the GEMM only before it
-  // exits, so that it runs on the SMs the GEMM's last round of tiles leaves
-  // idle.  (The GEMM lets it start after the first grid has completed.)
+  // The last launch (dA, or dB with dA) needs only dU's planes and the
+  // inputs, not dX: it follows the dX GEMM as a programmatic dependent that
+  // waits for the GEMM only before it exits, so that it runs on the SMs the
+  // GEMM's last round of tiles leaves idle.  (The GEMM lets it start after
+  // the launch before the GEMM, which wrote those planes, has completed.)
   second.a0.dep_late = 1;
   second.a1.dep_late = 1;
 
