@@ -256,8 +256,6 @@ PairGeom pair_geom(int64_t M0, int64_t C0, bool q0, int nq0, int64_t M1, int64_t
 // U [T, r] with dU [T, r]; dB [N, r] with dA [r, K] (written as [K, r] products)
 PairGeom geom_u_du(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(T, K, false, 1, T, N, true, 1, r); }
 PairGeom geom_db_da(int64_t T, int64_t N, int64_t K, int r) { return pair_geom(N, T, false, 2, K, T, false, 2, r); }
-// with U saved by the forward: dU with dB (both stream dY), then dA alone
-PairGeom geom_du_db(int64_t T, int64_t N, int r) { return pair_geom(T, N, true, 1, N, T, false, 2, r); }
 SkinnyTcGeom geom_da(int64_t T, int64_t K, int r) { return skinny_tc_geom(K, T, r, 2, false, kSplitSms); }
 size_t pair_partials(const PairGeom &pg) {
   return static_cast<size_t>(round_up(static_cast<int64_t>(pg.part0), 256)) + pg.part1;
@@ -290,9 +288,11 @@ WsLayout ws_layout(int op, int64_t T, int64_t N, int64_t K, int r) {
     L.duT_hi = off; off += t_plane;
     L.duT_lo = off; off += t_plane;
     L.bpad = off; off += static_cast<size_t>(round_up(N * r64 * 2, 256));
+    // the paired grids of the plain backward, dA, and the fused dU/dB kernel
+    // (the saved backward's two-launch dU and dB reduce in clusters: no partials)
     DuDbGeom gdd;
-    const size_t p[5] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r)),
-                         pair_partials(geom_du_db(T, N, r)), skinny_tc_partials_bytes(geom_da(T, K, r), K, r),
+    const size_t p[4] = {pair_partials(geom_u_du(T, N, K, r)), pair_partials(geom_db_da(T, N, K, r)),
+                         skinny_tc_partials_bytes(geom_da(T, K, r), K, r),
                          dudb_geom(T, N, r, kSplitSms, gdd) ? dudb_partials_bytes(gdd, T, N, r) : 0};
     for (size_t v : p) part = v > part ? v : part;
   }
