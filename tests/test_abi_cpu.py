@@ -213,6 +213,12 @@ def test_trace_attach_validation(L):
     assert L.qlora_trace_attach(recs, 4, C.byref(cnt)) == 0
     assert L.qlora_trace_attach(None, 0, None) == 0
     assert L.qlora_kernel_name(6) == b"nf4_gemm_fwd"
+    # the fused dU/dB kernel and the launch that sums its partials (the names
+    # the bench's per-kernel map and the kernel-choice tests read)
+    assert L.qlora_kernel_name(12) == b"lora_du+dB"
+    assert L.qlora_kernel_name(14) == b"lora_du+dB_sum"
+    assert L.qlora_kernel_name(15) == b"unknown"
+    assert L.qlora_kernel_name(-1) == b"unknown"
     assert L.qlora_kernel_name(99) == b"unknown"
 
 
